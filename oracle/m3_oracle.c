@@ -1,0 +1,529 @@
+/*
+ * m3_oracle.c -- fp64 CPU oracle for the Mamba-3 selective scan.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the slow, obviously-correct
+ * definition that the CUDA library is checked against.  Only the tests,
+ * the package's smoke check and the benchmark's CPU-baseline leg may load
+ * it.  It shares no code, header, table or helper with the CUDA path.
+ *
+ * Sources (the pages this restates, by title and section):
+ *   [dotLLM]  "Mamba-3 (real algorithm) kernel-level PoC" pull request,
+ *             sections "Stage A" (Discretize, QkNorm, DataRoPE, MimoProject,
+ *             SelectiveScan -- trapezoidal scan, Eq. 9, with a prev_Bx second
+ *             state), "Key findings" (lambda and theta are per token; BC-bias
+ *             after QkNorm, before RoPE), the streaming-decode comment
+ *             (shifted_gamma[t] = DT[t+1](1-trap[t+1]), scale = gamma +
+ *             shifted_gamma; boundary fold DT[0](1-trap[0]) applied before the
+ *             scan's alpha) and "Mamba-3 MIMO streaming decode" (state is
+ *             rank-summed; cum_angle is rank-free).
+ *   [torchmamba] "TorchMamba" README, sections "Models" (3-term trap
+ *             h = a h + b B_{-1} x_{-1} + g B x; MIMO = rank-R update on a
+ *             shared (N,P) state), "Math notes" (Prop. 1 Eqs. 5-6, Eq. 7
+ *             L = 1SS @ band, Props. 2-4 data-dependent pairwise rotations,
+ *             App. C per-head expand/contract vectors) and "Behavioral notes"
+ *             (RoPE needs even N; states never below fp32).
+ *
+ * Readings where the pages are silent (each is listed in the design notes):
+ *   alpha_t = exp(dt_t A_h), beta_t = (1-lam_t) dt_t alpha_t,
+ *   gamma_t = lam_t dt_t;  per-step angle dt_t * theta_t;  adjacent pairs
+ *   (2i, 2i+1) rotated by +Phi;  all N/2 pairs rotate;  h0 = prev_Bx0 = 0 and
+ *   Phi0 = 0 unless given;  MIMO expand/contract vectors W_x, W_y of shape
+ *   (H,R,P);  QkNorm gain of shape (N), bias of shape (H,R,N).
+ *
+ * Layouts (row-major, last index fastest):
+ *   x, y (Bt,T,H,P); dt, lam (Bt,T,H); A, D (H); theta (Bt,T,H,N/2);
+ *   B, C (Bt,T,H,R,N) with R = 1 for SISO; W_x, W_y (H,R,P);
+ *   h, prev_Bx (Bt,H,N,P); angle (Bt,H,N/2).
+ *
+ * Every function returns 0 on success, -1 on a bad argument.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+typedef struct {
+    long batch, seqlen, nheads, headdim, dstate, rank;
+} m3o_dims;
+
+typedef struct {
+    const double *normw_B, *normw_C; /* (N) or NULL: QkNorm off          */
+    const double *bias_B, *bias_C;   /* (H,R,N) or NULL: bias off         */
+    double eps;                      /* RMSNorm epsilon                   */
+} m3o_bcnorm;
+
+/* ------------------------------------------------------------------------ */
+/* S1: trapezoidal discretization (dotLLM "Stage A: Mamba3Discretize";      */
+/* torchmamba "Math notes", Prop. 1).                                        */
+/* ------------------------------------------------------------------------ */
+int m3o_discretize(const double *dt, const double *A, const double *lam,
+                   long Bt, long T, long H,
+                   double *alpha, double *beta, double *gamma)
+{
+    if (!dt || !A || !lam || !alpha || !beta || !gamma) return -1;
+    for (long b = 0; b < Bt; b++)
+        for (long t = 0; t < T; t++)
+            for (long h = 0; h < H; h++) {
+                long i = (b * T + t) * H + h;
+                double a = exp(dt[i] * A[h]);
+                alpha[i] = a;
+                beta[i] = (1.0 - lam[i]) * dt[i] * a;
+                gamma[i] = lam[i] * dt[i];
+            }
+    return 0;
+}
+
+/* QkNorm (RMSNorm over N, gain w) then per-head bias; dotLLM "Key findings":
+ * the bias is added after the norm and before the rotation. */
+static void bc_prepare(const double *src, long N, const double *w,
+                       const double *bias, double eps, double *dst)
+{
+    if (w) {
+        double ss = 0.0;
+        for (long n = 0; n < N; n++) ss += src[n] * src[n];
+        double inv = 1.0 / sqrt(ss / (double)N + eps);
+        for (long n = 0; n < N; n++) dst[n] = src[n] * inv * w[n];
+    } else {
+        for (long n = 0; n < N; n++) dst[n] = src[n];
+    }
+    if (bias)
+        for (long n = 0; n < N; n++) dst[n] += bias[n];
+}
+
+/* Rotate adjacent pairs (2i, 2i+1) of v by the angles phi[i]. */
+static void rotate_pairs(const double *v, const double *phi, long N, double *out)
+{
+    for (long i = 0; i < N / 2; i++) {
+        double c = cos(phi[i]), s = sin(phi[i]);
+        double v0 = v[2 * i], v1 = v[2 * i + 1];
+        out[2 * i] = c * v0 - s * v1;
+        out[2 * i + 1] = s * v0 + c * v1;
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* S2: QkNorm + BC-bias + data-dependent RoPE (dotLLM "Stage A:             */
+/* Mamba3QkNorm / Mamba3DataRoPE"; torchmamba "Math notes", Props. 2-4).    */
+/* Phi_t = Phi_{t-1} + dt_t * theta_t (per pair), B_rot = R(Phi_t) B.        */
+/* ------------------------------------------------------------------------ */
+int m3o_rope_bc(const double *B, const double *C, const double *theta,
+                const double *dt, const double *angle0, const m3o_bcnorm *nrm,
+                m3o_dims d, double *B_rot, double *C_rot, double *angle_final)
+{
+    long Bt = d.batch, T = d.seqlen, H = d.nheads, N = d.dstate;
+    long R = d.rank < 1 ? 1 : d.rank;
+    if (!B || !C || !theta || !dt || !B_rot || !C_rot) return -1;
+    if (N <= 0 || (N & 1)) return -1;
+    double *phi = (double *)malloc(sizeof(double) * (N / 2));
+    double *tmp = (double *)malloc(sizeof(double) * N);
+    for (long b = 0; b < Bt; b++)
+        for (long h = 0; h < H; h++) {
+            for (long i = 0; i < N / 2; i++)
+                phi[i] = angle0 ? angle0[(b * H + h) * (N / 2) + i] : 0.0;
+            for (long t = 0; t < T; t++) {
+                long bth = (b * T + t) * H + h;
+                for (long i = 0; i < N / 2; i++)
+                    phi[i] += dt[bth] * theta[bth * (N / 2) + i];
+                for (long r = 0; r < R; r++) {
+                    long off = (bth * R + r) * N;
+                    const double *bb = nrm && nrm->bias_B ? nrm->bias_B + (h * R + r) * N : NULL;
+                    const double *cb = nrm && nrm->bias_C ? nrm->bias_C + (h * R + r) * N : NULL;
+                    bc_prepare(B + off, N, nrm ? nrm->normw_B : NULL, bb, nrm ? nrm->eps : 0.0, tmp);
+                    rotate_pairs(tmp, phi, N, B_rot + off);
+                    bc_prepare(C + off, N, nrm ? nrm->normw_C : NULL, cb, nrm ? nrm->eps : 0.0, tmp);
+                    rotate_pairs(tmp, phi, N, C_rot + off);
+                }
+            }
+            if (angle_final)
+                for (long i = 0; i < N / 2; i++)
+                    angle_final[(b * H + h) * (N / 2) + i] = phi[i];
+        }
+    free(phi);
+    free(tmp);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Lane workers.  The (b,h) lanes are independent; each worker walks its    */
+/* lanes in order and each lane sequentially over t.                         */
+/* ------------------------------------------------------------------------ */
+typedef struct {
+    const double *x, *dt, *A, *lam, *theta, *B, *C, *D, *Wx, *Wy;
+    const m3o_bcnorm *nrm;
+    const double *h0, *prevBx0, *angle0;
+    m3o_dims d;
+    double *y, *h_out, *prevBx_out, *angle_out;
+    long chunk;       /* only for the chunked self-test variant */
+    long lane_begin, lane_end;
+    int kind;         /* 0 = SISO loop, 1 = MIMO loop, 2 = SISO chunked */
+} lane_job;
+
+/* SISO recurrence for one lane (dotLLM "Mamba3SelectiveScan", Eq. 9):
+ *   U_t   = B_rot_t x_t^T                      (N x P)
+ *   h_t   = alpha_t h_{t-1} + beta_t U_{t-1} + gamma_t U_t
+ *   y_t   = C_rot_t^T h_t + D_h x_t
+ * with h_{-1} = h0 and U_{-1} = prev_Bx0. */
+static void siso_lane(const lane_job *J, long b, long h)
+{
+    long T = J->d.seqlen, H = J->d.nheads, P = J->d.headdim, N = J->d.dstate;
+    long NP = N * P;
+    double *hs = (double *)malloc(sizeof(double) * NP);
+    double *Up = (double *)malloc(sizeof(double) * NP);
+    double *phi = (double *)malloc(sizeof(double) * (N / 2));
+    double *tmp = (double *)malloc(sizeof(double) * N);
+    double *Bb = (double *)malloc(sizeof(double) * N);
+    double *Cb = (double *)malloc(sizeof(double) * N);
+    long lane = b * H + h;
+    for (long k = 0; k < NP; k++) {
+        hs[k] = J->h0 ? J->h0[lane * NP + k] : 0.0;
+        Up[k] = J->prevBx0 ? J->prevBx0[lane * NP + k] : 0.0;
+    }
+    for (long i = 0; i < N / 2; i++)
+        phi[i] = J->angle0 ? J->angle0[lane * (N / 2) + i] : 0.0;
+    const m3o_bcnorm *nr = J->nrm;
+    for (long t = 0; t < T; t++) {
+        long bth = (b * T + t) * H + h;
+        double dl = J->dt[bth], lm = J->lam[bth];
+        double al = exp(dl * J->A[h]);
+        double be = (1.0 - lm) * dl * al;
+        double ga = lm * dl;
+        for (long i = 0; i < N / 2; i++) phi[i] += dl * J->theta[bth * (N / 2) + i];
+        bc_prepare(J->B + bth * N, N, nr ? nr->normw_B : NULL,
+                   nr && nr->bias_B ? nr->bias_B + h * N : NULL, nr ? nr->eps : 0.0, tmp);
+        rotate_pairs(tmp, phi, N, Bb);
+        bc_prepare(J->C + bth * N, N, nr ? nr->normw_C : NULL,
+                   nr && nr->bias_C ? nr->bias_C + h * N : NULL, nr ? nr->eps : 0.0, tmp);
+        rotate_pairs(tmp, phi, N, Cb);
+        const double *xt = J->x + bth * P;
+        for (long n = 0; n < N; n++)
+            for (long p = 0; p < P; p++) {
+                double u = Bb[n] * xt[p];
+                hs[n * P + p] = al * hs[n * P + p] + be * Up[n * P + p] + ga * u;
+                Up[n * P + p] = u;
+            }
+        double *yt = J->y + bth * P;
+        for (long p = 0; p < P; p++) {
+            double acc = 0.0;
+            for (long n = 0; n < N; n++) acc += Cb[n] * hs[n * P + p];
+            yt[p] = acc + J->D[h] * xt[p];
+        }
+    }
+    if (J->h_out) memcpy(J->h_out + lane * NP, hs, sizeof(double) * NP);
+    if (J->prevBx_out) memcpy(J->prevBx_out + lane * NP, Up, sizeof(double) * NP);
+    if (J->angle_out) memcpy(J->angle_out + lane * (N / 2), phi, sizeof(double) * (N / 2));
+    free(hs); free(Up); free(phi); free(tmp); free(Bb); free(Cb);
+}
+
+/* MIMO recurrence for one lane (torchmamba "Models": rank-R update on a
+ * shared (N,P) state; "Math notes" App. C: per-head x/y expand by learned
+ * vectors; dotLLM "MIMO streaming decode": state rank-summed, angle
+ * rank-free):
+ *   X_{t,r}[p] = W_x[h,r,p] x_t[p]
+ *   U_t        = sum_r B_rot_{t,r} X_{t,r}^T
+ *   h_t        = alpha_t h_{t-1} + beta_t U_{t-1} + gamma_t U_t
+ *   y_t[p]     = sum_r W_y[h,r,p] (C_rot_{t,r}^T h_t)[p] + D_h x_t[p]
+ * NULL W_x / W_y mean all ones. */
+static void mimo_lane(const lane_job *J, long b, long h)
+{
+    long T = J->d.seqlen, H = J->d.nheads, P = J->d.headdim, N = J->d.dstate;
+    long R = J->d.rank;
+    long NP = N * P;
+    double *hs = (double *)malloc(sizeof(double) * NP);
+    double *Up = (double *)malloc(sizeof(double) * NP);
+    double *Ut = (double *)malloc(sizeof(double) * NP);
+    double *phi = (double *)malloc(sizeof(double) * (N / 2));
+    double *tmp = (double *)malloc(sizeof(double) * N);
+    double *Bb = (double *)malloc(sizeof(double) * R * N);
+    double *Cb = (double *)malloc(sizeof(double) * R * N);
+    double *Xr = (double *)malloc(sizeof(double) * R * P);
+    long lane = b * H + h;
+    for (long k = 0; k < NP; k++) {
+        hs[k] = J->h0 ? J->h0[lane * NP + k] : 0.0;
+        Up[k] = J->prevBx0 ? J->prevBx0[lane * NP + k] : 0.0;
+    }
+    for (long i = 0; i < N / 2; i++)
+        phi[i] = J->angle0 ? J->angle0[lane * (N / 2) + i] : 0.0;
+    const m3o_bcnorm *nr = J->nrm;
+    for (long t = 0; t < T; t++) {
+        long bth = (b * T + t) * H + h;
+        double dl = J->dt[bth], lm = J->lam[bth];
+        double al = exp(dl * J->A[h]);
+        double be = (1.0 - lm) * dl * al;
+        double ga = lm * dl;
+        for (long i = 0; i < N / 2; i++) phi[i] += dl * J->theta[bth * (N / 2) + i];
+        const double *xt = J->x + bth * P;
+        for (long r = 0; r < R; r++) {
+            long off = (bth * R + r) * N;
+            bc_prepare(J->B + off, N, nr ? nr->normw_B : NULL,
+                       nr && nr->bias_B ? nr->bias_B + (h * R + r) * N : NULL, nr ? nr->eps : 0.0, tmp);
+            rotate_pairs(tmp, phi, N, Bb + r * N);
+            bc_prepare(J->C + off, N, nr ? nr->normw_C : NULL,
+                       nr && nr->bias_C ? nr->bias_C + (h * R + r) * N : NULL, nr ? nr->eps : 0.0, tmp);
+            rotate_pairs(tmp, phi, N, Cb + r * N);
+            for (long p = 0; p < P; p++)
+                Xr[r * P + p] = (J->Wx ? J->Wx[(h * R + r) * P + p] : 1.0) * xt[p];
+        }
+        for (long n = 0; n < N; n++)
+            for (long p = 0; p < P; p++) {
+                double u = 0.0;
+                for (long r = 0; r < R; r++) u += Bb[r * N + n] * Xr[r * P + p];
+                Ut[n * P + p] = u;
+            }
+        for (long k = 0; k < NP; k++) {
+            hs[k] = al * hs[k] + be * Up[k] + ga * Ut[k];
+            Up[k] = Ut[k];
+        }
+        double *yt = J->y + bth * P;
+        for (long p = 0; p < P; p++) {
+            double acc = 0.0;
+            for (long r = 0; r < R; r++) {
+                double yr = 0.0;
+                for (long n = 0; n < N; n++) yr += Cb[r * N + n] * hs[n * P + p];
+                acc += (J->Wy ? J->Wy[(h * R + r) * P + p] : 1.0) * yr;
+            }
+            yt[p] = acc + J->D[h] * xt[p];
+        }
+    }
+    if (J->h_out) memcpy(J->h_out + lane * NP, hs, sizeof(double) * NP);
+    if (J->prevBx_out) memcpy(J->prevBx_out + lane * NP, Up, sizeof(double) * NP);
+    if (J->angle_out) memcpy(J->angle_out + lane * (N / 2), phi, sizeof(double) * (N / 2));
+    free(hs); free(Up); free(Ut); free(phi); free(tmp); free(Bb); free(Cb); free(Xr);
+}
+
+/* Chunked form of the SISO scan, fp64, used only to self-test the
+ * shifted-gamma fold (dotLLM streaming-decode comment: shifted_gamma[t] =
+ * DT[t+1](1-trap[t+1]), scale = gamma + shifted_gamma, boundary fold
+ * DT[0](1-trap[0]) before the scan's alpha; torchmamba "Math notes": Mamba-2
+ * chunkwise intra-chunk quadratic part plus a factored inter-chunk carry).
+ *   g_t = h_t + sg_t U_t  with  sg_t = (1-lam_{t+1}) dt_{t+1}  (0 at t=T-1)
+ *   g_t = alpha_t g_{t-1} + w_t U_t,   w_t = gamma_t + sg_t
+ *   g_{-1} = h0 + (1-lam_0) dt_0 prev_Bx0
+ * Inside a chunk [t0, t1), with cum_t = sum_{k=t0..t} log alpha_k:
+ *   y_t  = e^{cum_t} C_t^T g_in + sum_{s<=t} M[t,s] (C_t.B_s) x_s + D x_t
+ *   M[t,s] = e^{cum_t - cum_s} w_s (s < t),  gamma_t (s == t)
+ *   g_out = e^{cum_end} g_in + sum_s e^{cum_end - cum_s} w_s B_s x_s^T
+ * At the end h_final = g_{T-1} and prev_Bx = B_{T-1} x_{T-1}^T. */
+static void siso_chunked_lane(const lane_job *J, long b, long h)
+{
+    long T = J->d.seqlen, H = J->d.nheads, P = J->d.headdim, N = J->d.dstate;
+    long Q = J->chunk;
+    long NP = N * P;
+    long lane = b * H + h;
+    const m3o_bcnorm *nr = J->nrm;
+    double *Bb = (double *)malloc(sizeof(double) * T * N);
+    double *Cb = (double *)malloc(sizeof(double) * T * N);
+    double *phi = (double *)malloc(sizeof(double) * (N / 2));
+    double *tmp = (double *)malloc(sizeof(double) * N);
+    double *la = (double *)malloc(sizeof(double) * T);   /* log alpha */
+    double *ga = (double *)malloc(sizeof(double) * T);
+    double *w = (double *)malloc(sizeof(double) * T);
+    double *g = (double *)malloc(sizeof(double) * NP);
+    double *gn = (double *)malloc(sizeof(double) * NP);
+    double *cum = (double *)malloc(sizeof(double) * Q);
+    for (long i = 0; i < N / 2; i++)
+        phi[i] = J->angle0 ? J->angle0[lane * (N / 2) + i] : 0.0;
+    for (long t = 0; t < T; t++) {
+        long bth = (b * T + t) * H + h;
+        double dl = J->dt[bth];
+        for (long i = 0; i < N / 2; i++) phi[i] += dl * J->theta[bth * (N / 2) + i];
+        bc_prepare(J->B + bth * N, N, nr ? nr->normw_B : NULL,
+                   nr && nr->bias_B ? nr->bias_B + h * N : NULL, nr ? nr->eps : 0.0, tmp);
+        rotate_pairs(tmp, phi, N, Bb + t * N);
+        bc_prepare(J->C + bth * N, N, nr ? nr->normw_C : NULL,
+                   nr && nr->bias_C ? nr->bias_C + h * N : NULL, nr ? nr->eps : 0.0, tmp);
+        rotate_pairs(tmp, phi, N, Cb + t * N);
+        la[t] = dl * J->A[h];
+        ga[t] = J->lam[bth] * dl;
+    }
+    for (long t = 0; t < T; t++) {
+        double sg = 0.0;
+        if (t + 1 < T) {
+            long nx = (b * T + t + 1) * H + h;
+            sg = (1.0 - J->lam[nx]) * J->dt[nx];
+        }
+        w[t] = ga[t] + sg;
+    }
+    {
+        long b0 = (b * T + 0) * H + h;
+        double f = T > 0 ? (1.0 - J->lam[b0]) * J->dt[b0] : 0.0;
+        for (long k = 0; k < NP; k++)
+            g[k] = (J->h0 ? J->h0[lane * NP + k] : 0.0) +
+                   f * (J->prevBx0 ? J->prevBx0[lane * NP + k] : 0.0);
+    }
+    for (long t0 = 0; t0 < T; t0 += Q) {
+        long t1 = t0 + Q < T ? t0 + Q : T;
+        double run = 0.0;
+        for (long t = t0; t < t1; t++) { run += la[t]; cum[t - t0] = run; }
+        double cend = cum[t1 - 1 - t0];
+        for (long t = t0; t < t1; t++) {
+            long bth = (b * T + t) * H + h;
+            double et = exp(cum[t - t0]);
+            for (long p = 0; p < P; p++) {
+                double acc = 0.0;
+                for (long n = 0; n < N; n++) acc += Cb[t * N + n] * g[n * P + p];
+                acc *= et;
+                for (long s = t0; s <= t; s++) {
+                    double cb = 0.0;
+                    for (long n = 0; n < N; n++) cb += Cb[t * N + n] * Bb[s * N + n];
+                    double m = (s == t) ? ga[t] : exp(cum[t - t0] - cum[s - t0]) * w[s];
+                    acc += m * cb * J->x[((b * T + s) * H + h) * P + p];
+                }
+                J->y[bth * P + p] = acc + J->D[h] * J->x[bth * P + p];
+            }
+        }
+        double ee = exp(cend);
+        for (long n = 0; n < N; n++)
+            for (long p = 0; p < P; p++) {
+                double acc = ee * g[n * P + p];
+                for (long s = t0; s < t1; s++)
+                    acc += exp(cend - cum[s - t0]) * w[s] * Bb[s * N + n] *
+                           J->x[((b * T + s) * H + h) * P + p];
+                gn[n * P + p] = acc;
+            }
+        memcpy(g, gn, sizeof(double) * NP);
+    }
+    if (J->h_out) memcpy(J->h_out + lane * NP, g, sizeof(double) * NP);
+    if (J->prevBx_out) {
+        for (long n = 0; n < N; n++)
+            for (long p = 0; p < P; p++)
+                J->prevBx_out[lane * NP + n * P + p] =
+                    T > 0 ? Bb[(T - 1) * N + n] * J->x[((b * T + T - 1) * H + h) * P + p]
+                          : (J->prevBx0 ? J->prevBx0[lane * NP + n * P + p] : 0.0);
+    }
+    if (J->angle_out) memcpy(J->angle_out + lane * (N / 2), phi, sizeof(double) * (N / 2));
+    free(Bb); free(Cb); free(phi); free(tmp); free(la); free(ga); free(w);
+    free(g); free(gn); free(cum);
+}
+
+static void *lane_worker(void *arg)
+{
+    lane_job *J = (lane_job *)arg;
+    long H = J->d.nheads;
+    for (long lane = J->lane_begin; lane < J->lane_end; lane++) {
+        long b = lane / H, h = lane % H;
+        if (J->kind == 0) siso_lane(J, b, h);
+        else if (J->kind == 1) mimo_lane(J, b, h);
+        else siso_chunked_lane(J, b, h);
+    }
+    return NULL;
+}
+
+static int run_lanes(lane_job *proto, int nthreads)
+{
+    long lanes = proto->d.batch * proto->d.nheads;
+    if (lanes <= 0) return 0;
+    if (nthreads <= 0) {
+        long nc = sysconf(_SC_NPROCESSORS_ONLN);
+        nthreads = nc > 0 ? (int)nc : 1;
+    }
+    if (nthreads > lanes) nthreads = (int)lanes;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * nthreads);
+    lane_job *jobs = (lane_job *)malloc(sizeof(lane_job) * nthreads);
+    for (int i = 0; i < nthreads; i++) {
+        jobs[i] = *proto;
+        jobs[i].lane_begin = lanes * i / nthreads;
+        jobs[i].lane_end = lanes * (i + 1) / nthreads;
+    }
+    for (int i = 1; i < nthreads; i++) pthread_create(&th[i], NULL, lane_worker, &jobs[i]);
+    lane_worker(&jobs[0]);
+    for (int i = 1; i < nthreads; i++) pthread_join(th[i], NULL);
+    free(th);
+    free(jobs);
+    return nthreads;
+}
+
+static int check_dims(m3o_dims d, int mimo)
+{
+    if (d.batch < 0 || d.seqlen < 0 || d.nheads <= 0 || d.headdim <= 0) return -1;
+    if (d.dstate <= 0 || (d.dstate & 1)) return -1;  /* RoPE needs even N */
+    if (mimo && d.rank < 1) return -1;
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Public oracle entry points.  Each returns the number of threads used     */
+/* (>= 1), 0 when there is no lane to run, or -1 on a bad argument.         */
+/* ------------------------------------------------------------------------ */
+int m3o_siso_loop(const double *x, const double *dt, const double *A,
+                  const double *lam, const double *theta, const double *B,
+                  const double *C, const double *D, const m3o_bcnorm *nrm,
+                  const double *h0, const double *prevBx0, const double *angle0,
+                  m3o_dims d, double *y, double *h_out, double *prevBx_out,
+                  double *angle_out, int nthreads)
+{
+    if (check_dims(d, 0)) return -1;
+    if (!x || !dt || !A || !lam || !theta || !B || !C || !D || !y) return -1;
+    lane_job J;
+    memset(&J, 0, sizeof J);
+    J.x = x; J.dt = dt; J.A = A; J.lam = lam; J.theta = theta; J.B = B; J.C = C;
+    J.D = D; J.nrm = nrm; J.h0 = h0; J.prevBx0 = prevBx0; J.angle0 = angle0;
+    J.d = d; J.d.rank = 1; J.y = y; J.h_out = h_out; J.prevBx_out = prevBx_out;
+    J.angle_out = angle_out; J.kind = 0;
+    return run_lanes(&J, nthreads);
+}
+
+int m3o_mimo_loop(const double *x, const double *dt, const double *A,
+                  const double *lam, const double *theta, const double *B,
+                  const double *C, const double *D, const double *Wx,
+                  const double *Wy, const m3o_bcnorm *nrm, const double *h0,
+                  const double *prevBx0, const double *angle0, m3o_dims d,
+                  double *y, double *h_out, double *prevBx_out,
+                  double *angle_out, int nthreads)
+{
+    if (check_dims(d, 1)) return -1;
+    if (!x || !dt || !A || !lam || !theta || !B || !C || !D || !y) return -1;
+    lane_job J;
+    memset(&J, 0, sizeof J);
+    J.x = x; J.dt = dt; J.A = A; J.lam = lam; J.theta = theta; J.B = B; J.C = C;
+    J.D = D; J.Wx = Wx; J.Wy = Wy; J.nrm = nrm; J.h0 = h0; J.prevBx0 = prevBx0;
+    J.angle0 = angle0; J.d = d; J.y = y; J.h_out = h_out;
+    J.prevBx_out = prevBx_out; J.angle_out = angle_out; J.kind = 1;
+    return run_lanes(&J, nthreads);
+}
+
+int m3o_siso_chunked(const double *x, const double *dt, const double *A,
+                     const double *lam, const double *theta, const double *B,
+                     const double *C, const double *D, const m3o_bcnorm *nrm,
+                     const double *h0, const double *prevBx0,
+                     const double *angle0, m3o_dims d, long chunk, double *y,
+                     double *h_out, double *prevBx_out, double *angle_out,
+                     int nthreads)
+{
+    if (check_dims(d, 0) || chunk < 1) return -1;
+    if (!x || !dt || !A || !lam || !theta || !B || !C || !D || !y) return -1;
+    lane_job J;
+    memset(&J, 0, sizeof J);
+    J.x = x; J.dt = dt; J.A = A; J.lam = lam; J.theta = theta; J.B = B; J.C = C;
+    J.D = D; J.nrm = nrm; J.h0 = h0; J.prevBx0 = prevBx0; J.angle0 = angle0;
+    J.d = d; J.d.rank = 1; J.y = y; J.h_out = h_out; J.prevBx_out = prevBx_out;
+    J.angle_out = angle_out; J.kind = 2; J.chunk = chunk;
+    return run_lanes(&J, nthreads);
+}
+
+/* One decode step (SISO): the loop body for a single token, carrying
+ * (h, prev_Bx, angle) in place.  Per-token inputs are shaped as a
+ * one-token sequence: x (Bt,1,H,P), dt/lam (Bt,1,H), theta (Bt,1,H,N/2),
+ * B/C (Bt,1,H,N); y (Bt,1,H,P). */
+int m3o_step_decode(const double *x, const double *dt, const double *A,
+                    const double *lam, const double *theta, const double *B,
+                    const double *C, const double *D, const m3o_bcnorm *nrm,
+                    m3o_dims d, double *h, double *prevBx, double *angle,
+                    double *y, int nthreads)
+{
+    if (!h || !prevBx || !angle) return -1;
+    d.seqlen = 1;
+    long lanes = d.batch * d.nheads, NP = d.dstate * d.headdim;
+    double *h1 = (double *)malloc(sizeof(double) * (lanes * NP + 1));
+    double *u1 = (double *)malloc(sizeof(double) * (lanes * NP + 1));
+    double *a1 = (double *)malloc(sizeof(double) * (lanes * (d.dstate / 2) + 1));
+    int rc = m3o_siso_loop(x, dt, A, lam, theta, B, C, D, nrm, h, prevBx, angle,
+                           d, y, h1, u1, a1, nthreads);
+    if (rc >= 0) {
+        memcpy(h, h1, sizeof(double) * lanes * NP);
+        memcpy(prevBx, u1, sizeof(double) * lanes * NP);
+        memcpy(angle, a1, sizeof(double) * lanes * (d.dstate / 2));
+    }
+    free(h1); free(u1); free(a1);
+    return rc;
+}

@@ -1,0 +1,58 @@
+"""Planted mistakes in the oracle must fail its pins (CPU only).
+
+Each case copies the oracle's C source, plants one plausible mistake (a
+dropped factor, a wrong sign, a wrong index, a swapped operand), compiles the
+copy and runs the pins of ``test_oracle_pins`` against it; at least one pin
+must fail.  This shows the pins constrain every step of the oracle.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import test_oracle_pins as pins
+
+MUTATIONS = [
+    ("beta without alpha", "double be = (1.0 - lm) * dl * al;", "double be = (1.0 - lm) * dl;"),
+    ("gamma with alpha", "double ga = lm * dl;", "double ga = lm * dl * al;"),
+    ("rotation sign", "out[2 * i] = c * v0 - s * v1;", "out[2 * i] = c * v0 + s * v1;"),
+    ("dropped D skip", "yt[p] = acc + J->D[h] * xt[p];", "yt[p] = acc;"),
+    ("swapped U terms", "hs[n * P + p] = al * hs[n * P + p] + be * Up[n * P + p] + ga * u;",
+     "hs[n * P + p] = al * hs[n * P + p] + be * u + ga * Up[n * P + p];"),
+    ("angle without dt", "phi[i] += dl * J->theta[bth * (N / 2) + i];",
+     "phi[i] += J->theta[bth * (N / 2) + i];"),
+    ("y from C transposed to B", "for (long n = 0; n < N; n++) acc += Cb[n] * hs[n * P + p];",
+     "for (long n = 0; n < N; n++) acc += Bb[n] * hs[n * P + p];"),
+    ("alpha sign", "double al = exp(dl * J->A[h]);\n        double be = (1.0 - lm) * dl * al;\n        double ga = lm * dl;\n        for (long i = 0; i < N / 2; i++) phi[i] += dl * J->theta[bth * (N / 2) + i];\n        bc_prepare",
+     "double al = exp(-dl * J->A[h]);\n        double be = (1.0 - lm) * dl * al;\n        double ga = lm * dl;\n        for (long i = 0; i < N / 2; i++) phi[i] += dl * J->theta[bth * (N / 2) + i];\n        bc_prepare"),
+    ("MIMO contract without W_y", "acc += (J->Wy ? J->Wy[(h * R + r) * P + p] : 1.0) * yr;", "acc += yr;"),
+    ("chunk lookahead dropped", "sg = (1.0 - J->lam[nx]) * J->dt[nx];", "sg = 0.0;"),
+]
+
+PIN_CASES = [
+    lambda o: pins.test_complex_ssm_equivalence(o),
+    lambda o: pins.test_matrix_form(o),
+    lambda o: pins.test_closed_form(o, 7),
+    lambda o: pins.test_reduction_mamba2(o),
+    lambda o: pins.test_mimo_r1_equals_siso(o),
+    lambda o: pins.test_mimo_is_r2_siso_calls(o),
+    lambda o: pins.test_split_schedules_siso(o, [2, 4]),
+    lambda o: pins.test_chunked_equals_loop(o, 4, 37),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_planted_mistake_is_caught(oracle_mod, tmp_path, name, old, new):
+    src = open(oracle_mod.oracle_source_path()).read()
+    assert src.count(old) >= 1, "mutation site not found: " + name
+    mutated = tmp_path / "m3_oracle_mut.c"
+    mutated.write_text(src.replace(old, new, 1))
+    lib = oracle_mod.compile_source(str(mutated), str(tmp_path / "libmut.so"))
+    failures = 0
+    with oracle_mod.use_library(lib):
+        for case in PIN_CASES:
+            try:
+                case(oracle_mod)
+            except AssertionError:
+                failures += 1
+    assert failures > 0, "no pin caught the planted mistake: " + name
