@@ -1,0 +1,183 @@
+/*
+ * m3.h -- C ABI of the B200 (sm_100a) Mamba-3 selective-scan library.
+ *
+ * The operation (restated from the pages this library follows; see the
+ * citations on each entry point):
+ *
+ *   alpha_t = exp(dt_t A_h)            beta_t = (1 - lam_t) dt_t alpha_t
+ *   gamma_t = lam_t dt_t
+ *   Phi_t   = Phi_{t-1} + dt_t theta_t          (per rotation pair i < N/2)
+ *   Bbar_t  = R(Phi_t) B_t,  Cbar_t = R(Phi_t) C_t   (pairs (2i, 2i+1))
+ *   U_t     = Bbar_t x_t^T                      (N x P)
+ *   h_t     = alpha_t h_{t-1} + beta_t U_{t-1} + gamma_t U_t
+ *   y_t     = Cbar_t^T h_t + D_h x_t
+ *
+ * with R(phi) the rotation [[cos, -sin], [sin, cos]] of each adjacent pair,
+ * h_{-1} = h0, U_{-1} = prev_Bx0, Phi_{-1} = angle0 (zero when NULL).
+ *
+ * Layouts: row-major, last index fastest, all buffers contiguous.
+ *   x, y        (batch, seqlen, nheads, headdim)         M3_F32 or M3_BF16
+ *   B, C        (batch, seqlen, nheads, dstate)          same dtype as x
+ *               (batch, seqlen, nheads, rank, dstate)    MIMO
+ *   dt, lam     (batch, seqlen, nheads)                  fp32, post-activation
+ *                                                        (dt > 0, 0 <= lam <= 1)
+ *   theta       (batch, seqlen, nheads, dstate/2)        fp32
+ *   A, D        (nheads)                                 fp32
+ *   W_x, W_y    (nheads, rank, headdim)                  fp32 (MIMO)
+ *   h, prev_Bx  (batch, nheads, dstate, headdim)         fp32
+ *   angle       (batch, nheads, dstate/2)                fp32
+ *
+ * Ownership and execution: the caller owns every buffer (device memory,
+ * including the workspace).  The library never allocates, frees or
+ * synchronises; every call validates its arguments on the host, then
+ * enqueues its kernels on `stream` (a cudaStream_t; NULL = legacy default
+ * stream) and returns.  Device pointers must be 16-byte aligned.  Outputs
+ * must not alias inputs, except where an entry point says in/out.
+ *
+ * Errors: validation happens before any launch; on an error nothing is
+ * enqueued and no output is written.  A failed launch returns M3_ERR_CUDA.
+ * No C++ exception crosses this boundary and there is no fallback path.
+ */
+#ifndef M3_H
+#define M3_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    M3_OK = 0,
+    M3_ERR_INVALID_ARG = 1,  /* null required pointer, bad size, odd dstate, misalignment */
+    M3_ERR_UNSUPPORTED = 2,  /* valid but outside this build's limits (see m3_limits)    */
+    M3_ERR_WORKSPACE = 3,    /* workspace missing or smaller than m3_workspace_bytes()   */
+    M3_ERR_CUDA = 4          /* a kernel launch failed                                   */
+} m3_status;
+
+typedef enum { M3_F32 = 0, M3_BF16 = 1 } m3_dtype;
+
+/* Problem sizes.  rank is ignored by the SISO entry points (taken as 1);
+ * chunk is the chunk length of the chunked algorithm (>= 1); seqlen is
+ * ignored by m3_step_decode. */
+typedef struct {
+    int64_t batch, seqlen, nheads, headdim, dstate, rank, chunk;
+} m3_dims;
+
+/* Optional QkNorm + BC-bias applied to B and C before the rotation
+ * (dotLLM pull request, "Key findings": bias after QkNorm, before RoPE):
+ *   B <- B / sqrt(mean_n B^2 + eps) * normw_B   (when normw_B != NULL)
+ *   B <- B + bias_B[h, r, :]                    (when bias_B  != NULL)
+ * and the same for C.  normw_* are (dstate) fp32, bias_* are
+ * (nheads, rank, dstate) fp32 (rank = 1 for SISO).  A NULL m3_bcnorm
+ * pointer turns both off. */
+typedef struct {
+    const float *normw_B, *normw_C, *bias_B, *bias_C;
+    float eps;
+} m3_bcnorm;
+
+/* Limits of this build: dstate <= 256 and even, headdim <= 256,
+ * dstate * headdim <= 16384, rank <= 8 (MIMO). */
+typedef struct {
+    int64_t max_dstate, max_headdim, max_state_elems, max_rank;
+} m3_limits;
+m3_limits m3_get_limits(void);
+
+/* S1 -- trapezoidal discretization.  (dotLLM pull request, "Stage A:
+ * Mamba3Discretize"; TorchMamba README, "Math notes": exponential-trapezoidal
+ * 3-term recurrence, Prop. 1 Eqs. 5-6.)
+ * In: dt, lam (batch, seqlen, nheads) fp32; A (nheads) fp32.
+ * Out: alpha, beta, gamma (batch, seqlen, nheads) fp32.
+ * Uses d.batch, d.seqlen, d.nheads. */
+m3_status m3_discretize(const float *dt, const float *A, const float *lam, m3_dims d,
+                        float *alpha, float *beta, float *gamma, void *stream);
+
+/* S2 -- QkNorm + BC-bias + data-dependent RoPE.  (dotLLM pull request,
+ * "Stage A: Mamba3QkNorm, Mamba3DataRoPE"; TorchMamba README, "Math notes":
+ * accumulated data-dependent pairwise rotations, Props. 2-4.)
+ * In: B, C (batch, seqlen, nheads, [rank,] dstate) of `dtype` (rank axis
+ * present when d.rank > 1); theta, dt; angle0 (batch, nheads, dstate/2) or
+ * NULL for zeros; norm or NULL.
+ * Out: B_rot, C_rot (same shape and dtype as B; values rotated in fp32 and
+ * rounded to nearest-even on store); angle_final (batch, nheads, dstate/2)
+ * or NULL.  Every rank uses the same angle. */
+m3_status m3_rope_bc(const void *B, const void *C, m3_dtype dtype, const float *theta,
+                     const float *dt, const float *angle0, const m3_bcnorm *norm,
+                     m3_dims d, void *B_rot, void *C_rot, float *angle_final,
+                     void *stream);
+
+/* S1+S2+S3 -- SISO chunked forward of the whole scan.  (dotLLM pull
+ * request, "Stage A: Mamba3SelectiveScan", trapezoidal scan Eq. 9 with the
+ * prev_Bx second state, and the streaming-decode comment: shifted_gamma and
+ * the boundary fold; TorchMamba README, "Math notes": Mamba-2 chunkwise
+ * intra-chunk quadratic part plus inter-chunk carry.)
+ * In: x, B, C of `dtype`; dt, lam, theta, A, D fp32; h0, prevBx0
+ * (batch, nheads, dstate, headdim) and angle0, each NULL for zeros.
+ * Out: y (dtype of x), h_final and prevBx_final (fp32, the state after the
+ * last token: h_{T-1} and U_{T-1}), angle_final (fp32); the three state
+ * outputs may be NULL when not wanted.  When seqlen == 0 the states pass
+ * through unchanged.
+ * workspace: device scratch of at least m3_workspace_bytes(M3_WS_SISO, d,
+ * dtype) bytes (may be NULL when that is 0); its contents on entry do not
+ * matter and are undefined on return. */
+m3_status m3_siso_chunked_fwd(const void *x, const float *dt, const float *A,
+                              const float *lam, const float *theta, const void *B,
+                              const void *C, const float *D, m3_dtype dtype,
+                              const m3_bcnorm *norm, const float *h0,
+                              const float *prevBx0, const float *angle0, m3_dims d,
+                              void *y, float *h_final, float *prevBx_final,
+                              float *angle_final, void *workspace, size_t workspace_bytes,
+                              void *stream);
+
+/* S4 -- rank-R MIMO chunked forward on a shared (dstate, headdim) state.
+ * (TorchMamba README, "Models" and "Math notes": rank-R update on a shared
+ * (N,P) state, R^2 SISO calls, App. C per-head expand/contract vectors;
+ * dotLLM pull request, "Mamba-3 MIMO streaming decode": the state is summed
+ * over ranks and the angle is rank-free.)
+ *   X_{t,r}[p] = W_x[h,r,p] x_t[p]
+ *   U_t        = sum_r Bbar_{t,r} X_{t,r}^T
+ *   y_t[p]     = sum_r W_y[h,r,p] (Cbar_{t,r}^T h_t)[p] + D_h x_t[p]
+ * Arguments as m3_siso_chunked_fwd plus W_x, W_y (nheads, rank, headdim)
+ * fp32, each NULL for all ones; B, C are (batch, seqlen, nheads, rank,
+ * dstate).  prevBx_final is U_{T-1} (summed over ranks). */
+m3_status m3_mimo_chunked_fwd(const void *x, const float *dt, const float *A,
+                              const float *lam, const float *theta, const void *B,
+                              const void *C, const float *D, const float *W_x,
+                              const float *W_y, m3_dtype dtype, const m3_bcnorm *norm,
+                              const float *h0, const float *prevBx0, const float *angle0,
+                              m3_dims d, void *y, float *h_final, float *prevBx_final,
+                              float *angle_final, void *workspace, size_t workspace_bytes,
+                              void *stream);
+
+/* S5 -- one SISO decode step for every (batch, head) lane.  (dotLLM pull
+ * request: persistent ssm_state / cum_angle and the single-token step;
+ * TorchMamba README: forward == prefill + step, cache (angle, ssm, ...).)
+ * In: x_t (batch, nheads, headdim) and B_t, C_t (batch, nheads, dstate) of
+ * `dtype`; dt_t, lam_t (batch, nheads), theta_t (batch, nheads, dstate/2),
+ * A, D (nheads) fp32.
+ * In/out: h, prevBx (batch, nheads, dstate, headdim) fp32 and angle
+ * (batch, nheads, dstate/2) fp32, updated in place.
+ * Out: y_t (batch, nheads, headdim) of `dtype`.  d.seqlen is ignored. */
+m3_status m3_step_decode(const void *x_t, const float *dt_t, const float *A,
+                         const float *lam_t, const float *theta_t, const void *B_t,
+                         const void *C_t, const float *D, m3_dtype dtype,
+                         const m3_bcnorm *norm, m3_dims d, float *h, float *prevBx,
+                         float *angle, void *y_t, void *stream);
+
+/* Workspace query for the chunked forwards. */
+enum { M3_WS_SISO = 0, M3_WS_MIMO = 1 };
+size_t m3_workspace_bytes(int which, m3_dims d, m3_dtype dtype);
+
+/* Static description of a status code (never NULL). */
+const char *m3_status_string(m3_status s);
+
+/* Number of kernels the library has enqueued since it was loaded (host-side
+ * counter, incremented once per launch; used to count launches in a timed
+ * region). */
+uint64_t m3_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* M3_H */

@@ -1,0 +1,206 @@
+// m3_api.cu -- the C ABI declared in include/m3.h: argument validation on
+// the host, then kernel launches on the caller's stream.  Nothing here
+// allocates, frees or synchronises.
+#include <atomic>
+#include <cmath>
+
+#include "m3_internal.cuh"
+
+namespace m3 {
+static std::atomic<uint64_t> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace m3
+
+using namespace m3;
+
+namespace {
+
+constexpr int64_t kMaxDstate = 256, kMaxHeaddim = 256, kMaxStateElems = 16384, kMaxRank = 8;
+
+inline bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+// required pointer: non-null and 16-byte aligned
+#define M3_REQ(p)                                                  \
+    do {                                                           \
+        if (!(p) || !aligned16(p)) return M3_ERR_INVALID_ARG;      \
+    } while (0)
+// optional pointer: null, or 16-byte aligned
+#define M3_OPT(p)                                                  \
+    do {                                                           \
+        if ((p) && !aligned16(p)) return M3_ERR_INVALID_ARG;       \
+    } while (0)
+
+m3_status check_dtype(m3_dtype t) {
+    return (t == M3_F32 || t == M3_BF16) ? M3_OK : M3_ERR_INVALID_ARG;
+}
+
+// Sizes shared by the scan, rope and decode entry points.
+m3_status check_core_dims(const m3_dims &d, bool need_seq) {
+    if (d.batch < 0 || d.nheads < 1 || d.headdim < 1 || d.dstate < 2) return M3_ERR_INVALID_ARG;
+    if (need_seq && d.seqlen < 0) return M3_ERR_INVALID_ARG;
+    if (d.dstate & 1) return M3_ERR_INVALID_ARG;  // RoPE pairs need an even dstate
+    if (d.dstate > kMaxDstate || d.headdim > kMaxHeaddim || d.dstate * d.headdim > kMaxStateElems)
+        return M3_ERR_UNSUPPORTED;
+    if (d.batch > (int64_t)1 << 24 || d.nheads > 4096 || (need_seq && d.seqlen > ((int64_t)1 << 31)))
+        return M3_ERR_UNSUPPORTED;
+    return M3_OK;
+}
+
+m3_status read_norm(const m3_bcnorm *n, NormArgs &o) {
+    o = NormArgs{nullptr, nullptr, nullptr, nullptr, 0.f};
+    if (!n) return M3_OK;
+    M3_OPT(n->normw_B);
+    M3_OPT(n->normw_C);
+    M3_OPT(n->bias_B);
+    M3_OPT(n->bias_C);
+    if ((n->normw_B || n->normw_C) && !(n->eps >= 0.f && std::isfinite(n->eps))) return M3_ERR_INVALID_ARG;
+    o = NormArgs{n->normw_B, n->normw_C, n->bias_B, n->bias_C, n->eps};
+    return M3_OK;
+}
+
+inline m3_status launched(cudaError_t e) { return e == cudaSuccess ? M3_OK : M3_ERR_CUDA; }
+
+m3_status chunked_common(const void *x, const float *dt, const float *A, const float *lam,
+                         const float *theta, const void *B, const void *C, const float *D,
+                         const float *Wx, const float *Wy, m3_dtype dtype, const m3_bcnorm *norm,
+                         const float *h0, const float *prevBx0, const float *angle0, m3_dims d,
+                         void *y, float *h_final, float *prevBx_final, float *angle_final,
+                         void *workspace, size_t ws_bytes, void *stream, bool mimo) {
+    m3_status st;
+    if ((st = check_dtype(dtype)) != M3_OK) return st;
+    if ((st = check_core_dims(d, true)) != M3_OK) return st;
+    if (d.chunk < 1) return M3_ERR_INVALID_ARG;
+    const int64_t R = mimo ? d.rank : 1;
+    if (mimo && d.rank < 1) return M3_ERR_INVALID_ARG;
+    if (R > kMaxRank) return M3_ERR_UNSUPPORTED;
+    M3_REQ(A);
+    M3_REQ(D);
+    const bool have_tokens = d.batch > 0 && d.seqlen > 0;
+    if (have_tokens) {
+        M3_REQ(x); M3_REQ(dt); M3_REQ(lam); M3_REQ(theta); M3_REQ(B); M3_REQ(C); M3_REQ(y);
+    } else {
+        M3_OPT(x); M3_OPT(dt); M3_OPT(lam); M3_OPT(theta); M3_OPT(B); M3_OPT(C); M3_OPT(y);
+    }
+    M3_OPT(Wx); M3_OPT(Wy); M3_OPT(h0); M3_OPT(prevBx0); M3_OPT(angle0);
+    M3_OPT(h_final); M3_OPT(prevBx_final); M3_OPT(angle_final); M3_OPT(workspace);
+    NormArgs nrm;
+    if ((st = read_norm(norm, nrm)) != M3_OK) return st;
+    const size_t need = m3_workspace_bytes(mimo ? M3_WS_MIMO : M3_WS_SISO, d, dtype);
+    if (need > 0 && (!workspace || ws_bytes < need)) return M3_ERR_WORKSPACE;
+    const int q = scan_simt_chunk(d.headdim, d.dstate, R, d.chunk);
+    if (q < 1) return M3_ERR_UNSUPPORTED;
+    if (d.batch == 0) return M3_OK;
+
+    ScanArgs a;
+    a.x = x; a.B = B; a.C = C;
+    a.dt = dt; a.A = A; a.lam = lam; a.theta = theta; a.D = D; a.Wx = Wx; a.Wy = Wy;
+    a.h0 = h0; a.prevBx0 = prevBx0; a.angle0 = angle0;
+    a.nrm = nrm;
+    a.y = y; a.h_out = h_final; a.prevBx_out = prevBx_final; a.angle_out = angle_final;
+    a.Bt = d.batch; a.T = d.seqlen; a.H = d.nheads; a.P = d.headdim; a.N = d.dstate; a.R = R;
+    a.Q = q;
+    a.mimo_layout = mimo ? 1 : 0;
+    return launched(launch_scan_simt(a, dtype, (cudaStream_t)stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+m3_limits m3_get_limits(void) { return m3_limits{kMaxDstate, kMaxHeaddim, kMaxStateElems, kMaxRank}; }
+
+uint64_t m3_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char *m3_status_string(m3_status s) {
+    switch (s) {
+        case M3_OK: return "M3_OK: success";
+        case M3_ERR_INVALID_ARG: return "M3_ERR_INVALID_ARG: null, misaligned or inconsistent argument";
+        case M3_ERR_UNSUPPORTED: return "M3_ERR_UNSUPPORTED: sizes outside this build's limits";
+        case M3_ERR_WORKSPACE: return "M3_ERR_WORKSPACE: workspace missing or too small";
+        case M3_ERR_CUDA: return "M3_ERR_CUDA: a kernel launch failed";
+    }
+    return "unknown m3_status";
+}
+
+size_t m3_workspace_bytes(int which, m3_dims d, m3_dtype dtype) {
+    (void)which; (void)d; (void)dtype;
+    return 0;
+}
+
+m3_status m3_discretize(const float *dt, const float *A, const float *lam, m3_dims d, float *alpha,
+                        float *beta, float *gamma, void *stream) {
+    if (d.batch < 0 || d.seqlen < 0 || d.nheads < 1) return M3_ERR_INVALID_ARG;
+    M3_REQ(A);
+    if (d.batch * d.seqlen == 0) return M3_OK;
+    M3_REQ(dt); M3_REQ(lam); M3_REQ(alpha); M3_REQ(beta); M3_REQ(gamma);
+    return launched(launch_discretize(dt, A, lam, d.batch, d.seqlen, d.nheads, alpha, beta, gamma,
+                                      (cudaStream_t)stream));
+}
+
+m3_status m3_rope_bc(const void *B, const void *C, m3_dtype dtype, const float *theta, const float *dt,
+                     const float *angle0, const m3_bcnorm *norm, m3_dims d, void *B_rot, void *C_rot,
+                     float *angle_final, void *stream) {
+    m3_status st;
+    if ((st = check_dtype(dtype)) != M3_OK) return st;
+    if ((st = check_core_dims(d, true)) != M3_OK) return st;
+    const int64_t R = d.rank > 1 ? d.rank : 1;
+    if (d.rank < 0) return M3_ERR_INVALID_ARG;
+    if (R > kMaxRank) return M3_ERR_UNSUPPORTED;
+    if (d.batch > 0 && d.seqlen > 0) {
+        M3_REQ(B); M3_REQ(C); M3_REQ(theta); M3_REQ(dt); M3_REQ(B_rot); M3_REQ(C_rot);
+    }
+    M3_OPT(angle0); M3_OPT(angle_final);
+    NormArgs nrm;
+    if ((st = read_norm(norm, nrm)) != M3_OK) return st;
+    if (d.batch == 0) return M3_OK;
+    RopeArgs a;
+    a.B = B; a.C = C; a.theta = theta; a.dt = dt; a.angle0 = angle0; a.nrm = nrm;
+    a.Bo = B_rot; a.Co = C_rot; a.angle_out = angle_final;
+    a.Bt = d.batch; a.T = d.seqlen; a.H = d.nheads; a.R = R; a.N = d.dstate;
+    return launched(launch_rope(a, dtype, (cudaStream_t)stream));
+}
+
+m3_status m3_siso_chunked_fwd(const void *x, const float *dt, const float *A, const float *lam,
+                              const float *theta, const void *B, const void *C, const float *D,
+                              m3_dtype dtype, const m3_bcnorm *norm, const float *h0,
+                              const float *prevBx0, const float *angle0, m3_dims d, void *y,
+                              float *h_final, float *prevBx_final, float *angle_final, void *workspace,
+                              size_t workspace_bytes, void *stream) {
+    return chunked_common(x, dt, A, lam, theta, B, C, D, nullptr, nullptr, dtype, norm, h0, prevBx0,
+                          angle0, d, y, h_final, prevBx_final, angle_final, workspace, workspace_bytes,
+                          stream, false);
+}
+
+m3_status m3_mimo_chunked_fwd(const void *x, const float *dt, const float *A, const float *lam,
+                              const float *theta, const void *B, const void *C, const float *D,
+                              const float *W_x, const float *W_y, m3_dtype dtype, const m3_bcnorm *norm,
+                              const float *h0, const float *prevBx0, const float *angle0, m3_dims d,
+                              void *y, float *h_final, float *prevBx_final, float *angle_final,
+                              void *workspace, size_t workspace_bytes, void *stream) {
+    return chunked_common(x, dt, A, lam, theta, B, C, D, W_x, W_y, dtype, norm, h0, prevBx0, angle0, d, y,
+                          h_final, prevBx_final, angle_final, workspace, workspace_bytes, stream, true);
+}
+
+m3_status m3_step_decode(const void *x_t, const float *dt_t, const float *A, const float *lam_t,
+                         const float *theta_t, const void *B_t, const void *C_t, const float *D,
+                         m3_dtype dtype, const m3_bcnorm *norm, m3_dims d, float *h, float *prevBx,
+                         float *angle, void *y_t, void *stream) {
+    m3_status st;
+    if ((st = check_dtype(dtype)) != M3_OK) return st;
+    if ((st = check_core_dims(d, false)) != M3_OK) return st;
+    M3_REQ(A); M3_REQ(D);
+    if (d.batch > 0) {
+        M3_REQ(x_t); M3_REQ(dt_t); M3_REQ(lam_t); M3_REQ(theta_t); M3_REQ(B_t); M3_REQ(C_t);
+        M3_REQ(h); M3_REQ(prevBx); M3_REQ(angle); M3_REQ(y_t);
+    }
+    NormArgs nrm;
+    if ((st = read_norm(norm, nrm)) != M3_OK) return st;
+    if (d.batch == 0) return M3_OK;
+    DecodeArgs a;
+    a.x = x_t; a.B = B_t; a.C = C_t; a.dt = dt_t; a.A = A; a.lam = lam_t; a.theta = theta_t; a.D = D;
+    a.nrm = nrm; a.h = h; a.prevBx = prevBx; a.angle = angle; a.y = y_t;
+    a.Bt = d.batch; a.H = d.nheads; a.P = d.headdim; a.N = d.dstate;
+    return launched(launch_decode(a, dtype, (cudaStream_t)stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,79 @@
+// m3_internal.cuh -- shared declarations of the CUDA side (not part of the ABI).
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "m3.h"
+
+namespace m3 {
+
+// ---- element access: every kernel computes in fp32 ------------------------
+__device__ __forceinline__ float ldf(const float *p, int64_t i) { return p[i]; }
+__device__ __forceinline__ float ldf(const __nv_bfloat16 *p, int64_t i) { return __bfloat162float(p[i]); }
+__device__ __forceinline__ void stf(float *p, int64_t i, float v) { p[i] = v; }
+__device__ __forceinline__ void stf(__nv_bfloat16 *p, int64_t i, float v) { p[i] = __float2bfloat16_rn(v); }
+
+// Sum over the whole block (blockDim.x a multiple of 32, <= 1024).  `red`
+// holds 32 floats of shared memory.  Every thread receives the total.
+__device__ __forceinline__ float block_sum(float v, float *red) {
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = blockDim.x >> 5;
+    __syncthreads();
+    if (l == 0) red[w] = v;
+    __syncthreads();
+    float s = 0.f;
+    for (int i = 0; i < nw; i++) s += red[i];
+    return s;
+}
+
+// ---- launch descriptions (host fills, kernels read) ----------------------
+struct NormArgs {
+    const float *wB, *wC, *biasB, *biasC;
+    float eps;
+};
+
+struct ScanArgs {
+    const void *x, *B, *C;
+    const float *dt, *A, *lam, *theta, *D, *Wx, *Wy;
+    const float *h0, *prevBx0, *angle0;
+    NormArgs nrm;
+    void *y;
+    float *h_out, *prevBx_out, *angle_out;
+    int64_t Bt, T, H, P, N, R;
+    int Q;             // chunk length actually used by the kernel
+    int mimo_layout;   // B/C carry a rank axis
+};
+
+struct DecodeArgs {
+    const void *x, *B, *C;
+    const float *dt, *A, *lam, *theta, *D;
+    NormArgs nrm;
+    float *h, *prevBx, *angle;
+    void *y;
+    int64_t Bt, H, P, N;
+};
+
+struct RopeArgs {
+    const void *B, *C;
+    const float *theta, *dt, *angle0;
+    NormArgs nrm;
+    void *Bo, *Co;
+    float *angle_out;
+    int64_t Bt, T, H, R, N;
+};
+
+// Host launchers (each returns cudaSuccess or the launch error).
+cudaError_t launch_discretize(const float *dt, const float *A, const float *lam, int64_t Bt,
+                              int64_t T, int64_t H, float *al, float *be, float *ga,
+                              cudaStream_t s);
+cudaError_t launch_rope(const RopeArgs &a, m3_dtype dt, cudaStream_t s);
+cudaError_t launch_scan_simt(const ScanArgs &a, m3_dtype dt, cudaStream_t s);
+size_t scan_simt_smem_bytes(int64_t P, int64_t N, int64_t R, int Q);
+int scan_simt_chunk(int64_t P, int64_t N, int64_t R, int64_t chunk);
+cudaError_t launch_decode(const DecodeArgs &a, m3_dtype dt, cudaStream_t s);
+
+// Launch counter shared by all launchers.
+void count_launch(int n = 1);
+
+}  // namespace m3

@@ -1,0 +1,238 @@
+"""Python binding of the C ABI in ``include/m3.h`` (ctypes).
+
+Argument marshalling only: every step of the scan runs in the CUDA library.
+Tensors are torch CUDA tensors (PyTorch supplies device memory and streams);
+outputs that the caller does not pass are allocated with ``torch.empty``.
+If the library has not been built, every call raises ``RuntimeError`` -- there
+is no other implementation behind these names.
+"""
+import ctypes
+import os
+
+import torch
+
+from .build import LIB
+
+M3_OK, M3_ERR_INVALID_ARG, M3_ERR_UNSUPPORTED, M3_ERR_WORKSPACE, M3_ERR_CUDA = range(5)
+M3_F32, M3_BF16 = 0, 1
+M3_WS_SISO, M3_WS_MIMO = 0, 1
+
+_DTYPE = {torch.float32: M3_F32, torch.bfloat16: M3_BF16}
+
+ABI_FUNCTIONS = (
+    "m3_get_limits", "m3_discretize", "m3_rope_bc", "m3_siso_chunked_fwd",
+    "m3_mimo_chunked_fwd", "m3_step_decode", "m3_workspace_bytes", "m3_status_string",
+    "m3_launch_count",
+)
+
+
+class M3Error(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__("%s: %s" % (where, status_string(status)))
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64),
+                ("nheads", ctypes.c_int64), ("headdim", ctypes.c_int64),
+                ("dstate", ctypes.c_int64), ("rank", ctypes.c_int64),
+                ("chunk", ctypes.c_int64)]
+
+
+class BcNorm(ctypes.Structure):
+    _fields_ = [("normw_B", ctypes.c_void_p), ("normw_C", ctypes.c_void_p),
+                ("bias_B", ctypes.c_void_p), ("bias_C", ctypes.c_void_p),
+                ("eps", ctypes.c_float)]
+
+
+class Limits(ctypes.Structure):
+    _fields_ = [("max_dstate", ctypes.c_int64), ("max_headdim", ctypes.c_int64),
+                ("max_state_elems", ctypes.c_int64), ("max_rank", ctypes.c_int64)]
+
+
+_lib = None
+_VP = ctypes.c_void_p
+
+
+def library_path():
+    return LIB
+
+
+def lib():
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB):
+        raise RuntimeError("the CUDA library %s is missing: run `python -m state_space_lm_b200.build`"
+                           % LIB)
+    L = ctypes.CDLL(LIB)
+    L.m3_get_limits.restype = Limits
+    L.m3_get_limits.argtypes = []
+    L.m3_status_string.restype = ctypes.c_char_p
+    L.m3_status_string.argtypes = [ctypes.c_int]
+    L.m3_workspace_bytes.restype = ctypes.c_size_t
+    L.m3_workspace_bytes.argtypes = [ctypes.c_int, Dims, ctypes.c_int]
+    L.m3_launch_count.restype = ctypes.c_uint64
+    L.m3_launch_count.argtypes = []
+    L.m3_discretize.restype = ctypes.c_int
+    L.m3_discretize.argtypes = [_VP, _VP, _VP, Dims, _VP, _VP, _VP, _VP]
+    L.m3_rope_bc.restype = ctypes.c_int
+    L.m3_rope_bc.argtypes = [_VP, _VP, ctypes.c_int, _VP, _VP, _VP, ctypes.POINTER(BcNorm), Dims,
+                             _VP, _VP, _VP, _VP]
+    L.m3_siso_chunked_fwd.restype = ctypes.c_int
+    L.m3_siso_chunked_fwd.argtypes = [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int,
+                                      ctypes.POINTER(BcNorm), _VP, _VP, _VP, Dims, _VP, _VP, _VP,
+                                      _VP, _VP, ctypes.c_size_t, _VP]
+    L.m3_mimo_chunked_fwd.restype = ctypes.c_int
+    L.m3_mimo_chunked_fwd.argtypes = [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+                                      ctypes.c_int, ctypes.POINTER(BcNorm), _VP, _VP, _VP, Dims,
+                                      _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t, _VP]
+    L.m3_step_decode.restype = ctypes.c_int
+    L.m3_step_decode.argtypes = [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int,
+                                 ctypes.POINTER(BcNorm), Dims, _VP, _VP, _VP, _VP, _VP]
+    _lib = L
+    return L
+
+
+def status_string(status):
+    return lib().m3_status_string(int(status)).decode()
+
+
+def launch_count():
+    return int(lib().m3_launch_count())
+
+
+def limits():
+    l = lib().m3_get_limits()
+    return dict(max_dstate=l.max_dstate, max_headdim=l.max_headdim,
+                max_state_elems=l.max_state_elems, max_rank=l.max_rank)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _norm(norm):
+    if norm is None:
+        return None, ()
+    keep = tuple(norm.get(k) for k in ("normw_B", "normw_C", "bias_B", "bias_C"))
+    s = BcNorm(*[_ptr(k) for k in keep], float(norm.get("eps", 1e-5)))
+    return ctypes.byref(s), keep + (s,)
+
+
+def _check(rc, where):
+    if rc != M3_OK:
+        raise M3Error(rc, where)
+
+
+def workspace_bytes(which, dims, dtype):
+    return int(lib().m3_workspace_bytes(int(which), dims, int(dtype)))
+
+
+def discretize(dt, A, lam, out=None, stream=None):
+    """S1: alpha, beta, gamma (Bt,T,H) fp32."""
+    Bt, T, H = dt.shape
+    al, be, ga = out if out is not None else tuple(torch.empty_like(dt) for _ in range(3))
+    d = Dims(Bt, T, H, 1, 2, 1, 1)
+    _check(lib().m3_discretize(_ptr(dt), _ptr(A), _ptr(lam), d, _ptr(al), _ptr(be), _ptr(ga),
+                               _stream(stream)), "m3_discretize")
+    return al, be, ga
+
+
+def rope_bc(B, C, theta, dt, angle0=None, norm=None, out=None, stream=None):
+    """S2: B_rot, C_rot (shape/dtype of B) and angle_final (Bt,H,N/2) fp32.
+    B, C are (Bt,T,H,N) or (Bt,T,H,R,N)."""
+    if B.dim() == 4:
+        Bt, T, H, N = B.shape
+        R = 1
+    else:
+        Bt, T, H, R, N = B.shape
+    if out is None:
+        out = (torch.empty_like(B), torch.empty_like(C),
+               torch.empty(Bt, H, N // 2, device=B.device, dtype=torch.float32))
+    Br, Cr, ang = out
+    nptr, keep = _norm(norm)
+    d = Dims(Bt, T, H, 1, N, R, 1)
+    _check(lib().m3_rope_bc(_ptr(B), _ptr(C), _DTYPE[B.dtype], _ptr(theta), _ptr(dt), _ptr(angle0),
+                            nptr, d, _ptr(Br), _ptr(Cr), _ptr(ang), _stream(stream)), "m3_rope_bc")
+    return Br, Cr, ang
+
+
+def _state_outs(x, N, P, out):
+    Bt, T, H = x.shape[0], x.shape[1], x.shape[2]
+    if out is not None:
+        return out
+    dev = x.device
+    return (torch.empty_like(x), torch.empty(Bt, H, N, P, device=dev, dtype=torch.float32),
+            torch.empty(Bt, H, N, P, device=dev, dtype=torch.float32),
+            torch.empty(Bt, H, N // 2, device=dev, dtype=torch.float32))
+
+
+def _workspace(which, d, dtype, workspace, dev):
+    need = workspace_bytes(which, d, dtype)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return workspace, nbytes
+
+
+def siso_chunked_fwd(x, dt, A, lam, theta, B, C, D, chunk, norm=None, h0=None, prevBx0=None,
+                     angle0=None, workspace=None, out=None, stream=None):
+    """S1+S2+S3: returns y (Bt,T,H,P), h_final, prevBx_final (Bt,H,N,P), angle_final."""
+    Bt, T, H, P = x.shape
+    N = B.shape[-1]
+    y, hf, uf, af = _state_outs(x, N, P, out)
+    d = Dims(Bt, T, H, P, N, 1, int(chunk))
+    dtype = _DTYPE[x.dtype]
+    ws, nbytes = _workspace(M3_WS_SISO, d, dtype, workspace, x.device)
+    nptr, keep = _norm(norm)
+    _check(lib().m3_siso_chunked_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(lam), _ptr(theta), _ptr(B),
+                                     _ptr(C), _ptr(D), dtype, nptr, _ptr(h0), _ptr(prevBx0),
+                                     _ptr(angle0), d, _ptr(y), _ptr(hf), _ptr(uf), _ptr(af),
+                                     _ptr(ws), nbytes, _stream(stream)), "m3_siso_chunked_fwd")
+    return y, hf, uf, af
+
+
+def mimo_chunked_fwd(x, dt, A, lam, theta, B, C, D, chunk, W_x=None, W_y=None, norm=None, h0=None,
+                     prevBx0=None, angle0=None, workspace=None, out=None, stream=None):
+    """S4: B, C (Bt,T,H,R,N); W_x, W_y (H,R,P) or None for ones."""
+    Bt, T, H, P = x.shape
+    R, N = B.shape[-2], B.shape[-1]
+    y, hf, uf, af = _state_outs(x, N, P, out)
+    d = Dims(Bt, T, H, P, N, R, int(chunk))
+    dtype = _DTYPE[x.dtype]
+    ws, nbytes = _workspace(M3_WS_MIMO, d, dtype, workspace, x.device)
+    nptr, keep = _norm(norm)
+    _check(lib().m3_mimo_chunked_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(lam), _ptr(theta), _ptr(B),
+                                     _ptr(C), _ptr(D), _ptr(W_x), _ptr(W_y), dtype, nptr, _ptr(h0),
+                                     _ptr(prevBx0), _ptr(angle0), d, _ptr(y), _ptr(hf), _ptr(uf),
+                                     _ptr(af), _ptr(ws), nbytes, _stream(stream)),
+           "m3_mimo_chunked_fwd")
+    return y, hf, uf, af
+
+
+def step_decode(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, prevBx, angle, norm=None, y_out=None,
+                stream=None):
+    """S5: one decode step; h, prevBx, angle are updated in place; returns y_t (Bt,H,P)."""
+    Bt, H, P = x_t.shape
+    N = B_t.shape[-1]
+    y = torch.empty_like(x_t) if y_out is None else y_out
+    d = Dims(Bt, 1, H, P, N, 1, 1)
+    nptr, keep = _norm(norm)
+    _check(lib().m3_step_decode(_ptr(x_t), _ptr(dt_t), _ptr(A), _ptr(lam_t), _ptr(theta_t),
+                                _ptr(B_t), _ptr(C_t), _ptr(D), _DTYPE[x_t.dtype], nptr, d, _ptr(h),
+                                _ptr(prevBx), _ptr(angle), _ptr(y), _stream(stream)),
+           "m3_step_decode")
+    return y

@@ -1,0 +1,123 @@
+"""The C-ABI library: it loads, exports every symbol include/m3.h declares, and
+rejects bad arguments on the host before any launch (CPU only: no call here
+passes validation, so no kernel is ever enqueued)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from state_space_lm_b200 import build as m3build
+from state_space_lm_b200 import m3
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    m3build.build()
+    return m3.lib()
+
+
+def header_symbols():
+    src = open(os.path.join(ROOT, "include", "m3.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(m3_[a-z_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    syms = header_symbols()
+    assert len(syms) >= 9
+    for s in syms:
+        assert hasattr(L, s), s
+    assert set(syms) == set(m3.ABI_FUNCTIONS)
+
+
+def test_status_strings_and_limits(L):
+    for code in range(5):
+        s = m3.status_string(code)
+        assert s.startswith("M3_")
+    assert "unknown" in m3.status_string(99)
+    lim = m3.limits()
+    assert lim["max_dstate"] >= 128 and lim["max_headdim"] >= 64 and lim["max_rank"] >= 4
+
+
+FAKE = 0x10000      # aligned, never dereferenced: every call below fails validation
+MIS = 0x10004       # misaligned
+
+
+def dims(**kw):
+    base = dict(batch=2, seqlen=8, nheads=2, headdim=4, dstate=4, rank=1, chunk=4)
+    base.update(kw)
+    return m3.Dims(*[base[k] for k in ("batch", "seqlen", "nheads", "headdim", "dstate", "rank", "chunk")])
+
+
+def siso(L, d, x=FAKE, dt=FAKE, A=FAKE, lam=FAKE, theta=FAKE, B=FAKE, C=FAKE, D=FAKE, dtype=m3.M3_BF16,
+         y=FAKE, ws=None, nbytes=0):
+    return L.m3_siso_chunked_fwd(x, dt, A, lam, theta, B, C, D, dtype, None, None, None, None, d, y,
+                                 None, None, None, ws, nbytes, None)
+
+
+def test_siso_validation(L):
+    assert siso(L, dims(dstate=5)) == m3.M3_ERR_INVALID_ARG              # odd N: RoPE needs pairs
+    assert siso(L, dims(dstate=0)) == m3.M3_ERR_INVALID_ARG
+    assert siso(L, dims(nheads=0)) == m3.M3_ERR_INVALID_ARG
+    assert siso(L, dims(batch=-1)) == m3.M3_ERR_INVALID_ARG
+    assert siso(L, dims(seqlen=-3)) == m3.M3_ERR_INVALID_ARG
+    assert siso(L, dims(chunk=0)) == m3.M3_ERR_INVALID_ARG
+    assert siso(L, dims(), x=None) == m3.M3_ERR_INVALID_ARG              # null required pointer
+    assert siso(L, dims(), theta=None) == m3.M3_ERR_INVALID_ARG
+    assert siso(L, dims(), y=MIS) == m3.M3_ERR_INVALID_ARG               # misaligned
+    assert siso(L, dims(), dtype=7) == m3.M3_ERR_INVALID_ARG
+    assert siso(L, dims(dstate=512)) == m3.M3_ERR_UNSUPPORTED
+    assert siso(L, dims(headdim=512)) == m3.M3_ERR_UNSUPPORTED
+    assert siso(L, dims(dstate=256, headdim=128)) == m3.M3_ERR_UNSUPPORTED
+    # an empty batch is valid and enqueues nothing
+    n0 = m3.launch_count()
+    assert siso(L, dims(batch=0), x=None, dt=None, lam=None, theta=None, B=None, C=None, y=None) == m3.M3_OK
+    assert m3.launch_count() == n0
+
+
+def test_mimo_validation(L):
+    def mimo(d, **kw):
+        a = dict(x=FAKE, dt=FAKE, A=FAKE, lam=FAKE, theta=FAKE, B=FAKE, C=FAKE, D=FAKE, Wx=None, Wy=None)
+        a.update(kw)
+        return L.m3_mimo_chunked_fwd(a["x"], a["dt"], a["A"], a["lam"], a["theta"], a["B"], a["C"], a["D"],
+                                     a["Wx"], a["Wy"], m3.M3_BF16, None, None, None, None, d, FAKE, None,
+                                     None, None, None, 0, None)
+    assert mimo(dims(rank=0)) == m3.M3_ERR_INVALID_ARG
+    assert mimo(dims(rank=64)) == m3.M3_ERR_UNSUPPORTED
+    assert mimo(dims(rank=2), Wx=MIS) == m3.M3_ERR_INVALID_ARG
+
+
+def test_norm_validation(L):
+    nrm = m3.BcNorm(FAKE, FAKE, None, None, -1.0)                       # negative eps
+    rc = L.m3_siso_chunked_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, m3.M3_BF16,
+                               ctypes.byref(nrm), None, None, None, dims(), FAKE, None, None, None, None,
+                               0, None)
+    assert rc == m3.M3_ERR_INVALID_ARG
+    nrm = m3.BcNorm(MIS, None, None, None, 1e-5)
+    rc = L.m3_siso_chunked_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, m3.M3_BF16,
+                               ctypes.byref(nrm), None, None, None, dims(), FAKE, None, None, None, None,
+                               0, None)
+    assert rc == m3.M3_ERR_INVALID_ARG
+
+
+def test_decode_rope_discretize_validation(L):
+    d = dims()
+    assert L.m3_step_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, m3.M3_BF16, None, dims(dstate=3),
+                            FAKE, FAKE, FAKE, FAKE, None) == m3.M3_ERR_INVALID_ARG
+    assert L.m3_step_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, m3.M3_BF16, None, d,
+                            None, FAKE, FAKE, FAKE, None) == m3.M3_ERR_INVALID_ARG
+    assert L.m3_rope_bc(FAKE, FAKE, m3.M3_BF16, FAKE, FAKE, None, None, dims(dstate=7), FAKE, FAKE, None,
+                        None) == m3.M3_ERR_INVALID_ARG
+    assert L.m3_rope_bc(FAKE, None, m3.M3_BF16, FAKE, FAKE, None, None, d, FAKE, FAKE, None,
+                        None) == m3.M3_ERR_INVALID_ARG
+    assert L.m3_discretize(FAKE, None, FAKE, d, FAKE, FAKE, FAKE, None) == m3.M3_ERR_INVALID_ARG
+    assert L.m3_discretize(FAKE, FAKE, FAKE, dims(nheads=0), FAKE, FAKE, FAKE, None) == m3.M3_ERR_INVALID_ARG
+
+
+def test_workspace_query(L):
+    for which in (m3.M3_WS_SISO, m3.M3_WS_MIMO):
+        n = m3.workspace_bytes(which, dims(), m3.M3_BF16)
+        assert n >= 0
