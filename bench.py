@@ -1,0 +1,453 @@
+"""Throughput of the Mamba-3 scan on B200 (tokens/s, B*T per second, all heads).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config I] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+for the chunked workloads one ``m3_siso_chunked_fwd`` / ``m3_mimo_chunked_fwd``
+call (discretization, rotation and scan fused), for the decode workload one
+``m3_step_decode`` over every (batch, head) lane.  The default workload is
+the SISO 434M-layer shape (batch 8, seqlen 2048, 16 heads, headdim 64,
+dState 128, chunk 64, bf16).
+
+For N > 1 (torchrun) every rank runs an independent replica of the workload on
+its own GPU: the (batch, head) lanes are independent, there is no exchange
+step and no collective on the data path (weak scaling); rank 0 prints the
+whole-job value = units of all ranks / max-over-ranks device time.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference this path
+has) on the host cores, on a bounded sample of the same workload per step.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from state_space_lm_b200 import inputs as gen  # noqa: E402
+
+METRIC = "Mamba-3 scan tokens/s (B·T) at H=16 and % of tensor/HBM roofline, 1×B200"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def aggregate(elapsed_s, units, dist=None, device=None):
+    """Whole-job throughput: sum of units over ranks / max of device time over
+    ranks.  Returns (value, max_elapsed_s, total_units)."""
+    if dist is None:
+        return units / elapsed_s, elapsed_s, units
+    t = torch.tensor([elapsed_s], dtype=torch.float64, device=device)
+    u = torch.tensor([units], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(u.item() / t.item()), float(t.item()), float(u.item())
+
+
+# ---------------------------------------------------------------------------
+# measurement helpers
+# ---------------------------------------------------------------------------
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons through NVML while running."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index, period_s=0.002):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = None
+            try:  # the NVML handle of the same physical GPU as the CUDA device
+                pr = torch.cuda.get_device_properties(device_index)
+                bus = "%08x:%02x:%02x.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.nv = None
+            self.err = str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self._reasons_fn(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def report(self):
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable: " + self.err]}
+        names = [k for k, v in self.REASONS.items() if self.reasons & v]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+def source_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(kernel, src_paths):
+    """DRAM bytes per launch from a committed ncu summary, only if the kernel's
+    sources are unchanged since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f).get(kernel)
+    if not rec or rec.get("source_hash") != source_hash(src_paths):
+        return None
+    return rec
+
+
+# ---------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------
+def scan_bytes(c):
+    """Algorithmic bytes of one chunked-scan call: every input once, every
+    output once, plus the final states (h, prev_Bx, angle)."""
+    Bt, T, H, P, N, R = c["batch"], c["seqlen"], c["nheads"], c["headdim"], c["dstate"], c["rank"]
+    es = 2 if c["dtype"] == "bf16" else 4
+    per_token_head = es * P + 2 * es * R * N + 4 + 4 + 4 * (N // 2) + es * P
+    states = Bt * H * (2 * N * P * 4 + (N // 2) * 4)
+    params = H * 8 + (2 * H * R * P * 4 if R > 1 else 0)
+    return Bt * T * H * per_token_head + states + params
+
+
+def scan_flops(c):
+    """Causal-lower-triangle flops of the chunked form (the dense work it
+    skips is not counted): per chunk 2*pairs*R^2*(N+P) + 4*Q*R*N*P + 2*N*P."""
+    Bt, T, H, P, N, R, Q = (c["batch"], c["seqlen"], c["nheads"], c["headdim"], c["dstate"], c["rank"],
+                            c["chunk"])
+    total = 0
+    for t0 in range(0, T, Q):
+        L = min(Q, T - t0)
+        pairs = L * (L + 1) // 2
+        total += 2 * pairs * R * R * (N + P) + 4 * L * R * N * P + 2 * N * P
+    return Bt * H * total
+
+
+def decode_bytes(c):
+    Bt, H, P, N = c["batch"], c["nheads"], c["headdim"], c["dstate"]
+    es = 2
+    per_lane = 2 * 2 * N * P * 4 + 2 * (N // 2) * 4 + es * P + 2 * es * N + 8 + 4 * (N // 2) + es * P
+    return Bt * H * per_lane
+
+
+class ScanWorkload:
+    def __init__(self, idx, device):
+        from state_space_lm_b200 import m3
+        self.m3 = m3
+        self.c = dict(gen.CONFIGS[idx])
+        self.idx = idx
+        c = self.c
+        self.host = gen.config_inputs(idx)
+        self.host.pop("generator")
+        self.dev = {k: v.to(device) for k, v in self.host.items() if isinstance(v, torch.Tensor)}
+        Bt, T, H, P, N = c["batch"], c["seqlen"], c["nheads"], c["headdim"], c["dstate"]
+        self.out = (torch.empty(Bt, T, H, P, device=device, dtype=self.dev["x"].dtype),
+                    torch.empty(Bt, H, N, P, device=device), torch.empty(Bt, H, N, P, device=device),
+                    torch.empty(Bt, H, N // 2, device=device))
+        self.mimo = c["rank"] > 1
+        d = self.m3.Dims(Bt, T, H, P, N, c["rank"], c["chunk"])
+        which = self.m3.M3_WS_MIMO if self.mimo else self.m3.M3_WS_SISO
+        nws = self.m3.workspace_bytes(which, d, self.m3.M3_BF16 if c["dtype"] == "bf16" else self.m3.M3_F32)
+        self.ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=device)
+        self.units = Bt * T                       # tokens (b, t), all heads
+        self.bytes = scan_bytes(c)
+        self.flops = scan_flops(c)
+        self.kernel = "k_scan"
+        self.srcs = [os.path.join(ROOT, "state_space_lm_b200", "csrc", f)
+                     for f in sorted(os.listdir(os.path.join(ROOT, "state_space_lm_b200", "csrc")))]
+        self.input_bytes = sum(v.numel() * v.element_size() for v in self.dev.values())
+
+    def step(self, dev=None, out=None, stream=None):
+        d = self.dev if dev is None else dev
+        o = self.out if out is None else out
+        if self.mimo:
+            self.m3.mimo_chunked_fwd(d["x"], d["dt"], d["A"], d["lam"], d["theta"], d["B"], d["C"], d["D"],
+                                     self.c["chunk"], W_x=d["Wx"], W_y=d["Wy"], workspace=self.ws, out=o,
+                                     stream=stream)
+        else:
+            self.m3.siso_chunked_fwd(d["x"], d["dt"], d["A"], d["lam"], d["theta"], d["B"], d["C"], d["D"],
+                                     self.c["chunk"], workspace=self.ws, out=o, stream=stream)
+
+    def config(self):
+        c = self.c
+        return {"workload": c["name"], "batch": c["batch"], "seqlen": c["seqlen"], "nheads": c["nheads"],
+                "headdim": c["headdim"], "dstate": c["dstate"], "rank": c["rank"], "chunk": c["chunk"],
+                "inputs": "x/B/C %s, dt/lam/theta/A/D fp32, seeded synthetic" % c["dtype"],
+                "l2": "inputs larger than L2 (%.0f MB vs 126 MB), no flush" % (self.input_bytes / 1e6)}
+
+    # ---- oracle on a bounded sample of lanes (CPU baseline) ----
+    def oracle_sample(self, n_lanes, threads):
+        import oracle
+        c = self.c
+        H = c["nheads"]
+        lanes = [(i // H, i % H) for i in range(min(n_lanes, c["batch"] * H))]
+        bs = sorted({b for b, _ in lanes})
+        hs = sorted({h for _, h in lanes})
+        sl = lambda t: t[bs[0]:bs[-1] + 1, :, hs[0]:hs[-1] + 1]
+        keys = ("x", "dt", "A", "lam", "theta", "B", "C", "D")
+        arr = {}
+        for k in keys:
+            v = self.host[k]
+            arr[k] = gen.to_f64(v[hs[0]:hs[-1] + 1] if k in ("A", "D") else sl(v))
+        nl = len(bs) * len(hs)
+        t0 = time.perf_counter()
+        if self.mimo:
+            for k in ("Wx", "Wy"):
+                arr[k] = gen.to_f64(self.host[k][hs[0]:hs[-1] + 1])
+            _, used = oracle.mimo_loop(**arr, nthreads=threads, return_threads=True)
+        else:
+            _, used = oracle.siso_loop(**arr, nthreads=threads, return_threads=True)
+        dt = time.perf_counter() - t0
+        return nl, dt, used
+
+
+def run_cpu_baseline(w, target_s=10.0):
+    """Time the oracle as it stands on the host cores on a bounded sample of
+    lanes; tokens/s are scaled to whole (b, t) tokens of all heads."""
+    cores = os.cpu_count() or 1
+    H = w.c["nheads"]
+    total_lanes = w.c["batch"] * H
+    n = min(total_lanes, max(1, cores))
+    nl, dt, used = w.oracle_sample(n, cores)
+    if dt < target_s / 4 and nl < total_lanes:
+        n = int(min(total_lanes, nl * max(1.0, target_s / max(dt, 1e-3))))
+        n = max(H, (n // H) * H)
+        nl, dt, used = w.oracle_sample(n, cores)
+    tokens = nl * w.c["seqlen"] / H
+    return {"value": tokens / dt, "unit": UNIT, "cores": int(used), "kind": "oracle",
+            "sample": "%d of %d (b,h) lanes x %d tokens, fp64 C loop, %.1f s wall"
+                      % (nl, total_lanes, w.c["seqlen"], dt)}
+
+
+# ---------------------------------------------------------------------------
+# the two arms
+# ---------------------------------------------------------------------------
+def run_ours(args, world, rank, local):
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist = init_dist(world, "nccl")
+    from state_space_lm_b200 import build, m3
+    if not os.path.exists(build.LIB):
+        raise SystemExit("CUDA library not built: run python -m state_space_lm_b200.build")
+    w = ScanWorkload(args.config, device)
+    stream = torch.cuda.current_stream(device)
+
+    for _ in range(args.warmup):
+        w.step()
+    torch.cuda.synchronize(device)
+
+    # ---- device-timed region: K steps, inputs resident in HBM ----
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    n0 = m3.launch_count()
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            evs[i][0].record(stream)
+            w.step()
+            evs[i][1].record(stream)
+        stop.record(stream)
+        torch.cuda.synchronize(device)
+    launches = m3.launch_count() - n0
+    if dist is not None:
+        dist.barrier()
+    elapsed = start.elapsed_time(stop) / 1e3
+    kernel_s = statistics.mean(a.elapsed_time(b) for a, b in evs) / 1e3
+    value, tmax, units = aggregate(elapsed, w.units * args.steps, dist, device)
+
+    # ---- end to end through the C ABI with host buffers ----
+    pinned = {k: v.pin_memory() for k, v in w.host.items() if isinstance(v, torch.Tensor)}
+    hout = tuple(torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in w.out)
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = sum(o.numel() * o.element_size() for o in hout)
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        for k, v in pinned.items():
+            w.dev[k].copy_(v, non_blocking=True)
+        w.step()
+        for o, ho in zip(w.out, hout):
+            ho.copy_(o, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(device)
+    if dist is not None:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_val, _, _ = aggregate(e0.elapsed_time(e1) / 1e3, w.units * e2e_steps, dist, device)
+
+    peaks, peak_kind = load_peaks()
+    achieved = w.bytes / kernel_s / 1e9
+    tr = traffic_record(w.kernel, w.srcs)
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": (tr["dram_bytes_per_launch"] if tr else None),
+            "kernel": w.kernel, "algorithmic_bytes": w.bytes,
+            "kernel_ms": round(kernel_s * 1e3, 4),
+            "tensor_tflops": round(w.flops / kernel_s / 1e12, 2),
+            "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
+            else "fallback 6.65 TB/s"}
+
+    line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tmax / args.steps * 1e3, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.c["dtype"],
+            "data": "synthetic (seeded; shapes of the pages' 434M-class layers)",
+            "config": dict(w.config(), parallelism="replicas x%d (independent lanes, no collective)" % world),
+            "roofline": roof,
+            "e2e": {"value": round(e2e_val, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "clocks": clk.report(), "gpu_launches": int(launches)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = run_cpu_baseline(w)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args, world, rank):
+    """The oracle arm: fp64 CPU loop on the host cores, a bounded sample of the
+    workload per step.  Under torchrun only rank 0 runs it."""
+    if rank != 0:
+        return
+    import oracle
+    oracle.build_oracle()
+    w = ScanWorkload.__new__(ScanWorkload)
+    w.c = dict(gen.CONFIGS[args.config])
+    w.idx = args.config
+    w.host = gen.config_inputs(args.config)
+    w.host.pop("generator")
+    w.mimo = w.c["rank"] > 1
+    cores = os.cpu_count() or 1
+    H = w.c["nheads"]
+    total_lanes = w.c["batch"] * H
+    n = min(total_lanes, max(H, (cores // H) * H if cores >= H else H))
+    for _ in range(args.warmup):
+        w.oracle_sample(n, cores)
+    times = []
+    used = cores
+    for _ in range(args.steps):
+        nl, dt, used = w.oracle_sample(n, cores)
+        times.append(dt)
+    tokens = nl * w.c["seqlen"] / H
+    el = sum(times)
+    value = tokens * args.steps / el
+    sample = "%d of %d (b,h) lanes x %d tokens per step, fp64 C loop" % (nl, total_lanes, w.c["seqlen"])
+    c = w.c
+    line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": c["name"], "batch": c["batch"], "seqlen": c["seqlen"],
+                       "nheads": c["nheads"], "headdim": c["headdim"], "dstate": c["dstate"],
+                       "rank": c["rank"], "chunk": c["chunk"]},
+            "impl": "reference",
+            "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": int(used), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=1, choices=[0, 1, 2, 3])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+    else:
+        run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()
