@@ -53,7 +53,8 @@ typedef enum {
     M3_ERR_INVALID_ARG = 1,  /* null required pointer, bad size, odd dstate, misalignment */
     M3_ERR_UNSUPPORTED = 2,  /* valid but outside this build's limits (see m3_limits)    */
     M3_ERR_WORKSPACE = 3,    /* workspace missing or smaller than m3_workspace_bytes()   */
-    M3_ERR_CUDA = 4          /* a kernel launch failed                                   */
+    M3_ERR_CUDA = 4,         /* a kernel launch failed                                   */
+    M3_ERR_TIMEOUT = 5       /* a bounded wait inside a kernel gave up (m3_device_error) */
 } m3_status;
 
 typedef enum { M3_F32 = 0, M3_BF16 = 1 } m3_dtype;
@@ -171,6 +172,16 @@ size_t m3_workspace_bytes(int which, m3_dims d, m3_dtype dtype);
 
 /* Static description of a status code (never NULL). */
 const char *m3_status_string(m3_status s);
+
+/* Device-side error report.  The tensor-core kernels bound every internal
+ * wait (about one second); a wait that runs out makes the kernel record the
+ * site, stop issuing work, drain what it has in flight and return, leaving
+ * its outputs undefined.  This call synchronises `stream`, returns
+ * M3_ERR_TIMEOUT if any kernel recorded such an error since the last call
+ * (and clears it), M3_ERR_CUDA if the stream reports a CUDA error, else
+ * M3_OK.  When `site` is not NULL it receives the recorded wait site (0 when
+ * none).  It is the one entry point that synchronises. */
+m3_status m3_device_error(void *stream, int *site);
 
 /* Number of kernels the library has enqueued since it was loaded (host-side
  * counter, incremented once per launch; used to count launches in a timed

@@ -90,6 +90,7 @@ m3_status chunked_common(const void *x, const float *dt, const float *A, const f
     const int q = scan_simt_chunk(d.headdim, d.dstate, R, d.chunk);
     if (q < 1) return M3_ERR_UNSUPPORTED;
     if (d.batch == 0) return M3_OK;
+    if (d.seqlen > ((int64_t)1 << 30)) return M3_ERR_UNSUPPORTED;
 
     ScanArgs a;
     a.x = x; a.B = B; a.C = C;
@@ -98,8 +99,10 @@ m3_status chunked_common(const void *x, const float *dt, const float *A, const f
     a.nrm = nrm;
     a.y = y; a.h_out = h_final; a.prevBx_out = prevBx_final; a.angle_out = angle_final;
     a.Bt = d.batch; a.T = d.seqlen; a.H = d.nheads; a.P = d.headdim; a.N = d.dstate; a.R = R;
-    a.Q = q;
     a.mimo_layout = mimo ? 1 : 0;
+    a.Q = (int)d.chunk;
+    if (scan_tc_supported(a, dtype)) return launched(launch_scan_tc(a, (cudaStream_t)stream));
+    a.Q = q;
     return launched(launch_scan_simt(a, dtype, (cudaStream_t)stream));
 }
 
@@ -118,8 +121,17 @@ const char *m3_status_string(m3_status s) {
         case M3_ERR_UNSUPPORTED: return "M3_ERR_UNSUPPORTED: sizes outside this build's limits";
         case M3_ERR_WORKSPACE: return "M3_ERR_WORKSPACE: workspace missing or too small";
         case M3_ERR_CUDA: return "M3_ERR_CUDA: a kernel launch failed";
+        case M3_ERR_TIMEOUT: return "M3_ERR_TIMEOUT: a bounded wait inside a kernel gave up";
     }
     return "unknown m3_status";
+}
+
+m3_status m3_device_error(void *stream, int *site) {
+    const int e = scan_tc_error_and_clear((cudaStream_t)stream);
+    if (site) *site = e > 0 ? e : 0;
+    if (e < 0) return M3_ERR_CUDA;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return M3_ERR_CUDA;
+    return e ? M3_ERR_TIMEOUT : M3_OK;
 }
 
 size_t m3_workspace_bytes(int which, m3_dims d, m3_dtype dtype) {

@@ -72,6 +72,10 @@ cudaError_t launch_scan_simt(const ScanArgs &a, m3_dtype dt, cudaStream_t s);
 size_t scan_simt_smem_bytes(int64_t P, int64_t N, int64_t R, int Q);
 int scan_simt_chunk(int64_t P, int64_t N, int64_t R, int64_t chunk);
 cudaError_t launch_decode(const DecodeArgs &a, m3_dtype dt, cudaStream_t s);
+// tensor-core SISO scan (bf16, headdim 64, dState 128, chunk 64)
+bool scan_tc_supported(const ScanArgs &a, m3_dtype dt);
+cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s);
+int scan_tc_error_and_clear(cudaStream_t s);
 
 // Launch counter shared by all launchers.
 void count_launch(int n = 1);

@@ -13,7 +13,7 @@ import torch
 
 from .build import LIB
 
-M3_OK, M3_ERR_INVALID_ARG, M3_ERR_UNSUPPORTED, M3_ERR_WORKSPACE, M3_ERR_CUDA = range(5)
+M3_OK, M3_ERR_INVALID_ARG, M3_ERR_UNSUPPORTED, M3_ERR_WORKSPACE, M3_ERR_CUDA, M3_ERR_TIMEOUT = range(6)
 M3_F32, M3_BF16 = 0, 1
 M3_WS_SISO, M3_WS_MIMO = 0, 1
 
@@ -22,7 +22,7 @@ _DTYPE = {torch.float32: M3_F32, torch.bfloat16: M3_BF16}
 ABI_FUNCTIONS = (
     "m3_get_limits", "m3_discretize", "m3_rope_bc", "m3_siso_chunked_fwd",
     "m3_mimo_chunked_fwd", "m3_step_decode", "m3_workspace_bytes", "m3_status_string",
-    "m3_launch_count",
+    "m3_launch_count", "m3_device_error",
 )
 
 
@@ -75,6 +75,8 @@ def lib():
     L.m3_workspace_bytes.argtypes = [ctypes.c_int, Dims, ctypes.c_int]
     L.m3_launch_count.restype = ctypes.c_uint64
     L.m3_launch_count.argtypes = []
+    L.m3_device_error.restype = ctypes.c_int
+    L.m3_device_error.argtypes = [_VP, ctypes.POINTER(ctypes.c_int)]
     L.m3_discretize.restype = ctypes.c_int
     L.m3_discretize.argtypes = [_VP, _VP, _VP, Dims, _VP, _VP, _VP, _VP]
     L.m3_rope_bc.restype = ctypes.c_int
@@ -101,6 +103,15 @@ def status_string(status):
 
 def launch_count():
     return int(lib().m3_launch_count())
+
+
+def device_error(stream=None, with_site=False):
+    """Synchronise the stream and return the device-side error status
+    (M3_OK, or M3_ERR_TIMEOUT when a bounded wait inside a kernel gave up);
+    with_site=True also returns the recorded wait site."""
+    site = ctypes.c_int(0)
+    st = int(lib().m3_device_error(_stream(stream), ctypes.byref(site)))
+    return (st, site.value) if with_site else st
 
 
 def limits():

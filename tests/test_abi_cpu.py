@@ -34,7 +34,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_status_strings_and_limits(L):
-    for code in range(5):
+    for code in range(6):
         s = m3.status_string(code)
         assert s.startswith("M3_")
     assert "unknown" in m3.status_string(99)

@@ -133,10 +133,28 @@ def test_siso_bf16_layer_shape(T, chunk):
     assert max(errs) <= 2e-2, errs
 
 
+@pytest.mark.parametrize("dt_shift,T", [(3.0, 200), (1.0, 130), (-6.0, 256)])
+def test_siso_bf16_decay_regimes(dt_shift, T):
+    # dt_shift 3: every chunk's log-decay range exceeds 60 (exact-mask path);
+    # 1: a mix; -6: almost no decay (long memory)
+    inp = gen.scan_inputs(2, T, 2, 64, 128, dtype=BF16, dt_shift=dt_shift, seed=int(50 + T))
+    errs = _siso_check(inp, 64, with_state=True, seed=T)
+    assert max(errs) <= 2e-2, errs
+    assert m3.device_error() == m3.M3_OK
+
+
 def test_siso_bf16_norm_bias():
     inp = gen.scan_inputs(1, 130, 2, 64, 128, dtype=BF16, seed=41, bcnorm=True)
     errs = _siso_check(inp, 64)
     assert max(errs) <= 2e-2, errs
+
+
+@pytest.mark.parametrize("T", [1, 2, 31, 32, 33, 63, 64, 65, 127, 129, 1000])
+def test_siso_bf16_ragged_lengths(T):
+    inp = gen.scan_inputs(3, T, 2, 64, 128, dtype=BF16, seed=90 + T)
+    errs = _siso_check(inp, 64, with_state=(T % 2 == 1), seed=T)
+    assert max(errs) <= 2e-2, errs
+    assert m3.device_error() == m3.M3_OK
 
 
 def test_siso_empty_sequence_passes_state_through():
