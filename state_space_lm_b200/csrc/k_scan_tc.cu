@@ -1,5 +1,5 @@
-// k_scan_tc.cu -- SISO chunked forward of the Mamba-3 scan on the sm_100a
-// tensor cores (bf16 inputs, headdim 64, dState 128, chunk 64).
+// k_scan_tc.cu -- chunked forward of the Mamba-3 scan, SISO and rank-R MIMO,
+// on the sm_100a tensor cores (bf16 inputs, headdim 64, dState 128).
 //
 // The method is the chunked form of the trapezoidal recurrence (dotLLM pull
 // request, "Stage A: Mamba3SelectiveScan" and the streaming-decode comment:
@@ -14,9 +14,16 @@
 //   g_out = e^{cum_end} g_in + sum_s e^{cum_end - cum_s} w_s Bbar_s x_s^T
 // with M[t,s] = e^{cum_t - cum_s} w_s (s < t), gamma_t (s = t).
 //
-// One CTA owns one (b, h) lane and walks its chunks in order.  Per chunk four
-// UMMAs (tcgen05.mma kind::f16, bf16 operands in shared memory, fp32
-// accumulators in tensor memory):
+// MIMO (rank R, TorchMamba README "Math notes": rank-R update on a shared
+// (N,P) state; App. C per-head expand/contract vectors) is the same chunked
+// form with R rows (t, r) per token: X_{t,r} = W_x[r] x_t, the mask depends on
+// the tokens only, the state update sums over all rows, and
+// y_t = sum_r W_y[r] Y_{t,r} + D x_t.  A chunk always holds 64 rows, i.e.
+// 64 / R tokens, so the UMMA shapes below are the same for every R.
+//
+// One CTA owns one (b, h) lane -- or one segment of it, see below -- and
+// walks its chunks in order.  Per chunk four UMMAs (tcgen05.mma kind::f16,
+// bf16 operands in shared memory, fp32 accumulators in tensor memory):
 //   D1 = Cbar . Bsc^T             scores            M=64  N=64  K=128
 //   D3 = Cbar . g_in              inter-chunk term  M=64  N=64  K=128
 //   D2 = S' . X                   intra-chunk term  M=64  N=64  K=64
@@ -29,11 +36,20 @@
 // such a chunk uses Bsc = Bbar, an exact per-element mask
 // e^{cum_t - cum_s} w_s and Xw = e^{cum_end - cum_s} w_s x_s instead.
 //
-// Warp roles (12 warps): 0 TMA producer, 1 MMA issuer (and TMEM owner),
-// 2 per-token coefficients, 3 Xw scaling, 4-7 rotation (QkNorm, bias, RoPE),
-// 8-11 epilogue (TMEM -> masked scores, outputs, fp32 state in registers).
-// Every wait is bounded: past ~1 s the kernel records an error, stops issuing
-// work, drains what it has in flight and returns.
+// Long sequences over few lanes are cut into segments of whole chunks: a
+// state-only pass computes every segment's end state from a zero start in
+// its own angle frame, a small combine kernel chains the segments, and the
+// full pass then runs all segments in parallel from their entering states.
+//
+// Warp roles (19 warps): 0 TMA producer, 1 MMA issuer (and TMEM owner),
+// 2 per-token coefficients, 3-10 rotation (QkNorm, bias, RoPE; each thread 4
+// pairs x 4 tokens with 16-byte shared-memory accesses) and the Xw scaling,
+// 11-18 epilogue (two warps per TMEM lane quarter, each owning 32 of the 64
+// columns: masked scores, fp32 state in registers, outputs).  Inputs stream
+// through two rings: B, C, theta (released once rotated) and x (released
+// once the outputs are written).  Every wait is bounded: past ~1 s the kernel
+// records an error, stops issuing work, drains what it has in flight and
+// returns.
 #include <cuda.h>
 
 #include "m3_internal.cuh"
@@ -42,52 +58,92 @@ namespace m3 {
 namespace tc {
 
 constexpr int Q = 64, P = 64, N = 128, NP2 = 64;
-constexpr int THREADS = 384;
-constexpr int W_TMA = 0, W_MMA = 1, W_COEF = 2, W_XW = 3, W_PREP0 = 4, W_EPI0 = 8;
+constexpr int NWARPS = 19, THREADS = NWARPS * 32;
+constexpr int W_TMA = 0, W_MMA = 1, W_COEF = 2, W_PREP0 = 3, NPREP = 8, W_EPI0 = 11;
+constexpr int PREP_THREADS = NPREP * 32;          // 256
+constexpr int EPI_THREADS = 256;                  // two warps per TMEM lane quarter
 
 // ---- shared-memory map (bytes from a 1024-aligned base) ------------------
-constexpr int SZ_X = Q * P * 2;          // 8 KB, bf16, 128B-swizzled (TMA)
-constexpr int SZ_BC = Q * N * 2;         // 16 KB, bf16, row-major (TMA)
-constexpr int SZ_TH = Q * NP2 * 4;       // 16 KB, fp32, row-major (TMA)
-constexpr int STAGE = SZ_X + 2 * SZ_BC + SZ_TH;
-constexpr int OFF_STAGE0 = 0;
-constexpr int OFF_BSC = 2 * STAGE;               // [2 atoms][Q][64] bf16, SW128
-constexpr int OFF_CB = OFF_BSC + Q * N * 2;      // [2 atoms][Q][64] bf16, SW128
-constexpr int OFF_SP = OFF_CB + Q * N * 2;       // [Q][Q] bf16, SW128
-constexpr int OFF_XW = OFF_SP + Q * Q * 2;       // [Q][P] bf16, SW128
-constexpr int OFF_GB = OFF_XW + Q * P * 2;       // [N][P] bf16, SW128
-constexpr int OFF_YT = OFF_GB + N * P * 2;       // [Q][P] bf16, SW128
-constexpr int OFF_COEF = OFF_YT + Q * P * 2;
-// per-chunk coefficient buffer (double-buffered), floats
+// Rank R: a chunk holds QT = Q / R tokens and Q rows (token, rank) of B and C;
+// the x, theta and output tiles have QT rows, and MIMO (R > 1) adds the
+// rank-expanded X_r = W_x[r] * x, the W_x / W_y vectors and R rows of the
+// last token's rotated B.
+constexpr int NB = 2, NX = 3, NC = 4;             // ring depths: B/C/theta, x, coefficients
+constexpr int SZ_BC = Q * N * 2;                  // 16 KB, bf16, row-major (TMA)
+constexpr int SZ_SP = Q * Q * 2, SZ_GB = N * P * 2;
+// per-chunk coefficient buffer (a ring of NC), floats; per token of the chunk
 constexpr int CF_W = 0, CF_GAM = Q, CF_E = 2 * Q, CF_R = 3 * Q, CF_EC = 4 * Q, CF_XS = 5 * Q,
               CF_C2 = 6 * Q, CF_DT = 7 * Q, CF_SCAL = 8 * Q, CF_FLOATS = 8 * Q + 8;
-constexpr int OFF_BLAST = OFF_COEF + 2 * CF_FLOATS * 4;  // fp32 [N]
-constexpr int OFF_PHIC = OFF_BLAST + N * 4;              // fp32 [NP2] running angle
-constexpr int OFF_PART = OFF_PHIC + NP2 * 4;             // fp32 [NP2] half-chunk angle sums
-constexpr int OFF_INV = OFF_PART + NP2 * 4;              // fp32 [2][Q] QkNorm inverse RMS
-constexpr int OFF_BAR = OFF_INV + 2 * Q * 4;             // mbarriers
-constexpr int NBAR = 18;
-constexpr int OFF_MISC = OFF_BAR + NBAR * 8;             // tmem slot, abort flag
-constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;         // + alignment slack
+template <int R>
+struct Lay {
+    static constexpr int QT = Q / R;
+    static constexpr int SZ_X = QT * P * 2;                   // bf16, 128B-swizzled (TMA)
+    static constexpr int SZ_TH = QT * NP2 * 4;                // fp32, row-major (TMA)
+    static constexpr int SZ_BCT = 2 * SZ_BC + SZ_TH;          // one B/C/theta stage
+    static constexpr int OFF_BCT = 0;                         // NB x [B | C | theta]
+    static constexpr int OFF_X = OFF_BCT + NB * SZ_BCT;       // NX x [QT][P]
+    static constexpr int OFF_BSC = OFF_X + NX * SZ_X;         // [2 atoms][Q rows][64] bf16, SW128
+    static constexpr int OFF_CB = OFF_BSC + Q * N * 2;        // [2 atoms][Q rows][64] bf16, SW128
+    static constexpr int OFF_SP = OFF_CB + Q * N * 2;         // [Q][Q] bf16, SW128
+    static constexpr int OFF_XW = OFF_SP + SZ_SP;             // [Q rows][P] bf16, SW128
+    static constexpr int OFF_XR = OFF_XW + Q * P * 2;         // [Q rows][P] bf16, SW128 (R > 1)
+    static constexpr int OFF_GB = OFF_XR + (R > 1 ? Q * P * 2 : 0);   // 2 x [N][P] bf16, SW128
+    static constexpr int OFF_YT = OFF_GB + 2 * SZ_GB;         // [QT][P] bf16, SW128
+    static constexpr int OFF_COEF = OFF_YT + ((QT * P * 2 + 1023) / 1024) * 1024;
+    static constexpr int OFF_BLAST = OFF_COEF + NC * CF_FLOATS * 4;  // fp32 [R][N]
+    static constexpr int OFF_WXY = OFF_BLAST + R * N * 4;            // fp32 [2][R][P] (R > 1)
+    static constexpr int OFF_PHIC = OFF_WXY + (R > 1 ? 2 * R * P * 4 : 0);  // fp32 [NP2]
+    static constexpr int OFF_PART = OFF_PHIC + NP2 * 4;       // fp32 [16][NP2] token-group angle sums
+    static constexpr int OFF_INV = OFF_PART + 16 * NP2 * 4;   // fp32 [2][Q] QkNorm inverse RMS
+    static constexpr int OFF_BAR = OFF_INV + 2 * Q * 4;       // mbarriers
+};
 
 // barrier indices
 enum {
-    B_FULL0 = 0, B_FULL1, B_EMPTY0, B_EMPTY1, B_CFULL0, B_CFULL1, B_CEMPTY0, B_CEMPTY1,
-    B_OPSREADY, B_OPSFREE, B_SFULL, B_STAKEN, B_SPFULL, B_YFULL, B_YTAKEN, B_STFULL, B_STTAKEN,
-    B_DRAIN
+    B_BFULL = 0,                    // NB: B/C/theta stage loaded (TMA)
+    B_BEMPTY = B_BFULL + NB,        // NB: stage rotated
+    B_XFULL = B_BEMPTY + NB,        // NX: x tile loaded (TMA)
+    B_XEMPTY = B_XFULL + NX,        // NX: Xw built, intra UMMA done, outputs written
+    B_CFULL = B_XEMPTY + NX,        // NC: coefficients ready
+    B_CEMPTY = B_CFULL + NC,        // NC: coefficients consumed
+    B_OPSREADY = B_CEMPTY + NC,     // rotated operands and Xw written
+    B_OPSFREE,                      // UMMAs reading them are done
+    B_SFULL, B_STAKEN, B_SPFULL,    // scores in TMEM / read / masked scores written
+    B_YFULL, B_YTAKEN,              // output accumulators done / read
+    B_STFULL, B_STTAKEN,            // chunk state done / folded into the state
+    B_DRAIN,
+    NBAR
 };
+template <int R>
+constexpr int smem_bytes() { return Lay<R>::OFF_BAR + NBAR * 8 + 16 + 1024; }   // + misc + alignment slack
+static_assert(smem_bytes<1>() <= 227 * 1024 && smem_bytes<2>() <= 227 * 1024 && smem_bytes<4>() <= 227 * 1024,
+              "shared memory budget");
 
 constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t COL_D1 = 0, COL_D2 = 64, COL_D3 = 128, COL_D4 = 192;
 
 struct TcArgs {
     const float *dt, *A, *lam, *D;
+    const float *Wx, *Wy;  // MIMO expand / contract vectors (H, R, P), NULL = ones
     const float *h0, *prevBx0, *angle0;
     NormArgs nrm;
     float *h_out, *prevBx_out, *angle_out;
     int64_t Bt, T, H;
+    int64_t seg_len;   // tokens per segment (a multiple of Q); one segment covers the whole sequence
+    int nseg;          // segments per lane
+    float *ws;         // segment slots (nseg > 1)
     int *err;
 };
+
+// Workspace slot of one (lane, segment j < nseg-1), in floats:
+//   [0, N*P)        after the state-only pass: the segment's end state from a
+//                   zero start, in the segment's own angle frame; after the
+//                   combine pass: the state entering segment j+1
+//   [N*P, +N/2)     angle increment over segment j
+//   [+N/2, +N/2)    angle entering segment j+1
+//   [N*P + N]       product of alpha over segment j
+constexpr int SLOT_G = 0, SLOT_PHIL = N * P, SLOT_PHIN = N * P + NP2, SLOT_E = N * P + N;
+constexpr int SLOT_FLOATS = N * P + N + 4;
 
 // ---- PTX wrappers ---------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -107,6 +163,16 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(10000000u)   // suspend up to 10 ms instead of spinning
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_try_spin(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
         "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
         : "=r"(ok)
         : "r"(bar), "r"(parity)
@@ -115,6 +181,22 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 }
 
 constexpr long long WAIT_LIMIT_CYCLES = 2000000000LL;  // ~1 s at 1.9 GHz
+
+// Bounded wait without the suspend hint (for the single MMA-issuing thread).
+__device__ __forceinline__ bool wait_bar_spin(uint32_t bar, uint32_t parity, volatile int *abort_flag, int *err,
+                                              int site) {
+    if (mbar_try_spin(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_spin(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+            *abort_flag = 1;
+            atomicCAS(err, 0, site);
+            return false;
+        }
+    }
+}
 
 // Bounded wait on an mbarrier phase.  Returns false when the kernel is
 // aborting (this wait timed out, or another thread's did).
@@ -162,6 +244,25 @@ __device__ __forceinline__ void tma_store4(const CUtensorMap *map, int c0, int c
                  "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(src)
                  : "memory");
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void tma_load5(uint32_t dst, const CUtensorMap *map, int c0, int c1, int c2, int c3, int c4,
+                                          uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, %6}], "
+        "[%7];" ::"r"(dst),
+        "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void tma_prefetch5(const CUtensorMap *map, int c0, int c1, int c2, int c3, int c4) {
+    asm volatile("cp.async.bulk.prefetch.tensor.5d.L2.global [%0, {%1, %2, %3, %4, %5}];" ::"l"(map), "r"(c0),
+                 "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+                 : "memory");
+}
+// Pull a box of the tensor into L2 ahead of its load (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch4(const CUtensorMap *map, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global [%0, {%1, %2, %3, %4}];" ::"l"(map), "r"(c0), "r"(c1),
+                 "r"(c2), "r"(c3)
+                 : "memory");
 }
 __device__ __forceinline__ void tma_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
@@ -231,29 +332,69 @@ __device__ __forceinline__ void sincos_rr(float x, float *s, float *c) {
     __sincosf(r, s, c);
 }
 
+// SO (state only): the first pass over all but the last segment of each lane;
+// it loads x, B, theta (no C), runs only the chunk-state UMMA, starts from a
+// zero state in the segment's own angle frame and writes the segment's end
+// state, angle increment and decay product to its workspace slot.
+template <bool SO, int R>
 __global__ void __launch_bounds__(THREADS, 1)
     k_scan_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
               const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_th,
               const __grid_constant__ CUtensorMap map_y, TcArgs a) {
+    using L = Lay<R>;
+    constexpr int QT = L::QT;                          // tokens per chunk
+    constexpr int TPT = QT / 16;                       // tokens per rotation thread
+    constexpr int OFF_MISC = L::OFF_BAR + NBAR * 8;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, l32 = tid & 31;
-    const int64_t lane_id = blockIdx.x, b = lane_id / a.H, h = lane_id % a.H;
+    const int nsb = SO ? a.nseg - 1 : a.nseg;          // CTAs per lane in this pass
+    const int64_t lane_id = blockIdx.x / nsb, b = lane_id / a.H, h = lane_id % a.H;
+    const int seg = blockIdx.x % nsb;
     const int64_t Tn = a.T, H = a.H;
-    const int nchunks = (int)((Tn + Q - 1) / Q);
-    auto bar = [&](int i) { return sbase + OFF_BAR + 8 * i; };
+    const int64_t t_beg = (int64_t)seg * a.seg_len;
+    const int64_t t_end = (t_beg + a.seg_len < Tn) ? t_beg + a.seg_len : Tn;
+    const int nchunks = (int)((t_end - t_beg + QT - 1) / QT);
+    const bool last_seg = SO ? false : (seg == a.nseg - 1);
+    float *slot_in = (!SO && seg > 0) ? a.ws + ((size_t)lane_id * (a.nseg - 1) + (seg - 1)) * SLOT_FLOATS : nullptr;
+    float *slot_out = SO ? a.ws + ((size_t)lane_id * (a.nseg - 1) + seg) * SLOT_FLOATS : nullptr;
+    auto bar = [&](int i) { return sbase + L::OFF_BAR + 8 * i; };
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_MISC + 4);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC);
-    float *coef0 = reinterpret_cast<float *>(sm + OFF_COEF);
-    float *blast = reinterpret_cast<float *>(sm + OFF_BLAST);
-    float *phic = reinterpret_cast<float *>(sm + OFF_PHIC);
-    float *part = reinterpret_cast<float *>(sm + OFF_PART);
-    float *inv = reinterpret_cast<float *>(sm + OFF_INV);
+    float *coef0 = reinterpret_cast<float *>(sm + L::OFF_COEF);
+    float *blast = reinterpret_cast<float *>(sm + L::OFF_BLAST);
+    float *wxs = reinterpret_cast<float *>(sm + L::OFF_WXY);            // [R][P] (R > 1)
+    float *wys = wxs + R * P;                                            // [R][P] (R > 1)
+    float *phic = reinterpret_cast<float *>(sm + L::OFF_PHIC);
+    float *part = reinterpret_cast<float *>(sm + L::OFF_PART);
+    float *inv = reinterpret_cast<float *>(sm + L::OFF_INV);
 
     if (tid == 0) {
-        const uint32_t counts[NBAR] = {1, 1, 4, 4, 1, 1, 3, 3, 2, 1, 1, 4, 4, 1, 4, 1, 4, 1};
-        for (int i = 0; i < NBAR; i++) mbar_init(bar(i), counts[i]);
+        for (int i = 0; i < NB; i++) {
+            mbar_init(bar(B_BFULL + i), 1);
+            mbar_init(bar(B_BEMPTY + i), 1);
+        }
+        // x tiles are released by the Xw builder, the intra UMMA and the output
+        // writer (state-only pass: the Xw builder alone)
+        for (int i = 0; i < NX; i++) {
+            mbar_init(bar(B_XFULL + i), 1);
+            mbar_init(bar(B_XEMPTY + i), SO ? 1 : 3);
+        }
+        for (int i = 0; i < NC; i++) {
+            mbar_init(bar(B_CFULL + i), 1);
+            mbar_init(bar(B_CEMPTY + i), 2);
+        }
+        mbar_init(bar(B_OPSREADY), 1);
+        mbar_init(bar(B_OPSFREE), 1);
+        mbar_init(bar(B_SFULL), 1);
+        mbar_init(bar(B_STAKEN), 8);
+        mbar_init(bar(B_SPFULL), 8);
+        mbar_init(bar(B_YFULL), 1);
+        mbar_init(bar(B_YTAKEN), 8);
+        mbar_init(bar(B_STFULL), 1);
+        mbar_init(bar(B_STTAKEN), 8);
+        mbar_init(bar(B_DRAIN), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&map_x) : "memory");
@@ -268,7 +409,17 @@ __global__ void __launch_bounds__(THREADS, 1)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    if (tid < NP2) phic[tid] = a.angle0 ? a.angle0[lane_id * NP2 + tid] : 0.f;
+    if (tid < NP2) {
+        float p0 = 0.f;                                   // state-only: the segment's own frame
+        if (!SO) p0 = slot_in ? slot_in[SLOT_PHIN + tid] : (a.angle0 ? a.angle0[lane_id * NP2 + tid] : 0.f);
+        phic[tid] = p0;
+    }
+    if (R > 1) {
+        for (int k = tid; k < R * P; k += THREADS) {
+            wxs[k] = a.Wx ? a.Wx[h * R * P + k] : 1.f;
+            wys[k] = a.Wy ? a.Wy[h * R * P + k] : 1.f;
+        }
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -277,24 +428,55 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (warp == W_TMA) {
         // ------------------------------------------------------------ producer
         if (l32 == 0) {
+            // B and C of a chunk: rows (token, rank) -- a 4-D box (N, H, T, Bt)
+            // for SISO, a 5-D box (N, R, H, T, Bt) for MIMO
+            auto load_bc = [&](uint32_t dst, const CUtensorMap *m, int t0, uint32_t fb) {
+                if (R == 1) tma_load4(dst, m, 0, (int)h, t0, (int)b, fb);
+                else tma_load5(dst, m, 0, 0, (int)h, t0, (int)b, fb);
+            };
+            auto prefetch_bc = [&](const CUtensorMap *m, int t0) {
+                if (R == 1) tma_prefetch4(m, 0, (int)h, t0, (int)b);
+                else tma_prefetch5(m, 0, 0, (int)h, t0, (int)b);
+            };
+            // L2 prefetch runs PFD chunks ahead of the shared-memory rings, so
+            // a load issued when a stage frees up finds its data in L2
+            constexpr int PFD = 3;
+            auto prefetch = [&](int c) {
+                if (c >= nchunks) return;
+                const int t0 = (int)(t_beg + (int64_t)c * QT);
+                prefetch_bc(&map_b, t0);
+                if (!SO) prefetch_bc(&map_c, t0);
+                tma_prefetch4(&map_th, 0, (int)h, t0, (int)b);
+                tma_prefetch4(&map_x, 0, (int)h, t0, (int)b);
+            };
+            for (int c = 1; c < PFD; c++) prefetch(c);
             int issued = 0;
             for (int c = 0; c < nchunks; c++) {
-                const int s = c & 1, k = c >> 1;
-                if (k > 0 && !wait_bar(bar(B_EMPTY0 + s), (k - 1) & 1, abort_flag, a.err, 1)) break;
-                const uint32_t st = sbase + OFF_STAGE0 + s * STAGE;
-                const uint32_t fb = bar(B_FULL0 + s);
-                mbar_expect_tx(fb, STAGE);
-                const int t0 = c * Q;
-                tma_load4(st, &map_x, 0, (int)h, t0, (int)b, fb);
-                tma_load4(st + SZ_X, &map_b, 0, (int)h, t0, (int)b, fb);
-                tma_load4(st + SZ_X + SZ_BC, &map_c, 0, (int)h, t0, (int)b, fb);
-                tma_load4(st + SZ_X + 2 * SZ_BC, &map_th, 0, (int)h, t0, (int)b, fb);
+                const int sb = c % NB, kb = c / NB, sx = c % NX, kx = c / NX;
+                const int t0 = (int)(t_beg + (int64_t)c * QT);
+                prefetch(c + PFD);
+                if (kb > 0 && !wait_bar(bar(B_BEMPTY + sb), (kb - 1) & 1, abort_flag, a.err, 1)) break;
+                const uint32_t st = sbase + L::OFF_BCT + sb * L::SZ_BCT;
+                const uint32_t fb = bar(B_BFULL + sb);
+                mbar_expect_tx(fb, SO ? SZ_BC + L::SZ_TH : L::SZ_BCT);
+                load_bc(st, &map_b, t0, fb);
+                if (!SO) load_bc(st + SZ_BC, &map_c, t0, fb);
+                tma_load4(st + 2 * SZ_BC, &map_th, 0, (int)h, t0, (int)b, fb);
+                if (kx > 0 && !wait_bar(bar(B_XEMPTY + sx), (kx - 1) & 1, abort_flag, a.err, 2)) break;
+                const uint32_t xb = bar(B_XFULL + sx);
+                mbar_expect_tx(xb, L::SZ_X);
+                tma_load4(sbase + L::OFF_X + sx * L::SZ_X, &map_x, 0, (int)h, t0, (int)b, xb);
                 issued = c + 1;
             }
             // never leave loads in flight into shared memory at exit
-            for (int c = (issued > 2 ? issued - 2 : 0); c < issued; c++) {
+            for (int c = (issued > NX ? issued - NX : 0); c < issued; c++) {
                 const long long t0 = clock64();
-                while (!mbar_try(bar(B_FULL0 + (c & 1)), (c >> 1) & 1) && clock64() - t0 < WAIT_LIMIT_CYCLES) {
+                while (!mbar_try(bar(B_XFULL + c % NX), (c / NX) & 1) && clock64() - t0 < WAIT_LIMIT_CYCLES) {
+                }
+            }
+            for (int c = (issued > NB ? issued - NB : 0); c < issued; c++) {
+                const long long t0 = clock64();
+                while (!mbar_try(bar(B_BFULL + c % NB), (c / NB) & 1) && clock64() - t0 < WAIT_LIMIT_CYCLES) {
                 }
             }
         }
@@ -304,30 +486,38 @@ __global__ void __launch_bounds__(THREADS, 1)
         const float A2 = a.A[h] * L2E;
         const float UNSAFE2 = 60.f * L2E;
         for (int c = 0; c < nchunks; c++) {
-            const int s = c & 1, k = c >> 1;
-            int ok = 1;
-            if (l32 == 0 && k > 0) ok = wait_bar(bar(B_CEMPTY0 + s), (k - 1) & 1, abort_flag, a.err, 2);
-            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            float *cf = coef0 + s * CF_FLOATS;
-            const int64_t t0 = (int64_t)c * Q;
-            const int L = (int)((Tn - t0) < Q ? (Tn - t0) : Q);
-            float la[2], wv[2], gv[2], dv[2];
+            const int s = c % NC, k = c / NC;
+            // fetch this chunk's dt and lam before waiting for the buffer
+            const int64_t t0 = t_beg + (int64_t)c * QT;
+            const int Lc = (int)((t_end - t0) < QT ? (t_end - t0) : QT);
+            float dl[2], lm[2], dn[2], ln[2];
 #pragma unroll
             for (int u = 0; u < 2; u++) {
                 const int i = l32 + 32 * u;
-                la[u] = wv[u] = gv[u] = dv[u] = 0.f;
-                if (i < L) {
+                dl[u] = lm[u] = dn[u] = 0.f;
+                ln[u] = 1.f;
+                if (i < Lc) {
                     const int64_t bt = (b * Tn + t0 + i) * H + h;
-                    const float dl = a.dt[bt], lm = a.lam[bt];
-                    float sg = 0.f;
-                    if (t0 + i + 1 < Tn) sg = (1.f - a.lam[bt + H]) * a.dt[bt + H];
-                    gv[u] = lm * dl;
-                    wv[u] = gv[u] + sg;
-                    la[u] = dl * A2;
-                    dv[u] = dl;
+                    dl[u] = a.dt[bt];
+                    lm[u] = a.lam[bt];
+                    if (t0 + i + 1 < Tn) {
+                        dn[u] = a.dt[bt + H];
+                        ln[u] = a.lam[bt + H];
+                    }
                 }
             }
-            // inclusive scan of log2(alpha) over the 64 tokens
+            int ok = 1;
+            if (l32 == 0 && k > 0) ok = wait_bar(bar(B_CEMPTY + s), (k - 1) & 1, abort_flag, a.err, 3);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            float *cf = coef0 + s * CF_FLOATS;
+            float la[2], wv[2], gv[2];
+#pragma unroll
+            for (int u = 0; u < 2; u++) {
+                gv[u] = lm[u] * dl[u];
+                wv[u] = gv[u] + (1.f - ln[u]) * dn[u];
+                la[u] = dl[u] * A2;
+            }
+            // inclusive scan of log2(alpha) over the chunk's tokens
 #pragma unroll
             for (int u = 0; u < 2; u++)
 #pragma unroll
@@ -336,161 +526,223 @@ __global__ void __launch_bounds__(THREADS, 1)
                     if (l32 >= o) la[u] += v;
                 }
             la[1] += __shfl_sync(0xffffffffu, la[0], 31);
-            const float cend = __shfl_sync(0xffffffffu, (L - 1) < 32 ? la[0] : la[1], (L - 1) & 31);
+            const float cend = __shfl_sync(0xffffffffu, (Lc - 1) < 32 ? la[0] : la[1], (Lc - 1) & 31);
             float dev = 0.f;
 #pragma unroll
             for (int u = 0; u < 2; u++) {
                 const int i = l32 + 32 * u;
-                if (i >= L) la[u] = cend;
+                if (i >= Lc) la[u] = cend;
                 dev = fmaxf(dev, fabsf(la[u] - cend));
             }
             const bool unsafe = __any_sync(0xffffffffu, dev > UNSAFE2);
 #pragma unroll
             for (int u = 0; u < 2; u++) {
                 const int i = l32 + 32 * u;
-                const float e = exp2f(cend - la[u]);
-                cf[CF_W + i] = wv[u];
-                cf[CF_GAM + i] = gv[u];
-                cf[CF_E + i] = unsafe ? 1.f : e;
-                cf[CF_R + i] = exp2f(la[u] - cend);
-                cf[CF_EC + i] = exp2f(la[u]);
-                cf[CF_XS + i] = unsafe ? e * wv[u] : wv[u];
-                cf[CF_C2 + i] = la[u];
-                cf[CF_DT + i] = dv[u];
+                if (i < QT) {
+                    const float e = exp2f(cend - la[u]);
+                    cf[CF_W + i] = wv[u];
+                    cf[CF_GAM + i] = gv[u];
+                    cf[CF_E + i] = unsafe ? 1.f : e;
+                    cf[CF_R + i] = exp2f(la[u] - cend);
+                    cf[CF_EC + i] = exp2f(la[u]);
+                    cf[CF_XS + i] = unsafe ? e * wv[u] : wv[u];
+                    cf[CF_C2 + i] = la[u];
+                    cf[CF_DT + i] = dl[u];
+                }
             }
             if (l32 == 0) {
                 cf[CF_SCAL + 0] = exp2f(cend);
                 cf[CF_SCAL + 1] = unsafe ? 1.f : 0.f;
-                cf[CF_SCAL + 2] = (float)L;
+                cf[CF_SCAL + 2] = (float)Lc;
             }
             __syncwarp();
-            if (l32 == 0) mbar_arrive(bar(B_CFULL0 + s));
+            if (l32 == 0) mbar_arrive(bar(B_CFULL + s));
         }
-    } else if (warp == W_XW) {
-        // ------------------------------------------------- Xw = diag(xs) . X
-        for (int c = 0; c < nchunks; c++) {
-            const int s = c & 1, k = c >> 1;
-            int ok = 1;
-            if (l32 == 0) {
-                ok = wait_bar(bar(B_FULL0 + s), k & 1, abort_flag, a.err, 3) &&
-                     wait_bar(bar(B_CFULL0 + s), k & 1, abort_flag, a.err, 4) &&
-                     (c == 0 || wait_bar(bar(B_OPSFREE), (c - 1) & 1, abort_flag, a.err, 5));
-            }
-            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            const float *cf = coef0 + s * CF_FLOATS;
-            const uint4 *src = reinterpret_cast<const uint4 *>(sm + OFF_STAGE0 + s * STAGE);
-            uint4 *dst = reinterpret_cast<uint4 *>(sm + OFF_XW);
-#pragma unroll 4
-            for (int v = l32; v < Q * P / 8; v += 32) {
-                const float sc = cf[CF_XS + (v >> 3)];   // 8 vectors per 128-byte row
-                uint4 d = src[v];
-                uint32_t *w = reinterpret_cast<uint32_t *>(&d);
-#pragma unroll
-                for (int q = 0; q < 4; q++) {
-                    const float2 f = unpack_bf16(w[q]);
-                    w[q] = pack_bf16(f.x * sc, f.y * sc);
-                }
-                dst[v] = d;
-            }
-            fence_async_smem();
-            __syncwarp();
-            if (l32 == 0) {
-                mbar_arrive(bar(B_OPSREADY));
-                mbar_arrive(bar(B_EMPTY0 + s));
-                mbar_arrive(bar(B_CEMPTY0 + s));
-            }
-        }
-    } else if (warp >= W_PREP0 && warp < W_PREP0 + 4) {
-        // ----------------------------------- QkNorm + bias + RoPE rotation
-        const int pt = tid - W_PREP0 * 32;         // 0..127
-        const int j = pt & 63, half = pt >> 6;     // pair, token half
+    } else if (warp >= W_PREP0 && warp < W_PREP0 + NPREP) {
+        // --------------- QkNorm + bias + RoPE rotation, then the X operands
+        // thread (j4, tg): pairs 4*j4 .. 4*j4+3 (elements 8*j4 .. 8*j4+7, one
+        // 16-byte chunk) of tokens TPT*tg .. TPT*tg+TPT-1, all ranks of each
+        const int pt = tid - W_PREP0 * 32;         // 0..255
+        const int j4 = pt & 15, tg = pt >> 4;
         const NormArgs nr = a.nrm;
         const bool has_norm = nr.wB || nr.wC;
-        const float wb0 = nr.wB ? nr.wB[2 * j] : 1.f, wb1 = nr.wB ? nr.wB[2 * j + 1] : 1.f;
-        const float wc0 = nr.wC ? nr.wC[2 * j] : 1.f, wc1 = nr.wC ? nr.wC[2 * j + 1] : 1.f;
-        const float bb0 = nr.biasB ? nr.biasB[h * N + 2 * j] : 0.f, bb1 = nr.biasB ? nr.biasB[h * N + 2 * j + 1] : 0.f;
-        const float bc0 = nr.biasC ? nr.biasC[h * N + 2 * j] : 0.f, bc1 = nr.biasC ? nr.biasC[h * N + 2 * j + 1] : 0.f;
-        uint8_t *bsc = sm + OFF_BSC;
-        uint8_t *cb = sm + OFF_CB;
-        // element (row i, n) of the two-atom [n/64][row][64] 128B-swizzled tiles
-        const uint32_t atom = (uint32_t)(j >> 5) * (Q * 128);
-        const int col = (2 * j) & 63;
+        const bool has_bias = nr.biasB || nr.biasC;
+        uint8_t *bsc = sm + L::OFF_BSC;
+        uint8_t *cb = sm + L::OFF_CB;
+        const uint32_t atom = (uint32_t)(j4 >> 3) * (Q * 128);
+        const int chk = j4 & 7;                    // 16-byte chunk within the 128-byte atom row
         for (int c = 0; c < nchunks; c++) {
-            const int s = c & 1, k = c >> 1;
+            const int sb = c % NB, kb = c / NB, sx = c % NX, kx = c / NX, scf = c % NC, kc = c / NC;
             bool fail = false;
             if (pt == 0) {
-                fail = !(wait_bar(bar(B_FULL0 + s), k & 1, abort_flag, a.err, 6) &&
-                         wait_bar(bar(B_CFULL0 + s), k & 1, abort_flag, a.err, 7) &&
-                         (c == 0 || wait_bar(bar(B_OPSFREE), (c - 1) & 1, abort_flag, a.err, 8)));
+                fail = !(wait_bar(bar(B_BFULL + sb), kb & 1, abort_flag, a.err, 4) &&
+                         wait_bar(bar(B_XFULL + sx), kx & 1, abort_flag, a.err, 5) &&
+                         wait_bar(bar(B_CFULL + scf), kc & 1, abort_flag, a.err, 6) &&
+                         (c == 0 || wait_bar(bar(B_OPSFREE), (c - 1) & 1, abort_flag, a.err, 7)));
             }
-            if (named_bar_or(1, 128, fail)) break;
-            const float *cf = coef0 + s * CF_FLOATS;
-            const uint8_t *stg = sm + OFF_STAGE0 + s * STAGE;
-            const uint32_t *braw = reinterpret_cast<const uint32_t *>(stg + SZ_X);
-            const uint32_t *craw = reinterpret_cast<const uint32_t *>(stg + SZ_X + SZ_BC);
-            const float *th = reinterpret_cast<const float *>(stg + SZ_X + 2 * SZ_BC);
-            const int L = (int)cf[CF_SCAL + 2];
+            if (named_bar_or(1, PREP_THREADS, fail)) break;
+            const float *cf = coef0 + scf * CF_FLOATS;
+            const uint8_t *stg = sm + L::OFF_BCT + sb * L::SZ_BCT;
+            const uint4 *braw = reinterpret_cast<const uint4 *>(stg);
+            const uint4 *craw = reinterpret_cast<const uint4 *>(stg + SZ_BC);
+            const float4 *th = reinterpret_cast<const float4 *>(stg + 2 * SZ_BC);
+            const int Lc = (int)cf[CF_SCAL + 2];
             if (has_norm) {
                 // inverse RMS of each B and C row of the chunk: one warp per row
                 const int wp = pt >> 5;
-                for (int r = wp; r < 2 * Q; r += 4) {
+                const uint32_t *b32 = reinterpret_cast<const uint32_t *>(braw);
+                const uint32_t *c32 = reinterpret_cast<const uint32_t *>(craw);
+                for (int r = wp; r < 2 * Q; r += NPREP) {
                     const int i = r & (Q - 1);
-                    const uint32_t *raw = (r < Q) ? braw : craw;
+                    const uint32_t *raw = (r < Q) ? b32 : c32;
                     float ss = 0.f;
-                    for (int q = l32; q < NP2; q += 32) {
-                        const float2 f = unpack_bf16(raw[i * NP2 + q]);
+                    for (int qq = l32; qq < NP2; qq += 32) {
+                        const float2 f = unpack_bf16(raw[i * NP2 + qq]);
                         ss += f.x * f.x + f.y * f.y;
                     }
                     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
                     if (l32 == 0) inv[r] = rsqrtf(ss / N + nr.eps);
                 }
             }
-            // pass 1: angle increments of my half of the chunk
-            float acc = 0.f;
-            const int i0 = half * 32;
-            for (int i = i0; i < i0 + 32; i++) acc += cf[CF_DT + i] * th[i * NP2 + j];
-            if (half == 0) part[j] = acc;
-            named_bar(1, 128);
-            float phi = phic[j] + (half ? part[j] : 0.f);
-            // pass 2: rotate
-            const bool last_chunk = (c == nchunks - 1);
-            for (int i = i0; i < i0 + 32; i++) {
-                uint32_t pb = 0u, pc = 0u;
-                if (i < L) {
-                    phi = fmaf(cf[CF_DT + i], th[i * NP2 + j], phi);
-                    float sn, cs;
-                    sincos_rr(phi, &sn, &cs);
-                    float2 bv = unpack_bf16(braw[i * NP2 + j]);
-                    float2 cv = unpack_bf16(craw[i * NP2 + j]);
-                    if (has_norm) {
-                        if (nr.wB) { bv.x *= inv[i] * wb0; bv.y *= inv[i] * wb1; }
-                        if (nr.wC) { cv.x *= inv[Q + i] * wc0; cv.y *= inv[Q + i] * wc1; }
-                    }
-                    bv.x += bb0; bv.y += bb1;
-                    cv.x += bc0; cv.y += bc1;
-                    const float rb0 = cs * bv.x - sn * bv.y, rb1 = sn * bv.x + cs * bv.y;
-                    const float rc0 = cs * cv.x - sn * cv.y, rc1 = sn * cv.x + cs * cv.y;
-                    const float e = cf[CF_E + i];
-                    pb = pack_bf16(rb0 * e, rb1 * e);
-                    pc = pack_bf16(rc0, rc1);
-                    if (last_chunk && i == L - 1) {
-                        blast[2 * j] = rb0;
-                        blast[2 * j + 1] = rb1;
-                    }
+            // pass 1: angle increments of my token group
+            const int i0 = tg * TPT;
+            float dph[TPT][4];
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int u = 0; u < TPT; u++) {
+                const float d = cf[CF_DT + i0 + u];
+                const float4 t4 = th[(i0 + u) * 16 + j4];
+                dph[u][0] = d * t4.x;
+                dph[u][1] = d * t4.y;
+                dph[u][2] = d * t4.z;
+                dph[u][3] = d * t4.w;
+#pragma unroll
+                for (int q = 0; q < 4; q++) acc[q] += dph[u][q];
+            }
+            *reinterpret_cast<float4 *>(part + tg * NP2 + 4 * j4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            named_bar(1, PREP_THREADS);
+            float phi[4];
+            {
+                const float4 p0 = *reinterpret_cast<const float4 *>(phic + 4 * j4);
+                phi[0] = p0.x; phi[1] = p0.y; phi[2] = p0.z; phi[3] = p0.w;
+                for (int g2 = 0; g2 < tg; g2++) {
+                    const float4 pg = *reinterpret_cast<const float4 *>(part + g2 * NP2 + 4 * j4);
+                    phi[0] += pg.x; phi[1] += pg.y; phi[2] += pg.z; phi[3] += pg.w;
                 }
-                *reinterpret_cast<uint32_t *>(bsc + atom + sw128(i, col)) = pb;
-                *reinterpret_cast<uint32_t *>(cb + atom + sw128(i, col)) = pc;
+            }
+            // pass 2: rotate my tokens (the same angles for every rank)
+            const bool last_chunk = last_seg && (c == nchunks - 1);
+#pragma unroll
+            for (int u = 0; u < TPT; u++) {
+                const int i = i0 + u;
+#pragma unroll
+                for (int q = 0; q < 4; q++) phi[q] += dph[u][q];
+                float sn[4], cs[4];
+#pragma unroll
+                for (int q = 0; q < 4; q++) sincos_rr(phi[q], &sn[q], &cs[q]);
+                const float e = cf[CF_E + i];
+#pragma unroll 1
+                for (int r = 0; r < R; r++) {
+                    const int row = i * R + r;
+                    uint4 ob = make_uint4(0u, 0u, 0u, 0u), oc = make_uint4(0u, 0u, 0u, 0u);
+                    if (i < Lc) {
+                        const uint4 rb = braw[row * 16 + j4];
+                        const uint4 rc = SO ? make_uint4(0u, 0u, 0u, 0u) : craw[row * 16 + j4];
+                        const uint32_t rbw[4] = {rb.x, rb.y, rb.z, rb.w}, rcw[4] = {rc.x, rc.y, rc.z, rc.w};
+                        uint32_t pbw[4], pcw[4];
+                        const float ib = (has_norm && nr.wB) ? inv[row] : 1.f;
+                        const float ic = (has_norm && nr.wC) ? inv[Q + row] : 1.f;
+#pragma unroll
+                        for (int q = 0; q < 4; q++) {
+                            float2 bv = unpack_bf16(rbw[q]), cv = unpack_bf16(rcw[q]);
+                            const int e0 = 8 * j4 + 2 * q;
+                            if (has_norm) {
+                                if (nr.wB) { bv.x *= ib * nr.wB[e0]; bv.y *= ib * nr.wB[e0 + 1]; }
+                                if (nr.wC) { cv.x *= ic * nr.wC[e0]; cv.y *= ic * nr.wC[e0 + 1]; }
+                            }
+                            if (has_bias) {
+                                const int64_t bo = (h * R + r) * N + e0;
+                                if (nr.biasB) { bv.x += nr.biasB[bo]; bv.y += nr.biasB[bo + 1]; }
+                                if (nr.biasC) { cv.x += nr.biasC[bo]; cv.y += nr.biasC[bo + 1]; }
+                            }
+                            const float rb0 = cs[q] * bv.x - sn[q] * bv.y, rb1 = sn[q] * bv.x + cs[q] * bv.y;
+                            pbw[q] = pack_bf16(rb0 * e, rb1 * e);
+                            if (!SO) pcw[q] = pack_bf16(cs[q] * cv.x - sn[q] * cv.y, sn[q] * cv.x + cs[q] * cv.y);
+                            else pcw[q] = 0u;
+                            if (last_chunk && i == Lc - 1) {
+                                blast[r * N + e0] = rb0;
+                                blast[r * N + e0 + 1] = rb1;
+                            }
+                        }
+                        ob = make_uint4(pbw[0], pbw[1], pbw[2], pbw[3]);
+                        oc = make_uint4(pcw[0], pcw[1], pcw[2], pcw[3]);
+                    }
+                    const uint32_t off = atom + (uint32_t)(row * 128 + ((chk ^ (row & 7)) << 4));
+                    *reinterpret_cast<uint4 *>(bsc + off) = ob;
+                    if (!SO) *reinterpret_cast<uint4 *>(cb + off) = oc;
+                }
+            }
+            // the X operands, 16-byte vectors of 128-byte rows (a vector keeps its
+            // place under the swizzle, so its row is its index / 8):
+            //   SISO:  Xw = diag(xs) x
+            //   MIMO:  Xr[(s,r)] = W_x[r] x_s (intra UMMA), Xw[(s,r)] = xs_s Xr[(s,r)]
+            {
+                const uint8_t *xt = sm + L::OFF_X + sx * L::SZ_X;
+                uint4 *dw = reinterpret_cast<uint4 *>(sm + L::OFF_XW);
+                uint4 *dr = reinterpret_cast<uint4 *>(sm + L::OFF_XR);
+#pragma unroll
+                for (int v = pt; v < Q * P / 8; v += PREP_THREADS) {
+                    const int row = v >> 3, pc = v & 7;
+                    const int sq = row / R;                       // token of the row
+                    const float sc = cf[CF_XS + sq];
+                    uint4 d, dxr;
+                    if (R == 1) {
+                        d = reinterpret_cast<const uint4 *>(xt)[v];
+                        uint32_t *w = reinterpret_cast<uint32_t *>(&d);
+#pragma unroll
+                        for (int q = 0; q < 4; q++) {
+                            const float2 f = unpack_bf16(w[q]);
+                            w[q] = pack_bf16(f.x * sc, f.y * sc);
+                        }
+                    } else {
+                        const int rr = row % R;
+                        const int cc = pc ^ (row & 7);            // logical 8-column chunk of this vector
+                        const uint4 xv =
+                            *reinterpret_cast<const uint4 *>(xt + sq * 128 + ((cc ^ (sq & 7)) << 4));
+                        const uint32_t xw4[4] = {xv.x, xv.y, xv.z, xv.w};
+                        uint32_t ow[4], orr[4];
+#pragma unroll
+                        for (int q = 0; q < 4; q++) {
+                            const float2 f = unpack_bf16(xw4[q]);
+                            const float x0 = f.x * wxs[rr * P + 8 * cc + 2 * q];
+                            const float x1 = f.y * wxs[rr * P + 8 * cc + 2 * q + 1];
+                            orr[q] = pack_bf16(x0, x1);
+                            ow[q] = pack_bf16(x0 * sc, x1 * sc);
+                        }
+                        d = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                        dxr = make_uint4(orr[0], orr[1], orr[2], orr[3]);
+                        if (!SO) dr[v] = dxr;
+                    }
+                    dw[v] = d;
+                }
             }
             fence_async_smem();
-            named_bar(1, 128);
-            if (half == 1) {
-                phic[j] = phi;      // the angle after the chunk's last token
-                if (last_chunk && a.angle_out) a.angle_out[lane_id * NP2 + j] = phi;
+            named_bar(1, PREP_THREADS);
+            if (tg == 15) {
+                // the last token group ends at the chunk's last token
+                *reinterpret_cast<float4 *>(phic + 4 * j4) = make_float4(phi[0], phi[1], phi[2], phi[3]);
+                if (last_chunk && a.angle_out)
+                    *reinterpret_cast<float4 *>(a.angle_out + lane_id * NP2 + 4 * j4) =
+                        make_float4(phi[0], phi[1], phi[2], phi[3]);
+                if (SO && c == nchunks - 1)
+                    *reinterpret_cast<float4 *>(slot_out + SLOT_PHIL + 4 * j4) =
+                        make_float4(phi[0], phi[1], phi[2], phi[3]);
             }
             if (pt == 0) {
                 mbar_arrive(bar(B_OPSREADY));
-                mbar_arrive(bar(B_EMPTY0 + s));
-                mbar_arrive(bar(B_CEMPTY0 + s));
+                mbar_arrive(bar(B_BEMPTY + sb));
+                mbar_arrive(bar(B_XEMPTY + sx));
+                mbar_arrive(bar(B_CEMPTY + scf));
             }
         }
     } else if (warp == W_MMA) {
@@ -499,40 +751,53 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t id_kk = idesc(64, 64, 0, 0);    // D1 = Cbar . Bsc^T
             const uint32_t id_kmn = idesc(64, 64, 0, 1);   // D2, D3: B operand MN-major
             const uint32_t id_st = idesc(128, 64, 1, 1);   // D4: A and B MN-major
-            const uint32_t a_bsc = sbase + OFF_BSC, a_cb = sbase + OFF_CB, a_sp = sbase + OFF_SP;
-            const uint32_t a_xw = sbase + OFF_XW, a_gb = sbase + OFF_GB;
+            const uint32_t a_bsc = sbase + L::OFF_BSC, a_cb = sbase + L::OFF_CB, a_sp = sbase + L::OFF_SP;
+            const uint32_t a_xw = sbase + L::OFF_XW;
             for (int c = 0; c < nchunks; c++) {
-                const int s = c & 1;
-                const uint32_t a_x = sbase + OFF_STAGE0 + s * STAGE;
-                if (!wait_bar(bar(B_OPSREADY), c & 1, abort_flag, a.err, 10)) break;
-                if (c > 0 && !wait_bar(bar(B_STAKEN), (c - 1) & 1, abort_flag, a.err, 11)) break;
+                const int sx = c % NX;
+                // intra UMMA operand: the x tile itself (SISO) or the rank-expanded Xr
+                const uint32_t a_x = (R == 1) ? sbase + L::OFF_X + sx * L::SZ_X : sbase + L::OFF_XR;
+                const uint32_t a_gprev = sbase + L::OFF_GB + ((c + 1) & 1) * SZ_GB;   // state after chunk c-1
+                if (!wait_bar_spin(bar(B_OPSREADY), c & 1, abort_flag, a.err, 10)) break;
+                if (SO) {
+                    // state-only pass: the chunk-state UMMA alone
+                    if (!wait_bar_spin(bar(B_STTAKEN), c & 1, abort_flag, a.err, 12)) break;
+                    tc_fence_after();
+                    for (int kk = 0; kk < Q / 16; kk++)
+                        umma(tmem + COL_D4, sdesc(a_bsc + kk * 2048, Q * 128, 1024),
+                             sdesc(a_xw + kk * 2048, Q * 128, 1024), id_st, kk > 0);
+                    umma_commit(bar(B_STFULL));
+                    umma_commit(bar(B_OPSFREE));
+                    continue;
+                }
+                if (c > 0 && !wait_bar_spin(bar(B_STAKEN), (c - 1) & 1, abort_flag, a.err, 11)) break;
                 tc_fence_after();
                 for (int kk = 0; kk < N / 16; kk++) {
                     const uint32_t off = (kk >> 2) * (Q * 128) + (kk & 3) * 32;
                     umma(tmem + COL_D1, sdesc(a_cb + off, 16, 1024), sdesc(a_bsc + off, 16, 1024), id_kk, kk > 0);
                 }
                 umma_commit(bar(B_SFULL));
-                if (!wait_bar(bar(B_STTAKEN), c & 1, abort_flag, a.err, 12)) break;
+                if (!wait_bar_spin(bar(B_STTAKEN), c & 1, abort_flag, a.err, 12)) break;
                 tc_fence_after();
                 for (int kk = 0; kk < Q / 16; kk++)
                     umma(tmem + COL_D4, sdesc(a_bsc + kk * 2048, Q * 128, 1024), sdesc(a_xw + kk * 2048, Q * 128, 1024),
                          id_st, kk > 0);
                 umma_commit(bar(B_STFULL));
-                if (c > 0 && !wait_bar(bar(B_YTAKEN), (c - 1) & 1, abort_flag, a.err, 13)) break;
+                if (c > 0 && !wait_bar_spin(bar(B_YTAKEN), (c - 1) & 1, abort_flag, a.err, 13)) break;
                 tc_fence_after();
                 for (int kk = 0; kk < N / 16; kk++) {
                     const uint32_t off = (kk >> 2) * (Q * 128) + (kk & 3) * 32;
-                    umma(tmem + COL_D3, sdesc(a_cb + off, 16, 1024), sdesc(a_gb + kk * 2048, N * 128, 1024), id_kmn,
+                    umma(tmem + COL_D3, sdesc(a_cb + off, 16, 1024), sdesc(a_gprev + kk * 2048, N * 128, 1024), id_kmn,
                          kk > 0);
                 }
                 umma_commit(bar(B_OPSFREE));
-                if (!wait_bar(bar(B_SPFULL), c & 1, abort_flag, a.err, 14)) break;
+                if (!wait_bar_spin(bar(B_SPFULL), c & 1, abort_flag, a.err, 14)) break;
                 tc_fence_after();
                 for (int kk = 0; kk < Q / 16; kk++)
                     umma(tmem + COL_D2, sdesc(a_sp + kk * 32, 16, 1024), sdesc(a_x + kk * 2048, Q * 128, 1024), id_kmn,
                          kk > 0);
                 umma_commit(bar(B_YFULL));
-                umma_commit(bar(B_EMPTY0 + s));
+                umma_commit(bar(B_XEMPTY + sx));
             }
             // drain: every MMA issued so far has completed before TMEM is freed
             umma_commit(bar(B_DRAIN));
@@ -542,202 +807,265 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else {
         // ------------------------------------------------------------- epilogue
+        // Per chunk: mask the scores, fold the chunk state into g (this runs
+        // while the intra UMMA completes), then write the outputs.
         const int q = warp & 3;                      // TMEM lane quarter
+        const int ch = (warp - W_EPI0) >> 2;         // column half: 32 * ch .. 32 * ch + 31
+        const int cb0 = 32 * ch;
         const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
         const int n = 32 * q + l32;                  // state row owned by this thread
         const int trow = 16 * q + l32;               // score/output row (valid for l32 < 16)
+        const int ttok = trow / R;                   // its token
         const bool rowv = l32 < 16;
+        const int et = tid - W_EPI0 * 32;            // 0..255
         const float Dh = a.D[h];
-        uint8_t *sp = sm + OFF_SP;
-        uint8_t *gb = sm + OFF_GB;
-        uint8_t *yt = sm + OFF_YT;
-        float g[P];
-        {
-            float f0 = 0.f;
-            if (Tn > 0) {
-                const int64_t i0 = (b * Tn) * H + h;
-                f0 = (1.f - a.lam[i0]) * a.dt[i0];
-            }
-            const int64_t base = (lane_id * N + n) * P;
-#pragma unroll
-            for (int p = 0; p < P; p += 4) {
-                float4 hv = a.h0 ? *reinterpret_cast<const float4 *>(a.h0 + base + p) : make_float4(0, 0, 0, 0);
-                float4 uv = a.prevBx0 ? *reinterpret_cast<const float4 *>(a.prevBx0 + base + p)
-                                      : make_float4(0, 0, 0, 0);
-                g[p] = hv.x + f0 * uv.x;
-                g[p + 1] = hv.y + f0 * uv.y;
-                g[p + 2] = hv.z + f0 * uv.z;
-                g[p + 3] = hv.w + f0 * uv.w;
-            }
-#pragma unroll
-            for (int cc = 0; cc < 8; cc++) {
-                uint4 v;
-                v.x = pack_bf16(g[8 * cc], g[8 * cc + 1]);
-                v.y = pack_bf16(g[8 * cc + 2], g[8 * cc + 3]);
-                v.z = pack_bf16(g[8 * cc + 4], g[8 * cc + 5]);
-                v.w = pack_bf16(g[8 * cc + 6], g[8 * cc + 7]);
-                *reinterpret_cast<uint4 *>(gb + n * 128 + ((cc ^ (n & 7)) << 4)) = v;
-            }
-            fence_async_smem();
-            __syncwarp();
-            if (l32 == 0) mbar_arrive(bar(B_STTAKEN));
-        }
-        const int et = tid - W_EPI0 * 32;
+        uint8_t *sp = sm + L::OFF_SP;
+        uint8_t *yt = sm + L::OFF_YT;
         // one thread waits, the group meets at a named barrier and leaves together
         auto group_wait = [&](int bi, uint32_t parity, int site) -> bool {
             bool fail = false;
             if (et == 0) fail = !wait_bar(bar(bi), parity, abort_flag, a.err, site);
-            return !named_bar_or(2, 128, fail);
+            return !named_bar_or(2, EPI_THREADS, fail);
         };
-        bool ok = true;
-        for (int c = 0; c < nchunks && ok; c++) {
-            const int s = c & 1, k = c >> 1;
-            const float *cf = coef0 + s * CF_FLOATS;
-            const uint8_t *xr = sm + OFF_STAGE0 + s * STAGE;
-            if (!(ok = group_wait(B_CFULL0 + s, k & 1, 20))) break;
-            const int L = (int)cf[CF_SCAL + 2];
-            const bool unsafe = cf[CF_SCAL + 1] != 0.f;
-            // ---- masked scores S' (rows of D1) ----
-            if (!(ok = group_wait(B_SFULL, c & 1, 21))) break;
-            tc_fence_after();
-            {
-                const int t = trow;
-                const float rt = rowv ? cf[CF_R + t] : 0.f;
-                const float c2t = rowv ? cf[CF_C2 + t] : 0.f;
+        auto store_g = [&](const float *gv, int slot) {
+            uint8_t *gb = sm + L::OFF_GB + slot * SZ_GB;
 #pragma unroll
-                for (int c16 = 0; c16 < Q / 16; c16++) {
-                    float v[16];
-                    tmem_ld16(tl + COL_D1 + 16 * c16, v);
-                    tmem_wait_ld();
-                    if (rowv) {
-#pragma unroll
-                        for (int u = 0; u < 16; u++) {
-                            const int s2 = 16 * c16 + u;
-                            float m;
-                            if (!unsafe)
-                                m = s2 < t ? rt * cf[CF_W + s2] : (s2 == t ? rt * cf[CF_GAM + t] : 0.f);
-                            else
-                                m = s2 < t ? exp2f(c2t - cf[CF_C2 + s2]) * cf[CF_W + s2]
-                                           : (s2 == t ? cf[CF_GAM + t] : 0.f);
-                            v[u] *= m;
-                        }
-#pragma unroll
-                        for (int hh = 0; hh < 2; hh++) {
-                            const int cc = 2 * c16 + hh;
-                            uint4 pk;
-                            pk.x = pack_bf16(v[8 * hh], v[8 * hh + 1]);
-                            pk.y = pack_bf16(v[8 * hh + 2], v[8 * hh + 3]);
-                            pk.z = pack_bf16(v[8 * hh + 4], v[8 * hh + 5]);
-                            pk.w = pack_bf16(v[8 * hh + 6], v[8 * hh + 7]);
-                            *reinterpret_cast<uint4 *>(sp + t * 128 + ((cc ^ (t & 7)) << 4)) = pk;
-                        }
-                    }
-                }
+            for (int k4 = 0; k4 < 4; k4++) {
+                const int cc = 4 * ch + k4;
+                uint4 v;
+                v.x = pack_bf16(gv[8 * k4], gv[8 * k4 + 1]);
+                v.y = pack_bf16(gv[8 * k4 + 2], gv[8 * k4 + 3]);
+                v.z = pack_bf16(gv[8 * k4 + 4], gv[8 * k4 + 5]);
+                v.w = pack_bf16(gv[8 * k4 + 6], gv[8 * k4 + 7]);
+                *reinterpret_cast<uint4 *>(gb + n * 128 + ((cc ^ (n & 7)) << 4)) = v;
             }
-            tc_fence_before();
-            __syncwarp();
-            if (l32 == 0) mbar_arrive(bar(B_STAKEN));
-            fence_async_smem();
-            __syncwarp();
-            if (l32 == 0) mbar_arrive(bar(B_SPFULL));
-            // ---- outputs y = D2 + e^{cum_t} D3 + D x ----
-            if (et == 0) tma_store_wait_read();   // the previous output tile has been read out
-            if (!(ok = group_wait(B_YFULL, c & 1, 22))) break;
-            tc_fence_after();
-            const float ect = rowv ? cf[CF_EC + trow] : 0.f;
-#pragma unroll
-            for (int c16 = 0; c16 < P / 16; c16++) {
-                float y2[16], y3[16];
-                tmem_ld16(tl + COL_D2 + 16 * c16, y2);
-                tmem_ld16(tl + COL_D3 + 16 * c16, y3);
-                tmem_wait_ld();
-                if (rowv) {
-                    const int t = trow;
-                    uint32_t pk[8];
-#pragma unroll
-                    for (int hh = 0; hh < 2; hh++) {
-                        const int cc = 2 * c16 + hh;   // 16-byte chunk (8 columns)
-                        const uint4 xv = *reinterpret_cast<const uint4 *>(xr + t * 128 + ((cc ^ (t & 7)) << 4));
-                        const uint32_t *xw = reinterpret_cast<const uint32_t *>(&xv);
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; e2++) {
-                            const float2 xf = unpack_bf16(xw[e2]);
-                            const int cidx = 8 * hh + 2 * e2;
-                            const float o0 = y2[cidx] + ect * y3[cidx] + Dh * xf.x;
-                            const float o1 = y2[cidx + 1] + ect * y3[cidx + 1] + Dh * xf.y;
-                            pk[4 * hh + e2] = pack_bf16(o0, o1);
-                        }
-                        *reinterpret_cast<uint4 *>(yt + t * 128 + ((cc ^ (t & 7)) << 4)) =
-                            make_uint4(pk[4 * hh], pk[4 * hh + 1], pk[4 * hh + 2], pk[4 * hh + 3]);
-                    }
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (l32 == 0) mbar_arrive(bar(B_YTAKEN));
-            fence_async_smem();
-            named_bar(2, 128);
-            if (et == 0) {
-                tma_store4(&map_y, 0, (int)h, c * Q, (int)b, sbase + OFF_YT);
-                mbar_arrive(bar(B_EMPTY0 + s));
-            }
-            // ---- state: g = e^{cum_end} g + D4 ----
-            if (!(ok = group_wait(B_STFULL, c & 1, 23))) break;
-            tc_fence_after();
+        };
+        auto fold_state = [&](const float *cf, float *gv) {
             const float E = cf[CF_SCAL + 0];
 #pragma unroll
-            for (int c16 = 0; c16 < P / 16; c16++) {
+            for (int c16 = 0; c16 < 2; c16++) {
                 float d4[16];
-                tmem_ld16(tl + COL_D4 + 16 * c16, d4);
+                tmem_ld16(tl + COL_D4 + cb0 + 16 * c16, d4);
                 tmem_wait_ld();
 #pragma unroll
-                for (int u = 0; u < 16; u++) g[16 * c16 + u] = fmaf(E, g[16 * c16 + u], d4[u]);
+                for (int u = 0; u < 16; u++) gv[16 * c16 + u] = fmaf(E, gv[16 * c16 + u], d4[u]);
             }
-            tc_fence_before();
+        };
+        float g[32];
+        if (SO) {
+            // state-only pass: g starts at zero, only the state update runs
 #pragma unroll
-            for (int cc = 0; cc < 8; cc++) {
-                uint4 pk;
-                pk.x = pack_bf16(g[8 * cc], g[8 * cc + 1]);
-                pk.y = pack_bf16(g[8 * cc + 2], g[8 * cc + 3]);
-                pk.z = pack_bf16(g[8 * cc + 4], g[8 * cc + 5]);
-                pk.w = pack_bf16(g[8 * cc + 6], g[8 * cc + 7]);
-                *reinterpret_cast<uint4 *>(gb + n * 128 + ((cc ^ (n & 7)) << 4)) = pk;
-            }
-            fence_async_smem();
+            for (int p = 0; p < 32; p++) g[p] = 0.f;
             __syncwarp();
             if (l32 == 0) mbar_arrive(bar(B_STTAKEN));
-            named_bar(2, 128);
-            if (et == 0) mbar_arrive(bar(B_CEMPTY0 + s));
-            (void)L;
-        }
-        if (et == 0) tma_store_wait_all();
-        // final state: h_{T-1} = g after the last chunk (no lookahead there)
-        if (!*abort_flag && a.h_out) {
-            float *ho = a.h_out + (lane_id * N + n) * P;
+            float eacc = 1.f;
+            bool ok2 = true;
+            for (int c = 0; c < nchunks && ok2; c++) {
+                const int scf = c % NC;
+                const float *cf = coef0 + scf * CF_FLOATS;
+                if (!(ok2 = group_wait(B_CFULL + scf, (c / NC) & 1, 24))) break;
+                if (!(ok2 = group_wait(B_STFULL, c & 1, 25))) break;
+                tc_fence_after();
+                eacc *= cf[CF_SCAL + 0];
+                fold_state(cf, g);
+                tc_fence_before();
+                __syncwarp();
+                if (l32 == 0) mbar_arrive(bar(B_STTAKEN));
+                named_bar(2, EPI_THREADS);
+                if (et == 0) mbar_arrive(bar(B_CEMPTY + scf));
+            }
+            if (!*abort_flag) {
+                float *go = slot_out + SLOT_G + n * P + cb0;
 #pragma unroll
-            for (int p = 0; p < P; p += 4) *reinterpret_cast<float4 *>(ho + p) = make_float4(g[p], g[p + 1], g[p + 2], g[p + 3]);
+                for (int p = 0; p < 32; p += 4)
+                    *reinterpret_cast<float4 *>(go + p) = make_float4(g[p], g[p + 1], g[p + 2], g[p + 3]);
+                if (et == 0) slot_out[SLOT_E] = eacc;
+            }
+        } else {
+            {
+                const int64_t base = (lane_id * N + n) * P + cb0;
+                if (slot_in) {
+                    // a later segment starts from the state the combine pass left in the slot
+#pragma unroll
+                    for (int p = 0; p < 32; p += 4) {
+                        const float4 gv = *reinterpret_cast<const float4 *>(slot_in + SLOT_G + n * P + cb0 + p);
+                        g[p] = gv.x; g[p + 1] = gv.y; g[p + 2] = gv.z; g[p + 3] = gv.w;
+                    }
+                } else {
+                    const int64_t i0 = (b * Tn) * H + h;
+                    const float f0 = (1.f - a.lam[i0]) * a.dt[i0];
+#pragma unroll
+                    for (int p = 0; p < 32; p += 4) {
+                        const float4 hv = a.h0 ? *reinterpret_cast<const float4 *>(a.h0 + base + p)
+                                               : make_float4(0, 0, 0, 0);
+                        const float4 uv = a.prevBx0 ? *reinterpret_cast<const float4 *>(a.prevBx0 + base + p)
+                                                    : make_float4(0, 0, 0, 0);
+                        g[p] = fmaf(f0, uv.x, hv.x);
+                        g[p + 1] = fmaf(f0, uv.y, hv.y);
+                        g[p + 2] = fmaf(f0, uv.z, hv.z);
+                        g[p + 3] = fmaf(f0, uv.w, hv.w);
+                    }
+                }
+                store_g(g, 1);                       // read by the inter-chunk UMMA of chunk 0
+                fence_async_smem();
+                __syncwarp();
+                if (l32 == 0) mbar_arrive(bar(B_STTAKEN));
+            }
+            bool ok = true;
+            for (int c = 0; c < nchunks && ok; c++) {
+                const int scf = c % NC, kc = c / NC, sx = c % NX;
+                const float *cf = coef0 + scf * CF_FLOATS;
+                const uint8_t *xr = sm + L::OFF_X + sx * L::SZ_X;
+                if (!(ok = group_wait(B_CFULL + scf, kc & 1, 20))) break;
+                const bool unsafe = cf[CF_SCAL + 1] != 0.f;
+                // ---- masked scores S' (rows of D1, my 32 columns) ----
+                if (!(ok = group_wait(B_SFULL, c & 1, 21))) break;
+                tc_fence_after();
+                {
+                    const int t = ttok;
+                    const float rt = rowv ? cf[CF_R + t] : 0.f;
+                    const float c2t = rowv ? cf[CF_C2 + t] : 0.f;
+                    const float gt = rowv ? cf[CF_GAM + t] : 0.f;
+#pragma unroll
+                    for (int c16 = 0; c16 < 2; c16++) {
+                        const int s0 = cb0 + 16 * c16;
+                        float v[16];
+                        tmem_ld16(tl + COL_D1 + s0, v);
+                        tmem_wait_ld();
+                        if (rowv) {
+#pragma unroll
+                            for (int k2 = 0; k2 < 16 / R; k2++) {
+                                const int s2 = s0 / R + k2;      // token of columns k2*R .. k2*R+R-1
+                                const float wsv = cf[CF_W + s2];
+                                float m;
+                                if (!unsafe)
+                                    m = s2 < t ? rt * wsv : (s2 == t ? rt * gt : 0.f);
+                                else
+                                    m = s2 < t ? exp2f(c2t - cf[CF_C2 + s2]) * wsv : (s2 == t ? gt : 0.f);
+#pragma unroll
+                                for (int r2 = 0; r2 < R; r2++) v[k2 * R + r2] *= m;
+                            }
+#pragma unroll
+                            for (int hh = 0; hh < 2; hh++) {
+                                const int cc = (s0 >> 3) + hh;
+                                uint4 pk;
+                                pk.x = pack_bf16(v[8 * hh], v[8 * hh + 1]);
+                                pk.y = pack_bf16(v[8 * hh + 2], v[8 * hh + 3]);
+                                pk.z = pack_bf16(v[8 * hh + 4], v[8 * hh + 5]);
+                                pk.w = pack_bf16(v[8 * hh + 6], v[8 * hh + 7]);
+                                *reinterpret_cast<uint4 *>(sp + trow * 128 + ((cc ^ (trow & 7)) << 4)) = pk;
+                            }
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (l32 == 0) mbar_arrive(bar(B_STAKEN));
+                fence_async_smem();
+                __syncwarp();
+                if (l32 == 0) mbar_arrive(bar(B_SPFULL));
+                // ---- state after chunk c: g = e^{cum_end} g + D4 (my 32 columns) ----
+                if (!(ok = group_wait(B_STFULL, c & 1, 23))) break;
+                tc_fence_after();
+                fold_state(cf, g);
+                tc_fence_before();
+                store_g(g, c & 1);
+                fence_async_smem();
+                __syncwarp();
+                if (l32 == 0) mbar_arrive(bar(B_STTAKEN));
+                // ---- outputs y_t = sum_r W_y[r] (D2 + e^{cum_t} D3)_{(t,r)} + D x_t ----
+                if (et == 0) tma_store_wait_read();   // the previous output tile has been read out
+                if (!(ok = group_wait(B_YFULL, c & 1, 22))) break;
+                tc_fence_after();
+                const float ect = rowv ? cf[CF_EC + ttok] : 0.f;
+                const int rr = trow % R;
+#pragma unroll
+                for (int c16 = 0; c16 < 2; c16++) {
+                    const int p0 = cb0 + 16 * c16;
+                    float y2[16], y3[16];
+                    tmem_ld16(tl + COL_D2 + p0, y2);
+                    tmem_ld16(tl + COL_D3 + p0, y3);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; e++) {
+                        float v = fmaf(ect, y3[e], y2[e]);
+                        if (R > 1) {
+                            // contract the R rows of a token (adjacent lanes) with W_y
+                            v *= wys[rr * P + p0 + e];
+#pragma unroll
+                            for (int o = 1; o < R; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                        }
+                        y2[e] = v;
+                    }
+                    if (rowv && rr == 0) {
+                        const int t = ttok;
+#pragma unroll
+                        for (int hh = 0; hh < 2; hh++) {
+                            const int cc = (p0 >> 3) + hh;   // 16-byte chunk (8 columns)
+                            const uint4 xv = *reinterpret_cast<const uint4 *>(xr + t * 128 + ((cc ^ (t & 7)) << 4));
+                            const uint32_t xw4[4] = {xv.x, xv.y, xv.z, xv.w};
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int e2 = 0; e2 < 4; e2++) {
+                                const float2 xf = unpack_bf16(xw4[e2]);
+                                const int cidx = 8 * hh + 2 * e2;
+                                pk[e2] = pack_bf16(fmaf(Dh, xf.x, y2[cidx]), fmaf(Dh, xf.y, y2[cidx + 1]));
+                            }
+                            *reinterpret_cast<uint4 *>(yt + t * 128 + ((cc ^ (t & 7)) << 4)) =
+                                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (l32 == 0) mbar_arrive(bar(B_YTAKEN));
+                fence_async_smem();
+                named_bar(2, EPI_THREADS);
+                if (et == 0) {
+                    tma_store4(&map_y, 0, (int)h, (int)(t_beg + (int64_t)c * QT), (int)b, sbase + L::OFF_YT);
+                    mbar_arrive(bar(B_XEMPTY + sx));
+                    mbar_arrive(bar(B_CEMPTY + scf));
+                }
+            }
+            if (et == 0) tma_store_wait_all();
+            // final state: h_{T-1} = g after the last chunk (no lookahead there)
+            if (!*abort_flag && a.h_out && last_seg) {
+                float *ho = a.h_out + (lane_id * N + n) * P + cb0;
+#pragma unroll
+                for (int p = 0; p < 32; p += 4)
+                    *reinterpret_cast<float4 *>(ho + p) = make_float4(g[p], g[p + 1], g[p + 2], g[p + 3]);
+            }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    // prev_Bx = Bbar_{T-1} x_{T-1}^T (rotated, unscaled B row kept by the rotation warps)
-    if (!*abort_flag && a.prevBx_out && warp >= W_EPI0) {
-        const int n = tid - W_EPI0 * 32;
-        const int c = nchunks - 1, s = c & 1;
-        const int L = (int)(Tn - (int64_t)c * Q);
-        const uint8_t *xr = sm + OFF_STAGE0 + s * STAGE;
-        const int t = L - 1;
-        const float bn = blast[n];
+    // prev_Bx = sum_r Bbar_{T-1,r} X_{T-1,r}^T (rotated, unscaled B rows kept by
+    // the rotation warps; X_{T-1,r} = W_x[r] x_{T-1})
+    if (!SO && last_seg && !*abort_flag && a.prevBx_out && warp >= W_EPI0) {
+        const int et = tid - W_EPI0 * 32;
+        const int n = et & (N - 1), half = et >> 7;
+        const int c = nchunks - 1;
+        const int Lc = (int)(t_end - t_beg - (int64_t)c * QT);
+        const uint8_t *xr = sm + L::OFF_X + (c % NX) * L::SZ_X;
+        const int t = Lc - 1;
         float *uo = a.prevBx_out + (lane_id * N + n) * P;
-        for (int cc = 0; cc < 8; cc++) {
+        for (int cc = 4 * half; cc < 4 * half + 4; cc++) {
             const uint4 xv = *reinterpret_cast<const uint4 *>(xr + t * 128 + ((cc ^ (t & 7)) << 4));
-            const uint32_t *xw = reinterpret_cast<const uint32_t *>(&xv);
+            const uint32_t xw4[4] = {xv.x, xv.y, xv.z, xv.w};
             float o[8];
             for (int e2 = 0; e2 < 4; e2++) {
-                const float2 f = unpack_bf16(xw[e2]);
-                o[2 * e2] = bn * f.x;
-                o[2 * e2 + 1] = bn * f.y;
+                const float2 f = unpack_bf16(xw4[e2]);
+                const int p = 8 * cc + 2 * e2;
+                float u0 = 0.f, u1 = 0.f;
+                for (int r = 0; r < R; r++) {
+                    const float bn = blast[r * N + n];
+                    const float w0 = (R > 1) ? wxs[r * P + p] : 1.f, w1 = (R > 1) ? wxs[r * P + p + 1] : 1.f;
+                    u0 += bn * w0 * f.x;
+                    u1 += bn * w1 * f.y;
+                }
+                o[2 * e2] = u0;
+                o[2 * e2 + 1] = u1;
             }
             *reinterpret_cast<float4 *>(uo + 8 * cc) = make_float4(o[0], o[1], o[2], o[3]);
             *reinterpret_cast<float4 *>(uo + 8 * cc + 4) = make_float4(o[4], o[5], o[6], o[7]);
@@ -766,52 +1094,155 @@ static EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 4-D map over a (Bt, T, H, inner) tensor: dims (inner, H, T, Bt).
+// 4-D map over a (Bt, T, H, inner) tensor: dims (inner, H, T, Bt); with
+// rank > 0 a 5-D map over (Bt, T, H, rank, inner): dims (inner, rank, H, T, Bt)
+// whose box holds every rank.
 static bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize, int64_t inner,
-                     int64_t H, int64_t T, int64_t Bt, uint32_t box_inner, uint32_t box_t, CUtensorMapSwizzle sw) {
+                     int64_t H, int64_t T, int64_t Bt, uint32_t box_inner, uint32_t box_t, CUtensorMapSwizzle sw,
+                     int64_t rank = 0) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    if (rank > 0) {
+        cuuint64_t dims[5] = {(cuuint64_t)inner, (cuuint64_t)rank, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)Bt};
+        cuuint64_t strides[4] = {(cuuint64_t)(inner * esize), (cuuint64_t)(inner * rank * esize),
+                                 (cuuint64_t)(inner * rank * H * esize), (cuuint64_t)(inner * rank * H * T * esize)};
+        cuuint32_t box[5] = {box_inner, (cuuint32_t)rank, 1, box_t, 1};
+        return fn(m, dt, 5, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    }
     cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)Bt};
     cuuint64_t strides[3] = {(cuuint64_t)(inner * esize), (cuuint64_t)(inner * H * esize),
                              (cuuint64_t)(inner * H * T * esize)};
     cuuint32_t box[4] = {box_inner, 1, box_t, 1};
-    cuuint32_t estr[4] = {1, 1, 1, 1};
     return fn(m, dt, 4, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 __device__ int g_tc_error;
 
+// Segment plan: when there are too few (b, h) lanes to fill the GPU, each
+// lane's sequence is cut into segments of whole chunks that run in parallel.
+struct SegPlan {
+    int nseg;
+    int64_t seg_len;
+};
+static SegPlan seg_plan(int64_t lanes, int64_t T) {
+    SegPlan p{1, T};
+    if (lanes >= 96 || T <= 8 * Q) return p;
+    const int64_t target = (4 * 148 + lanes - 1) / lanes;   // about four CTAs per SM in all
+    int64_t len = (T + target - 1) / target;
+    len = ((len + Q - 1) / Q) * Q;
+    if (len < 4 * Q) len = 4 * Q;
+    const int64_t ns = (T + len - 1) / len;
+    if (ns < 2) return p;
+    p.nseg = (int)ns;
+    p.seg_len = len;
+    return p;
+}
+
+// Chains the segments of every lane: the state entering segment j+1 is
+//   g_in(j+1) = A_j g_in(j) + R(Phi_in(j)) g_loc(j),   Phi_in(j+1) = Phi_in(j) + dPhi_j
+// where g_loc(j) is segment j's end state from a zero start in its own angle
+// frame, A_j its decay product and R rotates every pair of state rows (2i,
+// 2i+1) by the angle of pair i (the rotation moves the local frame to the
+// absolute one: Bbar = R(Phi_in + phi_local) B).  One thread per (pair, column).
+__global__ void __launch_bounds__(256) k_seg_combine(TcArgs a) {
+    const int64_t lane = blockIdx.x, b = lane / a.H, h = lane % a.H;
+    const int idx = blockIdx.y * 256 + threadIdx.x;
+    const int i = idx / P, p = idx % P;
+    const int64_t i0 = (b * a.T) * a.H + h;
+    const float f0 = (1.f - a.lam[i0]) * a.dt[i0];
+    const int64_t r0 = (lane * N + 2 * i) * P + p, r1 = r0 + P;
+    float g0 = (a.h0 ? a.h0[r0] : 0.f) + f0 * (a.prevBx0 ? a.prevBx0[r0] : 0.f);
+    float g1 = (a.h0 ? a.h0[r1] : 0.f) + f0 * (a.prevBx0 ? a.prevBx0[r1] : 0.f);
+    float phi = a.angle0 ? a.angle0[lane * NP2 + i] : 0.f;
+    for (int j = 0; j < a.nseg - 1; j++) {
+        float *sl = a.ws + ((size_t)lane * (a.nseg - 1) + j) * SLOT_FLOATS;
+        const float l0 = sl[SLOT_G + 2 * i * P + p], l1 = sl[SLOT_G + (2 * i + 1) * P + p];
+        const float E = sl[SLOT_E], dphi = sl[SLOT_PHIL + i];
+        float sn, cs;
+        sincosf(phi, &sn, &cs);
+        g0 = fmaf(E, g0, cs * l0 - sn * l1);
+        g1 = fmaf(E, g1, sn * l0 + cs * l1);
+        sl[SLOT_G + 2 * i * P + p] = g0;
+        sl[SLOT_G + (2 * i + 1) * P + p] = g1;
+        phi += dphi;
+        if (p == 0) sl[SLOT_PHIN + i] = phi;
+    }
+}
+
 }  // namespace tc
 
+size_t scan_tc_workspace_bytes(int64_t Bt, int64_t H, int64_t T) {
+    const tc::SegPlan pl = tc::seg_plan(Bt * H, T);
+    if (pl.nseg <= 1) return 0;
+    return (size_t)(Bt * H) * (size_t)(pl.nseg - 1) * tc::SLOT_FLOATS * sizeof(float);
+}
+
+// The kernel's chunk is 64 rows: 64 tokens (SISO) or 64 / R tokens of R
+// ranks (MIMO, R = 2 or 4).  A requested chunk that is a multiple of that runs
+// as sub-chunks (the same result up to rounding order).
 bool scan_tc_supported(const ScanArgs &a, m3_dtype dt) {
-    return dt == M3_BF16 && a.R == 1 && !a.mimo_layout && a.P == tc::P && a.N == tc::N && a.Q == tc::Q &&
+    const bool shape = a.mimo_layout ? (a.R == 2 || a.R == 4) : (a.R == 1);
+    return dt == M3_BF16 && shape && a.P == tc::P && a.N == tc::N && a.Q > 0 && a.Q % (tc::Q / a.R) == 0 &&
            a.T > 0 && a.T <= ((int64_t)1 << 30) && a.Bt <= 65535 && a.H <= 65535;
 }
 
-cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s) {
+template <int R>
+static cudaError_t launch_tc_r(const ScanArgs &a, cudaStream_t s) {
     using namespace tc;
+    constexpr int QT = Q / R;
     CUtensorMap mx, mb, mc, mth, my;
-    if (!make_map(&mx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P, a.H, a.T, a.Bt, P, Q, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mb, a.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, a.H, a.T, a.Bt, N, Q, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&mc, a.C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, a.H, a.T, a.Bt, N, Q, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&mth, a.theta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, NP2, a.H, a.T, a.Bt, NP2, Q,
+    const int64_t rk = R > 1 ? R : 0;
+    if (!make_map(&mx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P, a.H, a.T, a.Bt, P, QT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mb, a.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, a.H, a.T, a.Bt, N, QT, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  rk) ||
+        !make_map(&mc, a.C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, a.H, a.T, a.Bt, N, QT, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  rk) ||
+        !make_map(&mth, a.theta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, NP2, a.H, a.T, a.Bt, NP2, QT,
                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&my, a.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P, a.H, a.T, a.Bt, P, Q, CU_TENSOR_MAP_SWIZZLE_128B))
+        !make_map(&my, a.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P, a.H, a.T, a.Bt, P, QT, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     TcArgs t;
     t.dt = a.dt; t.A = a.A; t.lam = a.lam; t.D = a.D;
+    t.Wx = a.Wx; t.Wy = a.Wy;
     t.h0 = a.h0; t.prevBx0 = a.prevBx0; t.angle0 = a.angle0;
     t.nrm = a.nrm;
     t.h_out = a.h_out; t.prevBx_out = a.prevBx_out; t.angle_out = a.angle_out;
     t.Bt = a.Bt; t.T = a.T; t.H = a.H;
+    const SegPlan pl = seg_plan(a.Bt * a.H, a.T);
+    t.nseg = pl.nseg;
+    t.seg_len = pl.seg_len;
+    t.ws = static_cast<float *>(a.ws);
     int *err = nullptr;
-    cudaGetSymbolAddress(reinterpret_cast<void **>(&err), g_tc_error);
+    cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void **>(&err), g_tc_error);
+    if (e != cudaSuccess) return e;
     t.err = err;
-    cudaFuncSetAttribute(k_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    k_scan_tc<<<(unsigned)(a.Bt * a.H), THREADS, SMEM_BYTES, s>>>(mx, mb, mc, mth, my, t);
+    const int64_t lanes = a.Bt * a.H;
+    constexpr int SMEM = smem_bytes<R>();
+    if (pl.nseg > 1) {
+        cudaFuncSetAttribute(k_scan_tc<true, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+        k_scan_tc<true, R><<<(unsigned)(lanes * (pl.nseg - 1)), THREADS, SMEM, s>>>(mx, mb, mc, mth, my, t);
+        count_launch();
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        k_seg_combine<<<dim3((unsigned)lanes, NP2 * P / 256), 256, 0, s>>>(t);
+        count_launch();
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    cudaFuncSetAttribute(k_scan_tc<false, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    k_scan_tc<false, R><<<(unsigned)(lanes * pl.nseg), THREADS, SMEM, s>>>(mx, mb, mc, mth, my, t);
     count_launch();
     return cudaGetLastError();
+}
+
+cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s) {
+    switch (a.R) {
+        case 1: return launch_tc_r<1>(a, s);
+        case 2: return launch_tc_r<2>(a, s);
+        case 4: return launch_tc_r<4>(a, s);
+    }
+    return cudaErrorInvalidValue;
 }
 
 int scan_tc_error_and_clear(cudaStream_t s) {

@@ -100,6 +100,7 @@ m3_status chunked_common(const void *x, const float *dt, const float *A, const f
     a.y = y; a.h_out = h_final; a.prevBx_out = prevBx_final; a.angle_out = angle_final;
     a.Bt = d.batch; a.T = d.seqlen; a.H = d.nheads; a.P = d.headdim; a.N = d.dstate; a.R = R;
     a.mimo_layout = mimo ? 1 : 0;
+    a.ws = workspace;
     a.Q = (int)d.chunk;
     if (scan_tc_supported(a, dtype)) return launched(launch_scan_tc(a, (cudaStream_t)stream));
     a.Q = q;
@@ -135,8 +136,14 @@ m3_status m3_device_error(void *stream, int *site) {
 }
 
 size_t m3_workspace_bytes(int which, m3_dims d, m3_dtype dtype) {
-    (void)which; (void)d; (void)dtype;
-    return 0;
+    // only the tensor-core path uses scratch (long sequences over few lanes)
+    if ((which != M3_WS_SISO && which != M3_WS_MIMO) || check_core_dims(d, true) != M3_OK || d.chunk < 1) return 0;
+    ScanArgs a{};
+    a.Bt = d.batch; a.T = d.seqlen; a.H = d.nheads; a.P = d.headdim; a.N = d.dstate;
+    a.R = which == M3_WS_MIMO ? d.rank : 1;
+    a.Q = (int)d.chunk; a.mimo_layout = which == M3_WS_MIMO ? 1 : 0;
+    if (!scan_tc_supported(a, dtype)) return 0;
+    return scan_tc_workspace_bytes(d.batch, d.nheads, d.seqlen);
 }
 
 m3_status m3_discretize(const float *dt, const float *A, const float *lam, m3_dims d, float *alpha,

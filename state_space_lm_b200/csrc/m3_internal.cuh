@@ -43,6 +43,7 @@ struct ScanArgs {
     int64_t Bt, T, H, P, N, R;
     int Q;             // chunk length actually used by the kernel
     int mimo_layout;   // B/C carry a rank axis
+    void *ws;          // caller's workspace (may be null when none is needed)
 };
 
 struct DecodeArgs {
@@ -76,6 +77,7 @@ cudaError_t launch_decode(const DecodeArgs &a, m3_dtype dt, cudaStream_t s);
 bool scan_tc_supported(const ScanArgs &a, m3_dtype dt);
 cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s);
 int scan_tc_error_and_clear(cudaStream_t s);
+size_t scan_tc_workspace_bytes(int64_t Bt, int64_t H, int64_t T);
 
 // Launch counter shared by all launchers.
 void count_launch(int n = 1);

@@ -121,3 +121,13 @@ def test_workspace_query(L):
     for which in (m3.M3_WS_SISO, m3.M3_WS_MIMO):
         n = m3.workspace_bytes(which, dims(), m3.M3_BF16)
         assert n >= 0
+    # long sequences over few lanes need scratch for the segment states
+    long3 = dims(batch=1, seqlen=32768, nheads=32, headdim=64, dstate=128, chunk=128)
+    need = m3.workspace_bytes(m3.M3_WS_SISO, long3, m3.M3_BF16)
+    assert need > 0
+    assert m3.workspace_bytes(m3.M3_WS_SISO, long3, m3.M3_F32) == 0      # FFMA path: no scratch
+    many = dims(batch=8, seqlen=2048, nheads=16, headdim=64, dstate=128, chunk=64)
+    assert m3.workspace_bytes(m3.M3_WS_SISO, many, m3.M3_BF16) == 0      # enough lanes: one segment
+    # a missing or short workspace is rejected before any launch
+    assert siso(L, long3) == m3.M3_ERR_WORKSPACE
+    assert siso(L, long3, ws=FAKE, nbytes=need - 16) == m3.M3_ERR_WORKSPACE

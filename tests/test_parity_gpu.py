@@ -157,6 +157,19 @@ def test_siso_bf16_ragged_lengths(T):
     assert m3.device_error() == m3.M3_OK
 
 
+@pytest.mark.parametrize("Bt,H,T,with_state", [(1, 2, 3000, True), (1, 1, 1000, False), (2, 3, 2560, True),
+                                                (1, 2, 600, True)])
+def test_siso_bf16_segmented_long_sequences(Bt, H, T, with_state):
+    # few lanes and long sequences: each lane is cut into segments that run in
+    # parallel (state-only pass, combine pass, full pass with workspace)
+    d = m3.Dims(Bt, T, H, 64, 128, 1, 64)
+    assert m3.workspace_bytes(m3.M3_WS_SISO, d, m3.M3_BF16) > 0
+    inp = gen.scan_inputs(Bt, T, H, 64, 128, dtype=BF16, seed=300 + T, dt_shift=-4.0)
+    errs = _siso_check(inp, 64, with_state=with_state, seed=T)
+    assert max(errs) <= 2e-2, errs
+    assert m3.device_error() == m3.M3_OK
+
+
 def test_siso_empty_sequence_passes_state_through():
     inp = gen.scan_inputs(2, 0, 3, 8, 6, dtype=FP32, seed=5)
     h0, u0, a0 = _states(2, 3, 6, 8, 9)
@@ -211,11 +224,29 @@ def test_mimo_fp32_norm_bias():
     assert max(errs) <= 1e-5, errs
 
 
-@pytest.mark.parametrize("T", [40, 129])
-def test_mimo_bf16_layer_shape(T):
-    inp = gen.scan_inputs(1, T, 2, 64, 128, rank=4, dtype=BF16, seed=62 + T, mimo_weights=True)
+@pytest.mark.parametrize("R,T", [(4, 40), (4, 129), (4, 1), (4, 17), (2, 100), (2, 33)])
+def test_mimo_bf16_layer_shape(R, T):
+    # headdim 64, dState 128, rank 2 or 4: the tensor-core path (64 rows per chunk)
+    inp = gen.scan_inputs(2, T, 2, 64, 128, rank=R, dtype=BF16, seed=62 + T + R, mimo_weights=True)
     errs = _mimo_check(inp, 64, with_state=True, seed=4)
     assert max(errs) <= 2e-2, errs
+    assert m3.device_error() == m3.M3_OK
+
+
+def test_mimo_bf16_norm_bias():
+    inp = gen.scan_inputs(1, 70, 2, 64, 128, rank=4, dtype=BF16, seed=65, mimo_weights=True, bcnorm=True)
+    errs = _mimo_check(inp, 64, with_state=True, seed=5)
+    assert max(errs) <= 2e-2, errs
+
+
+@pytest.mark.parametrize("R,T", [(4, 1000), (2, 700)])
+def test_mimo_bf16_segmented(R, T):
+    d = m3.Dims(1, T, 2, 64, 128, R, 64)
+    assert m3.workspace_bytes(m3.M3_WS_MIMO, d, m3.M3_BF16) > 0
+    inp = gen.scan_inputs(1, T, 2, 64, 128, rank=R, dtype=BF16, seed=66 + T, mimo_weights=True, dt_shift=-4.0)
+    errs = _mimo_check(inp, 64, with_state=True, seed=6)
+    assert max(errs) <= 2e-2, errs
+    assert m3.device_error() == m3.M3_OK
 
 
 # ----------------------------------------------------------------------------
