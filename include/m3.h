@@ -166,6 +166,41 @@ m3_status m3_step_decode(const void *x_t, const float *dt_t, const float *A,
                          const m3_bcnorm *norm, m3_dims d, float *h, float *prevBx,
                          float *angle, void *y_t, void *stream);
 
+/* Size in bytes of the scratch buffer built into the library for
+ * m3_siso_chunked_fwd_noalloc (32 MiB). */
+#define M3_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/* The SISO chunked forward for callers that cannot allocate device memory.
+ * The paper has no counterpart to this entry point; it is a deployment
+ * variant of m3_siso_chunked_fwd.
+ *
+ * Who it is for: code that may not call cudaMalloc (or any allocator) --
+ * a plugin running inside a framework that owns all device memory, or a
+ * host that must not allocate once it is serving -- has nowhere to take a
+ * workspace from.  This entry point takes the arguments of
+ * m3_siso_chunked_fwd without the workspace, and uses instead a scratch
+ * buffer of M3_NOALLOC_SCRATCH_BYTES that is part of the library: a static
+ * device array, held on every GPU that loads the library until the process
+ * exits.  It allocates nothing and calls no allocating routine.
+ *  - Set-up: the first call on each device looks up the buffer's device
+ *    address (cudaGetSymbolAddress, with that device current).  Make that
+ *    first call before any stream capture.
+ *  - Limit: sizes whose scratch need, m3_workspace_bytes(M3_WS_SISO, d,
+ *    dtype), exceeds M3_NOALLOC_SCRATCH_BYTES are rejected with
+ *    M3_ERR_WORKSPACE before anything is enqueued.
+ *  - Sharing: every call on a device uses the same buffer, and the buffer
+ *    keeps the last call's contents (nothing in it needs to start at zero).
+ *    Calls that can overlap on the GPU -- on different streams, or from
+ *    different host threads -- race on it; the caller must serialise them.
+ * Results, errors and all other rules are those of m3_siso_chunked_fwd. */
+m3_status m3_siso_chunked_fwd_noalloc(const void *x, const float *dt, const float *A,
+                                      const float *lam, const float *theta, const void *B,
+                                      const void *C, const float *D, m3_dtype dtype,
+                                      const m3_bcnorm *norm, const float *h0,
+                                      const float *prevBx0, const float *angle0, m3_dims d,
+                                      void *y, float *h_final, float *prevBx_final,
+                                      float *angle_final, void *stream);
+
 /* Workspace query for the chunked forwards. */
 enum { M3_WS_SISO = 0, M3_WS_MIMO = 1 };
 size_t m3_workspace_bytes(int which, m3_dims d, m3_dtype dtype);

@@ -22,7 +22,7 @@ _DTYPE = {torch.float32: M3_F32, torch.bfloat16: M3_BF16}
 ABI_FUNCTIONS = (
     "m3_get_limits", "m3_discretize", "m3_rope_bc", "m3_siso_chunked_fwd",
     "m3_mimo_chunked_fwd", "m3_step_decode", "m3_workspace_bytes", "m3_status_string",
-    "m3_launch_count", "m3_device_error",
+    "m3_launch_count", "m3_device_error", "m3_siso_chunked_fwd_noalloc",
 )
 
 
