@@ -276,6 +276,50 @@ class ScanWorkload:
         return nl, dt, used
 
 
+class DecodeWorkload:
+    """Decode steps of the SISO scan: every step advances all (batch, head)
+    lanes by one token.  The carried state comes from a seeded prefill (a
+    chunked forward over the first ``seqlen`` tokens, untimed); the per-step
+    inputs of every step are drawn up front and resident in HBM."""
+
+    def __init__(self, idx, device, nsteps):
+        from state_space_lm_b200 import m3
+        self.m3 = m3
+        self.c = dict(gen.CONFIGS[idx])
+        c = self.c
+        Bt, H, P, N = c["batch"], c["nheads"], c["headdim"], c["dstate"]
+        inp = gen.config_inputs(idx)
+        g = inp.pop("generator")
+        self.host_prefill = inp
+        d = {k: v.to(device) for k, v in inp.items() if isinstance(v, torch.Tensor)}
+        _, self.h, self.u, self.a = m3.siso_chunked_fwd(d["x"], d["dt"], d["A"], d["lam"], d["theta"], d["B"],
+                                                        d["C"], d["D"], c["chunk"])
+        self.A, self.D = d["A"], d["D"]
+        self.steps_host = [gen.decode_step_inputs(g, Bt, H, P, N) for _ in range(nsteps)]
+        self.steps_dev = [{k: v.to(device) for k, v in st.items()} for st in self.steps_host]
+        self.y = torch.empty(Bt, H, P, device=device, dtype=torch.bfloat16)
+        self.i = 0
+        self.units = Bt                           # one token per sequence per step
+        self.bytes = decode_bytes(c)
+        self.flops = 0
+        self.kernel = self.kernel_label = "k_decode"
+        self.srcs = [os.path.join(ROOT, "state_space_lm_b200", "csrc", "k_decode.cu")]
+        self.input_bytes = 2 * Bt * H * N * P * 4
+
+    def step(self, dev=None, out=None, stream=None):
+        st = self.steps_dev[self.i % len(self.steps_dev)] if dev is None else dev
+        self.i += 1
+        self.m3.step_decode(st["x"], st["dt"], self.A, st["lam"], st["theta"], st["B"], st["C"], self.D,
+                            self.h, self.u, self.a, y_out=self.y if out is None else out, stream=stream)
+
+    def config(self):
+        c = self.c
+        return {"workload": c["name"], "batch": c["batch"], "nheads": c["nheads"], "headdim": c["headdim"],
+                "dstate": c["dstate"], "prefill": c["seqlen"], "decode_steps_per_call": 1,
+                "inputs": "x/B/C bf16, dt/lam/theta fp32 per step; fp32 state h, prev_Bx, angle",
+                "l2": "state larger than L2 (%.0f MB vs 126 MB), no flush" % (self.input_bytes / 1e6)}
+
+
 def run_cpu_baseline(w, target_s=10.0):
     """Time the oracle as it stands on the host cores on a bounded sample of
     lanes; tokens/s are scaled to whole (b, t) tokens of all heads."""
@@ -304,7 +348,10 @@ def run_ours(args, world, rank, local):
     from state_space_lm_b200 import build, m3
     if not os.path.exists(build.LIB):
         raise SystemExit("CUDA library not built: run python -m state_space_lm_b200.build")
-    w = ScanWorkload(args.config, device)
+    if args.config == 4:
+        w = DecodeWorkload(args.config, device, args.steps + args.warmup)
+    else:
+        w = ScanWorkload(args.config, device)
     stream = torch.cuda.current_stream(device)
 
     for _ in range(args.warmup):
@@ -336,18 +383,34 @@ def run_ours(args, world, rank, local):
     value, tmax, units = aggregate(elapsed, w.units * args.steps, dist, device)
 
     # ---- end to end through the C ABI with host buffers ----
-    pinned = {k: v.pin_memory() for k, v in w.host.items() if isinstance(v, torch.Tensor)}
-    hout = tuple(torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in w.out)
-    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
-    d2h = sum(o.numel() * o.element_size() for o in hout)
     e2e_steps = max(3, min(args.steps, 20))
+    if isinstance(w, DecodeWorkload):
+        pinned = [{k: v.pin_memory() for k, v in st.items()} for st in w.steps_host[:e2e_steps]]
+        stage = {k: torch.empty_like(v) for k, v in w.steps_dev[0].items()}
+        hy = torch.empty(w.y.shape, dtype=w.y.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in pinned[0].values())
+        d2h = hy.numel() * hy.element_size()
+        e2e_i = [0]
 
-    def e2e_step():
-        for k, v in pinned.items():
-            w.dev[k].copy_(v, non_blocking=True)
-        w.step()
-        for o, ho in zip(w.out, hout):
-            ho.copy_(o, non_blocking=True)
+        def e2e_step():
+            src = pinned[e2e_i[0] % len(pinned)]
+            e2e_i[0] += 1
+            for k, v in src.items():
+                stage[k].copy_(v, non_blocking=True)
+            w.step(dev=stage)
+            hy.copy_(w.y, non_blocking=True)
+    else:
+        pinned = {k: v.pin_memory() for k, v in w.host.items() if isinstance(v, torch.Tensor)}
+        hout = tuple(torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in w.out)
+        h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+        d2h = sum(o.numel() * o.element_size() for o in hout)
+
+        def e2e_step():
+            for k, v in pinned.items():
+                w.dev[k].copy_(v, non_blocking=True)
+            w.step()
+            for o, ho in zip(w.out, hout):
+                ho.copy_(o, non_blocking=True)
 
     for _ in range(2):
         e2e_step()
@@ -384,7 +447,7 @@ def run_ours(args, world, rank, local):
             "e2e": {"value": round(e2e_val, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "clocks": clk.report(), "gpu_launches": int(launches)}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and isinstance(w, ScanWorkload):
         line["cpu_baseline"] = run_cpu_baseline(w)
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -440,7 +503,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=1, choices=[0, 1, 2, 3])
+    ap.add_argument("--config", type=int, default=1, choices=[0, 1, 2, 3, 4])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -57,6 +57,8 @@
 namespace m3 {
 namespace tc {
 
+template <bool V> struct BoolC { static constexpr bool value = V; };
+
 constexpr int Q = 64, P = 64, N = 128, NP2 = 64;
 constexpr int NWARPS = 19, THREADS = NWARPS * 32;
 constexpr int W_TMA = 0, W_MMA = 1, W_COEF = 2, W_PREP0 = 3, NPREP = 8, W_EPI0 = 11;
@@ -68,28 +70,27 @@ constexpr int EPI_THREADS = 256;                  // two warps per TMEM lane qua
 // the x, theta and output tiles have QT rows, and MIMO (R > 1) adds the
 // rank-expanded X_r = W_x[r] * x, the W_x / W_y vectors and R rows of the
 // last token's rotated B.
-constexpr int NB = 2, NX = 3, NC = 4;             // ring depths: B/C/theta, x, coefficients
+constexpr int NB = 2, NX = 3, NC = 4;             // ring depths: B/C, x, coefficients
 constexpr int SZ_BC = Q * N * 2;                  // 16 KB, bf16, row-major (TMA)
 constexpr int SZ_SP = Q * Q * 2, SZ_GB = N * P * 2;
 // per-chunk coefficient buffer (a ring of NC), floats; per token of the chunk
 constexpr int CF_W = 0, CF_GAM = Q, CF_E = 2 * Q, CF_R = 3 * Q, CF_EC = 4 * Q, CF_XS = 5 * Q,
-              CF_C2 = 6 * Q, CF_DT = 7 * Q, CF_SCAL = 8 * Q, CF_FLOATS = 8 * Q + 8;
+              CF_C2 = 6 * Q, CF_DT = 7 * Q, CF_WM = 8 * Q, CF_SCAL = 9 * Q, CF_FLOATS = 9 * Q + 8;
 template <int R>
 struct Lay {
     static constexpr int QT = Q / R;
+    static constexpr int NXR = (R == 2) ? 2 : NX;             // x ring depth (rank 2: shared memory is full)
     static constexpr int SZ_X = QT * P * 2;                   // bf16, 128B-swizzled (TMA)
-    static constexpr int SZ_TH = QT * NP2 * 4;                // fp32, row-major (TMA)
-    static constexpr int SZ_BCT = 2 * SZ_BC + SZ_TH;          // one B/C/theta stage
-    static constexpr int OFF_BCT = 0;                         // NB x [B | C | theta]
+    static constexpr int SZ_BCT = 2 * SZ_BC;                  // one B/C stage
+    static constexpr int OFF_BCT = 0;                         // NB x [B | C]
     static constexpr int OFF_X = OFF_BCT + NB * SZ_BCT;       // NX x [QT][P]
-    static constexpr int OFF_BSC = OFF_X + NX * SZ_X;         // [2 atoms][Q rows][64] bf16, SW128
-    static constexpr int OFF_CB = OFF_BSC + Q * N * 2;        // [2 atoms][Q rows][64] bf16, SW128
-    static constexpr int OFF_SP = OFF_CB + Q * N * 2;         // [Q][Q] bf16, SW128
-    static constexpr int OFF_XW = OFF_SP + SZ_SP;             // [Q rows][P] bf16, SW128
-    static constexpr int OFF_XR = OFF_XW + Q * P * 2;         // [Q rows][P] bf16, SW128 (R > 1)
-    static constexpr int OFF_GB = OFF_XR + (R > 1 ? Q * P * 2 : 0);   // 2 x [N][P] bf16, SW128
-    static constexpr int OFF_YT = OFF_GB + 2 * SZ_GB;         // [QT][P] bf16, SW128
-    static constexpr int OFF_COEF = OFF_YT + ((QT * P * 2 + 1023) / 1024) * 1024;
+    static constexpr int OFF_BSC = ((OFF_X + NXR * SZ_X + 1023) / 1024) * 1024;   // 2 x [2 atoms][Q rows][64]
+    static constexpr int OFF_CB = OFF_BSC + 2 * Q * N * 2;    // 2 x [2 atoms][Q rows][64] bf16, SW128
+    static constexpr int OFF_SP = OFF_CB + 2 * Q * N * 2;     // [Q][Q] bf16, SW128
+    static constexpr int OFF_XW = OFF_SP + SZ_SP;             // 2 x [Q rows][P] bf16, SW128
+    static constexpr int OFF_XR = OFF_XW + 2 * Q * P * 2;     // 2 x [Q rows][P] bf16, SW128 (R > 1)
+    static constexpr int OFF_GB = OFF_XR + (R > 1 ? 2 * Q * P * 2 : 0);   // 2 x [N][P] bf16, SW128
+    static constexpr int OFF_COEF = OFF_GB + 2 * SZ_GB;
     static constexpr int OFF_BLAST = OFF_COEF + NC * CF_FLOATS * 4;  // fp32 [R][N]
     static constexpr int OFF_WXY = OFF_BLAST + R * N * 4;            // fp32 [2][R][P] (R > 1)
     static constexpr int OFF_PHIC = OFF_WXY + (R > 1 ? 2 * R * P * 4 : 0);  // fp32 [NP2]
@@ -106,9 +107,10 @@ enum {
     B_XEMPTY = B_XFULL + NX,        // NX: Xw built, intra UMMA done, outputs written
     B_CFULL = B_XEMPTY + NX,        // NC: coefficients ready
     B_CEMPTY = B_CFULL + NC,        // NC: coefficients consumed
-    B_OPSREADY = B_CEMPTY + NC,     // rotated operands and Xw written
-    B_OPSFREE,                      // UMMAs reading them are done
-    B_SFULL, B_STAKEN, B_SPFULL,    // scores in TMEM / read / masked scores written
+    B_OPSREADY = B_CEMPTY + NC,     // 2: rotated operands and Xw written (double-buffered)
+    B_OPSFREE = B_OPSREADY + 2,     // 2: the UMMAs reading them are done
+    B_SFULL = B_OPSFREE + 2,
+    B_STAKEN, B_SPFULL,             // scores in TMEM / read / masked scores written
     B_YFULL, B_YTAKEN,              // output accumulators done / read
     B_STFULL, B_STTAKEN,            // chunk state done / folded into the state
     B_DRAIN,
@@ -123,6 +125,8 @@ constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t COL_D1 = 0, COL_D2 = 64, COL_D3 = 128, COL_D4 = 192;
 
 struct TcArgs {
+    void *y;               // (Bt, T, H, P) bf16
+    const float *theta;    // (Bt, T, H, N/2) fp32
     const float *dt, *A, *lam, *D;
     const float *Wx, *Wy;  // MIMO expand / contract vectors (H, R, P), NULL = ones
     const float *h0, *prevBx0, *angle0;
@@ -183,12 +187,13 @@ __device__ __forceinline__ bool mbar_try_spin(uint32_t bar, uint32_t parity) {
 constexpr long long WAIT_LIMIT_CYCLES = 2000000000LL;  // ~1 s at 1.9 GHz
 
 // Bounded wait without the suspend hint (for the single MMA-issuing thread).
-__device__ __forceinline__ bool wait_bar_spin(uint32_t bar, uint32_t parity, volatile int *abort_flag, int *err,
-                                              int site) {
-    if (mbar_try_spin(bar, parity)) return true;
+// The first probe is inline; the polling loop is one out-of-line copy shared
+// by every call site, which keeps the hot loops of the kernel small.
+__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag, int *err,
+                                           int site, bool spin) {
     const long long t0 = clock64();
     while (true) {
-        if (mbar_try_spin(bar, parity)) return true;
+        if (spin ? mbar_try_spin(bar, parity) : mbar_try(bar, parity)) return true;
         if (*abort_flag) return false;
         if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
             *abort_flag = 1;
@@ -197,22 +202,16 @@ __device__ __forceinline__ bool wait_bar_spin(uint32_t bar, uint32_t parity, vol
         }
     }
 }
+__device__ __forceinline__ bool wait_bar_spin(uint32_t bar, uint32_t parity, volatile int *abort_flag, int *err,
+                                              int site) {
+    return mbar_try_spin(bar, parity) || wait_bar_slow(bar, parity, abort_flag, err, site, true);
+}
 
 // Bounded wait on an mbarrier phase.  Returns false when the kernel is
 // aborting (this wait timed out, or another thread's did).
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag, int *err,
                                          int site) {
-    if (mbar_try(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (true) {
-        if (mbar_try(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
-            *abort_flag = 1;
-            atomicCAS(err, 0, site);
-            return false;
-        }
-    }
+    return mbar_try(bar, parity) || wait_bar_slow(bar, parity, abort_flag, err, site, false);
 }
 
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
@@ -339,8 +338,7 @@ __device__ __forceinline__ void sincos_rr(float x, float *s, float *c) {
 template <bool SO, int R>
 __global__ void __launch_bounds__(THREADS, 1)
     k_scan_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
-              const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_th,
-              const __grid_constant__ CUtensorMap map_y, TcArgs a) {
+              const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_th, TcArgs a) {
     using L = Lay<R>;
     constexpr int QT = L::QT;                          // tokens per chunk
     constexpr int TPT = QT / 16;                       // tokens per rotation thread
@@ -377,7 +375,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         // x tiles are released by the Xw builder, the intra UMMA and the output
         // writer (state-only pass: the Xw builder alone)
-        for (int i = 0; i < NX; i++) {
+        for (int i = 0; i < L::NXR; i++) {
             mbar_init(bar(B_XFULL + i), 1);
             mbar_init(bar(B_XEMPTY + i), SO ? 1 : 3);
         }
@@ -385,8 +383,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(bar(B_CFULL + i), 1);
             mbar_init(bar(B_CEMPTY + i), 2);
         }
-        mbar_init(bar(B_OPSREADY), 1);
-        mbar_init(bar(B_OPSFREE), 1);
+        for (int i = 0; i < 2; i++) {
+            mbar_init(bar(B_OPSREADY + i), 1);
+            mbar_init(bar(B_OPSFREE + i), 1);
+        }
         mbar_init(bar(B_SFULL), 1);
         mbar_init(bar(B_STAKEN), 8);
         mbar_init(bar(B_SPFULL), 8);
@@ -401,7 +401,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         asm volatile("prefetch.tensormap [%0];" ::"l"(&map_b) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&map_c) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&map_th) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(&map_y) : "memory");
     }
     if (warp == W_MMA) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -452,16 +451,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int c = 1; c < PFD; c++) prefetch(c);
             int issued = 0;
             for (int c = 0; c < nchunks; c++) {
-                const int sb = c % NB, kb = c / NB, sx = c % NX, kx = c / NX;
+                const int sb = c % NB, kb = c / NB, sx = c % L::NXR, kx = c / L::NXR;
                 const int t0 = (int)(t_beg + (int64_t)c * QT);
                 prefetch(c + PFD);
                 if (kb > 0 && !wait_bar(bar(B_BEMPTY + sb), (kb - 1) & 1, abort_flag, a.err, 1)) break;
                 const uint32_t st = sbase + L::OFF_BCT + sb * L::SZ_BCT;
                 const uint32_t fb = bar(B_BFULL + sb);
-                mbar_expect_tx(fb, SO ? SZ_BC + L::SZ_TH : L::SZ_BCT);
+                mbar_expect_tx(fb, SO ? SZ_BC : L::SZ_BCT);
                 load_bc(st, &map_b, t0, fb);
                 if (!SO) load_bc(st + SZ_BC, &map_c, t0, fb);
-                tma_load4(st + 2 * SZ_BC, &map_th, 0, (int)h, t0, (int)b, fb);
                 if (kx > 0 && !wait_bar(bar(B_XEMPTY + sx), (kx - 1) & 1, abort_flag, a.err, 2)) break;
                 const uint32_t xb = bar(B_XFULL + sx);
                 mbar_expect_tx(xb, L::SZ_X);
@@ -469,9 +467,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                 issued = c + 1;
             }
             // never leave loads in flight into shared memory at exit
-            for (int c = (issued > NX ? issued - NX : 0); c < issued; c++) {
+            for (int c = (issued > L::NXR ? issued - L::NXR : 0); c < issued; c++) {
                 const long long t0 = clock64();
-                while (!mbar_try(bar(B_XFULL + c % NX), (c / NX) & 1) && clock64() - t0 < WAIT_LIMIT_CYCLES) {
+                while (!mbar_try(bar(B_XFULL + c % L::NXR), (c / L::NXR) & 1) && clock64() - t0 < WAIT_LIMIT_CYCLES) {
                 }
             }
             for (int c = (issued > NB ? issued - NB : 0); c < issued; c++) {
@@ -540,10 +538,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const int i = l32 + 32 * u;
                 if (i < QT) {
                     const float e = exp2f(cend - la[u]);
+                    // mask factors: row r_t and column w_s, or ones when the chunk
+                    // takes the exact path (the scores then get e^{cum_t-cum_s} w_s
+                    // one by one)
                     cf[CF_W + i] = wv[u];
+                    cf[CF_WM + i] = unsafe ? 1.f : wv[u];
                     cf[CF_GAM + i] = gv[u];
                     cf[CF_E + i] = unsafe ? 1.f : e;
-                    cf[CF_R + i] = exp2f(la[u] - cend);
+                    cf[CF_R + i] = unsafe ? 1.f : exp2f(la[u] - cend);
                     cf[CF_EC + i] = exp2f(la[u]);
                     cf[CF_XS + i] = unsafe ? e * wv[u] : wv[u];
                     cf[CF_C2 + i] = la[u];
@@ -567,25 +569,40 @@ __global__ void __launch_bounds__(THREADS, 1)
         const NormArgs nr = a.nrm;
         const bool has_norm = nr.wB || nr.wC;
         const bool has_bias = nr.biasB || nr.biasC;
-        uint8_t *bsc = sm + L::OFF_BSC;
-        uint8_t *cb = sm + L::OFF_CB;
         const uint32_t atom = (uint32_t)(j4 >> 3) * (Q * 128);
         const int chk = j4 & 7;                    // 16-byte chunk within the 128-byte atom row
+        const int i0 = tg * TPT;
+        // theta of my tokens comes straight from global memory into registers,
+        // one chunk ahead (the producer has already pulled it into L2)
+        const float4 *thg = reinterpret_cast<const float4 *>(a.theta);
+        float4 thv[TPT];
+        auto load_theta = [&](int c) {
+            const int64_t t0 = t_beg + (int64_t)c * QT;
+#pragma unroll
+            for (int u = 0; u < TPT; u++) {
+                const int64_t t = t0 + i0 + u;
+                thv[u] = (c < nchunks && t < t_end) ? thg[((b * Tn + t) * H + h) * (NP2 / 4) + j4]
+                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        };
+        load_theta(0);
         for (int c = 0; c < nchunks; c++) {
-            const int sb = c % NB, kb = c / NB, sx = c % NX, kx = c / NX, scf = c % NC, kc = c / NC;
+            const int sb = c % NB, kb = c / NB, sx = c % L::NXR, kx = c / L::NXR, scf = c % NC, kc = c / NC;
+            const int ob = c & 1;                  // operand buffer
             bool fail = false;
             if (pt == 0) {
                 fail = !(wait_bar(bar(B_BFULL + sb), kb & 1, abort_flag, a.err, 4) &&
                          wait_bar(bar(B_XFULL + sx), kx & 1, abort_flag, a.err, 5) &&
                          wait_bar(bar(B_CFULL + scf), kc & 1, abort_flag, a.err, 6) &&
-                         (c == 0 || wait_bar(bar(B_OPSFREE), (c - 1) & 1, abort_flag, a.err, 7)));
+                         (c < 2 || wait_bar(bar(B_OPSFREE + ob), ((c >> 1) - 1) & 1, abort_flag, a.err, 7)));
             }
             if (named_bar_or(1, PREP_THREADS, fail)) break;
+            uint8_t *bsc = sm + L::OFF_BSC + ob * (Q * N * 2);
+            uint8_t *cb = sm + L::OFF_CB + ob * (Q * N * 2);
             const float *cf = coef0 + scf * CF_FLOATS;
             const uint8_t *stg = sm + L::OFF_BCT + sb * L::SZ_BCT;
             const uint4 *braw = reinterpret_cast<const uint4 *>(stg);
             const uint4 *craw = reinterpret_cast<const uint4 *>(stg + SZ_BC);
-            const float4 *th = reinterpret_cast<const float4 *>(stg + 2 * SZ_BC);
             const int Lc = (int)cf[CF_SCAL + 2];
             if (has_norm) {
                 // inverse RMS of each B and C row of the chunk: one warp per row
@@ -605,13 +622,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
             }
             // pass 1: angle increments of my token group
-            const int i0 = tg * TPT;
             float dph[TPT][4];
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int u = 0; u < TPT; u++) {
                 const float d = cf[CF_DT + i0 + u];
-                const float4 t4 = th[(i0 + u) * 16 + j4];
+                const float4 t4 = thv[u];
                 dph[u][0] = d * t4.x;
                 dph[u][1] = d * t4.y;
                 dph[u][2] = d * t4.z;
@@ -630,66 +646,83 @@ __global__ void __launch_bounds__(THREADS, 1)
                     phi[0] += pg.x; phi[1] += pg.y; phi[2] += pg.z; phi[3] += pg.w;
                 }
             }
-            // pass 2: rotate my tokens (the same angles for every rank)
+            // pass 2: rotate my tokens (the same angles for every rank).  The
+            // token loop stays rolled (a small hot loop); the QkNorm / bias
+            // variant is a separate copy of it, so the plain one carries none
+            // of that code.
             const bool last_chunk = last_seg && (c == nchunks - 1);
-#pragma unroll
-            for (int u = 0; u < TPT; u++) {
-                const int i = i0 + u;
-#pragma unroll
-                for (int q = 0; q < 4; q++) phi[q] += dph[u][q];
-                float sn[4], cs[4];
-#pragma unroll
-                for (int q = 0; q < 4; q++) sincos_rr(phi[q], &sn[q], &cs[q]);
-                const float e = cf[CF_E + i];
+            auto rotate_tokens = [&](auto generic) {
+                constexpr bool G = decltype(generic)::value;
 #pragma unroll 1
-                for (int r = 0; r < R; r++) {
-                    const int row = i * R + r;
-                    uint4 ob = make_uint4(0u, 0u, 0u, 0u), oc = make_uint4(0u, 0u, 0u, 0u);
-                    if (i < Lc) {
-                        const uint4 rb = braw[row * 16 + j4];
-                        const uint4 rc = SO ? make_uint4(0u, 0u, 0u, 0u) : craw[row * 16 + j4];
-                        const uint32_t rbw[4] = {rb.x, rb.y, rb.z, rb.w}, rcw[4] = {rc.x, rc.y, rc.z, rc.w};
-                        uint32_t pbw[4], pcw[4];
-                        const float ib = (has_norm && nr.wB) ? inv[row] : 1.f;
-                        const float ic = (has_norm && nr.wC) ? inv[Q + row] : 1.f;
+                for (int u = 0; u < TPT; u++) {
+                    const int i = i0 + u;
+                    float d[4] = {dph[0][0], dph[0][1], dph[0][2], dph[0][3]};
 #pragma unroll
-                        for (int q = 0; q < 4; q++) {
-                            float2 bv = unpack_bf16(rbw[q]), cv = unpack_bf16(rcw[q]);
-                            const int e0 = 8 * j4 + 2 * q;
-                            if (has_norm) {
-                                if (nr.wB) { bv.x *= ib * nr.wB[e0]; bv.y *= ib * nr.wB[e0 + 1]; }
-                                if (nr.wC) { cv.x *= ic * nr.wC[e0]; cv.y *= ic * nr.wC[e0 + 1]; }
-                            }
-                            if (has_bias) {
-                                const int64_t bo = (h * R + r) * N + e0;
-                                if (nr.biasB) { bv.x += nr.biasB[bo]; bv.y += nr.biasB[bo + 1]; }
-                                if (nr.biasC) { cv.x += nr.biasC[bo]; cv.y += nr.biasC[bo + 1]; }
-                            }
-                            const float rb0 = cs[q] * bv.x - sn[q] * bv.y, rb1 = sn[q] * bv.x + cs[q] * bv.y;
-                            pbw[q] = pack_bf16(rb0 * e, rb1 * e);
-                            if (!SO) pcw[q] = pack_bf16(cs[q] * cv.x - sn[q] * cv.y, sn[q] * cv.x + cs[q] * cv.y);
-                            else pcw[q] = 0u;
-                            if (last_chunk && i == Lc - 1) {
-                                blast[r * N + e0] = rb0;
-                                blast[r * N + e0 + 1] = rb1;
-                            }
+                    for (int k = 1; k < TPT; k++)
+                        if (u == k) {
+                            d[0] = dph[k][0]; d[1] = dph[k][1]; d[2] = dph[k][2]; d[3] = dph[k][3];
                         }
-                        ob = make_uint4(pbw[0], pbw[1], pbw[2], pbw[3]);
-                        oc = make_uint4(pcw[0], pcw[1], pcw[2], pcw[3]);
+                    float sn[4], cs[4];
+#pragma unroll
+                    for (int q = 0; q < 4; q++) {
+                        phi[q] += d[q];
+                        sincos_rr(phi[q], &sn[q], &cs[q]);
                     }
-                    const uint32_t off = atom + (uint32_t)(row * 128 + ((chk ^ (row & 7)) << 4));
-                    *reinterpret_cast<uint4 *>(bsc + off) = ob;
-                    if (!SO) *reinterpret_cast<uint4 *>(cb + off) = oc;
+                    const float e = cf[CF_E + i];
+#pragma unroll 1
+                    for (int r = 0; r < R; r++) {
+                        const int row = i * R + r;
+                        uint4 ob = make_uint4(0u, 0u, 0u, 0u), oc = make_uint4(0u, 0u, 0u, 0u);
+                        if (i < Lc) {
+                            const uint4 rb = braw[row * 16 + j4];
+                            const uint4 rc = SO ? make_uint4(0u, 0u, 0u, 0u) : craw[row * 16 + j4];
+                            const uint32_t rbw[4] = {rb.x, rb.y, rb.z, rb.w}, rcw[4] = {rc.x, rc.y, rc.z, rc.w};
+                            uint32_t pbw[4], pcw[4];
+                            float ib = 1.f, ic = 1.f;
+                            if (G) {
+                                ib = nr.wB ? inv[row] : 1.f;
+                                ic = nr.wC ? inv[Q + row] : 1.f;
+                            }
+#pragma unroll
+                            for (int q = 0; q < 4; q++) {
+                                float2 bv = unpack_bf16(rbw[q]), cv = unpack_bf16(rcw[q]);
+                                if (G) {
+                                    const int e0 = 8 * j4 + 2 * q;
+                                    const int64_t bo = (h * R + r) * N + e0;
+                                    if (nr.wB) { bv.x *= ib * nr.wB[e0]; bv.y *= ib * nr.wB[e0 + 1]; }
+                                    if (nr.wC) { cv.x *= ic * nr.wC[e0]; cv.y *= ic * nr.wC[e0 + 1]; }
+                                    if (nr.biasB) { bv.x += nr.biasB[bo]; bv.y += nr.biasB[bo + 1]; }
+                                    if (nr.biasC) { cv.x += nr.biasC[bo]; cv.y += nr.biasC[bo + 1]; }
+                                }
+                                const float rb0 = cs[q] * bv.x - sn[q] * bv.y, rb1 = sn[q] * bv.x + cs[q] * bv.y;
+                                pbw[q] = pack_bf16(rb0 * e, rb1 * e);
+                                if (!SO) pcw[q] = pack_bf16(cs[q] * cv.x - sn[q] * cv.y, sn[q] * cv.x + cs[q] * cv.y);
+                                else pcw[q] = 0u;
+                                if (last_chunk && i == Lc - 1) {
+                                    blast[r * N + 8 * j4 + 2 * q] = rb0;
+                                    blast[r * N + 8 * j4 + 2 * q + 1] = rb1;
+                                }
+                            }
+                            ob = make_uint4(pbw[0], pbw[1], pbw[2], pbw[3]);
+                            oc = make_uint4(pcw[0], pcw[1], pcw[2], pcw[3]);
+                        }
+                        const uint32_t off = atom + (uint32_t)(row * 128 + ((chk ^ (row & 7)) << 4));
+                        *reinterpret_cast<uint4 *>(bsc + off) = ob;
+                        if (!SO) *reinterpret_cast<uint4 *>(cb + off) = oc;
+                    }
                 }
-            }
+            };
+            if (has_norm || has_bias) rotate_tokens(BoolC<true>{});
+            else rotate_tokens(BoolC<false>{});
+            load_theta(c + 1);                     // in flight while the X operands are built
             // the X operands, 16-byte vectors of 128-byte rows (a vector keeps its
             // place under the swizzle, so its row is its index / 8):
             //   SISO:  Xw = diag(xs) x
             //   MIMO:  Xr[(s,r)] = W_x[r] x_s (intra UMMA), Xw[(s,r)] = xs_s Xr[(s,r)]
             {
                 const uint8_t *xt = sm + L::OFF_X + sx * L::SZ_X;
-                uint4 *dw = reinterpret_cast<uint4 *>(sm + L::OFF_XW);
-                uint4 *dr = reinterpret_cast<uint4 *>(sm + L::OFF_XR);
+                uint4 *dw = reinterpret_cast<uint4 *>(sm + L::OFF_XW + ob * (Q * P * 2));
+                uint4 *dr = reinterpret_cast<uint4 *>(sm + L::OFF_XR + ob * (Q * P * 2));
 #pragma unroll
                 for (int v = pt; v < Q * P / 8; v += PREP_THREADS) {
                     const int row = v >> 3, pc = v & 7;
@@ -739,7 +772,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         make_float4(phi[0], phi[1], phi[2], phi[3]);
             }
             if (pt == 0) {
-                mbar_arrive(bar(B_OPSREADY));
+                mbar_arrive(bar(B_OPSREADY + ob));
                 mbar_arrive(bar(B_BEMPTY + sb));
                 mbar_arrive(bar(B_XEMPTY + sx));
                 mbar_arrive(bar(B_CEMPTY + scf));
@@ -751,52 +784,65 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t id_kk = idesc(64, 64, 0, 0);    // D1 = Cbar . Bsc^T
             const uint32_t id_kmn = idesc(64, 64, 0, 1);   // D2, D3: B operand MN-major
             const uint32_t id_st = idesc(128, 64, 1, 1);   // D4: A and B MN-major
-            const uint32_t a_bsc = sbase + L::OFF_BSC, a_cb = sbase + L::OFF_CB, a_sp = sbase + L::OFF_SP;
-            const uint32_t a_xw = sbase + L::OFF_XW;
+            // Descriptors are built once; a K-step of a UMMA only moves the start
+            // address field (16-byte units, low bits of the descriptor).
+            // (a buffer switch adds its byte offset / 16 to the start field)
+            const uint64_t d_sp = sdesc(sbase + L::OFF_SP, 16, 1024);
+            const uint64_t d_bsc_k0 = sdesc(sbase + L::OFF_BSC, 16, 1024);
+            const uint64_t d_cb_k0 = sdesc(sbase + L::OFF_CB, 16, 1024);
+            const uint64_t d_bsc_mn0 = sdesc(sbase + L::OFF_BSC, Q * 128, 1024);
+            const uint64_t d_xw0 = sdesc(sbase + L::OFF_XW, Q * 128, 1024);
+            const uint64_t d_xr0 = sdesc(sbase + L::OFF_XR, Q * 128, 1024);
+            const uint64_t d_gb0 = sdesc(sbase + L::OFF_GB, N * 128, 1024);
+            const uint64_t d_x0 = sdesc(sbase + L::OFF_X, Q * 128, 1024);
+            constexpr uint64_t STEP_BC = (Q * N * 2) >> 4, STEP_XP = (Q * P * 2) >> 4, STEP_GB = SZ_GB >> 4;
+            constexpr uint64_t STEP_X = L::SZ_X >> 4;
+            // K-major operand, K-step kk of 16: 32 bytes inside a 128-byte atom row,
+            // the second atom (K 64..127) Q*128 bytes further
+            auto kstep_k = [](int kk) { return (uint64_t)(((kk >> 2) * (Q * 128) + (kk & 3) * 32) >> 4); };
+            // MN-major operand, K-step kk of 16: two 8-row groups of 1024 bytes
+            auto kstep_mn = [](int kk) { return (uint64_t)((kk * 2048) >> 4); };
             for (int c = 0; c < nchunks; c++) {
-                const int sx = c % NX;
-                // intra UMMA operand: the x tile itself (SISO) or the rank-expanded Xr
-                const uint32_t a_x = (R == 1) ? sbase + L::OFF_X + sx * L::SZ_X : sbase + L::OFF_XR;
-                const uint32_t a_gprev = sbase + L::OFF_GB + ((c + 1) & 1) * SZ_GB;   // state after chunk c-1
-                if (!wait_bar_spin(bar(B_OPSREADY), c & 1, abort_flag, a.err, 10)) break;
+                const int sx = c % L::NXR, ob = c & 1;
+                const uint64_t d_bsc_k = d_bsc_k0 + ob * STEP_BC, d_cb_k = d_cb_k0 + ob * STEP_BC;
+                const uint64_t d_bsc_mn = d_bsc_mn0 + ob * STEP_BC, d_xw = d_xw0 + ob * STEP_XP;
+                const uint64_t dx = (R == 1) ? d_x0 + (uint64_t)sx * STEP_X : d_xr0 + ob * STEP_XP;
+                const uint64_t dg = d_gb0 + ((c + 1) & 1) * STEP_GB;   // state after chunk c-1
+                if (!wait_bar_spin(bar(B_OPSREADY + ob), (c >> 1) & 1, abort_flag, a.err, 10)) break;
                 if (SO) {
                     // state-only pass: the chunk-state UMMA alone
                     if (!wait_bar_spin(bar(B_STTAKEN), c & 1, abort_flag, a.err, 12)) break;
                     tc_fence_after();
                     for (int kk = 0; kk < Q / 16; kk++)
-                        umma(tmem + COL_D4, sdesc(a_bsc + kk * 2048, Q * 128, 1024),
-                             sdesc(a_xw + kk * 2048, Q * 128, 1024), id_st, kk > 0);
+                        umma(tmem + COL_D4, d_bsc_mn + kstep_mn(kk), d_xw + kstep_mn(kk), id_st, kk > 0);
                     umma_commit(bar(B_STFULL));
-                    umma_commit(bar(B_OPSFREE));
+                    umma_commit(bar(B_OPSFREE + ob));
                     continue;
                 }
                 if (c > 0 && !wait_bar_spin(bar(B_STAKEN), (c - 1) & 1, abort_flag, a.err, 11)) break;
                 tc_fence_after();
-                for (int kk = 0; kk < N / 16; kk++) {
-                    const uint32_t off = (kk >> 2) * (Q * 128) + (kk & 3) * 32;
-                    umma(tmem + COL_D1, sdesc(a_cb + off, 16, 1024), sdesc(a_bsc + off, 16, 1024), id_kk, kk > 0);
-                }
+#pragma unroll 1
+                for (int kk = 0; kk < N / 16; kk++)
+                    umma(tmem + COL_D1, d_cb_k + kstep_k(kk), d_bsc_k + kstep_k(kk), id_kk, kk > 0);
                 umma_commit(bar(B_SFULL));
                 if (!wait_bar_spin(bar(B_STTAKEN), c & 1, abort_flag, a.err, 12)) break;
                 tc_fence_after();
+#pragma unroll 1
                 for (int kk = 0; kk < Q / 16; kk++)
-                    umma(tmem + COL_D4, sdesc(a_bsc + kk * 2048, Q * 128, 1024), sdesc(a_xw + kk * 2048, Q * 128, 1024),
-                         id_st, kk > 0);
+                    umma(tmem + COL_D4, d_bsc_mn + kstep_mn(kk), d_xw + kstep_mn(kk), id_st, kk > 0);
                 umma_commit(bar(B_STFULL));
                 if (c > 0 && !wait_bar_spin(bar(B_YTAKEN), (c - 1) & 1, abort_flag, a.err, 13)) break;
                 tc_fence_after();
-                for (int kk = 0; kk < N / 16; kk++) {
-                    const uint32_t off = (kk >> 2) * (Q * 128) + (kk & 3) * 32;
-                    umma(tmem + COL_D3, sdesc(a_cb + off, 16, 1024), sdesc(a_gprev + kk * 2048, N * 128, 1024), id_kmn,
-                         kk > 0);
-                }
-                umma_commit(bar(B_OPSFREE));
+#pragma unroll 1
+                for (int kk = 0; kk < N / 16; kk++)
+                    umma(tmem + COL_D3, d_cb_k + kstep_k(kk), dg + kstep_mn(kk), id_kmn, kk > 0);
                 if (!wait_bar_spin(bar(B_SPFULL), c & 1, abort_flag, a.err, 14)) break;
                 tc_fence_after();
+#pragma unroll 1
                 for (int kk = 0; kk < Q / 16; kk++)
-                    umma(tmem + COL_D2, sdesc(a_sp + kk * 32, 16, 1024), sdesc(a_x + kk * 2048, Q * 128, 1024), id_kmn,
-                         kk > 0);
+                    umma(tmem + COL_D2, d_sp + (uint64_t)((kk * 32) >> 4), dx + kstep_mn(kk), id_kmn, kk > 0);
                 umma_commit(bar(B_YFULL));
+                umma_commit(bar(B_OPSFREE + ob));      // every operand of chunk c has been read
                 umma_commit(bar(B_XEMPTY + sx));
             }
             // drain: every MMA issued so far has completed before TMEM is freed
@@ -820,7 +866,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int et = tid - W_EPI0 * 32;            // 0..255
         const float Dh = a.D[h];
         uint8_t *sp = sm + L::OFF_SP;
-        uint8_t *yt = sm + L::OFF_YT;
+        __nv_bfloat16 *yg = static_cast<__nv_bfloat16 *>(a.y);
         // one thread waits, the group meets at a named barrier and leaves together
         auto group_wait = [&](int bi, uint32_t parity, int site) -> bool {
             bool fail = false;
@@ -913,7 +959,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             bool ok = true;
             for (int c = 0; c < nchunks && ok; c++) {
-                const int scf = c % NC, kc = c / NC, sx = c % NX;
+                const int scf = c % NC, kc = c / NC, sx = c % L::NXR;
                 const float *cf = coef0 + scf * CF_FLOATS;
                 const uint8_t *xr = sm + L::OFF_X + sx * L::SZ_X;
                 if (!(ok = group_wait(B_CFULL + scf, kc & 1, 20))) break;
@@ -924,24 +970,25 @@ __global__ void __launch_bounds__(THREADS, 1)
                 {
                     const int t = ttok;
                     const float rt = rowv ? cf[CF_R + t] : 0.f;
-                    const float c2t = rowv ? cf[CF_C2 + t] : 0.f;
                     const float gt = rowv ? cf[CF_GAM + t] : 0.f;
-#pragma unroll
+#pragma unroll 1
                     for (int c16 = 0; c16 < 2; c16++) {
                         const int s0 = cb0 + 16 * c16;
                         float v[16];
                         tmem_ld16(tl + COL_D1 + s0, v);
                         tmem_wait_ld();
                         if (rowv) {
+                            // column factors of the 16/R tokens of these columns
+                            float wm[16 / R];
+#pragma unroll
+                            for (int k4 = 0; k4 < 16 / R; k4 += 4) {
+                                const float4 w4 = *reinterpret_cast<const float4 *>(cf + CF_WM + s0 / R + k4);
+                                wm[k4] = w4.x; wm[k4 + 1] = w4.y; wm[k4 + 2] = w4.z; wm[k4 + 3] = w4.w;
+                            }
 #pragma unroll
                             for (int k2 = 0; k2 < 16 / R; k2++) {
-                                const int s2 = s0 / R + k2;      // token of columns k2*R .. k2*R+R-1
-                                const float wsv = cf[CF_W + s2];
-                                float m;
-                                if (!unsafe)
-                                    m = s2 < t ? rt * wsv : (s2 == t ? rt * gt : 0.f);
-                                else
-                                    m = s2 < t ? exp2f(c2t - cf[CF_C2 + s2]) * wsv : (s2 == t ? gt : 0.f);
+                                const int s2 = s0 / R + k2;  // token of columns k2*R .. k2*R+R-1
+                                const float m = s2 < t ? rt * wm[k2] : (s2 == t ? rt * gt : 0.f);
 #pragma unroll
                                 for (int r2 = 0; r2 < R; r2++) v[k2 * R + r2] *= m;
                             }
@@ -954,6 +1001,20 @@ __global__ void __launch_bounds__(THREADS, 1)
                                 pk.z = pack_bf16(v[8 * hh + 4], v[8 * hh + 5]);
                                 pk.w = pack_bf16(v[8 * hh + 6], v[8 * hh + 7]);
                                 *reinterpret_cast<uint4 *>(sp + trow * 128 + ((cc ^ (trow & 7)) << 4)) = pk;
+                            }
+                        }
+                    }
+                    if (unsafe && rowv) {
+                        // exact path: the scores below the diagonal were stored
+                        // unscaled; give each its factor e^{cum_t - cum_s} w_s here
+                        const float c2t = cf[CF_C2 + t];
+#pragma unroll 1
+                        for (int col = cb0; col < cb0 + 32; col++) {
+                            const int s2 = col / R;
+                            if (s2 < t) {
+                                __nv_bfloat16 *pv = reinterpret_cast<__nv_bfloat16 *>(sp + sw128(trow, col));
+                                const float m = exp2f(c2t - cf[CF_C2 + s2]) * cf[CF_W + s2];
+                                *pv = __float2bfloat16_rn(__bfloat162float(*pv) * m);
                             }
                         }
                     }
@@ -974,12 +1035,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                 __syncwarp();
                 if (l32 == 0) mbar_arrive(bar(B_STTAKEN));
                 // ---- outputs y_t = sum_r W_y[r] (D2 + e^{cum_t} D3)_{(t,r)} + D x_t ----
-                if (et == 0) tma_store_wait_read();   // the previous output tile has been read out
                 if (!(ok = group_wait(B_YFULL, c & 1, 22))) break;
                 tc_fence_after();
                 const float ect = rowv ? cf[CF_EC + ttok] : 0.f;
                 const int rr = trow % R;
-#pragma unroll
+#pragma unroll 1
                 for (int c16 = 0; c16 < 2; c16++) {
                     const int p0 = cb0 + 16 * c16;
                     float y2[16], y3[16];
@@ -997,8 +1057,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                         }
                         y2[e] = v;
                     }
-                    if (rowv && rr == 0) {
+                    const int64_t tglob = t_beg + (int64_t)c * QT + ttok;
+                    if (rowv && rr == 0 && tglob < t_end) {
                         const int t = ttok;
+                        __nv_bfloat16 *yrow = yg + ((b * Tn + tglob) * H + h) * P;
 #pragma unroll
                         for (int hh = 0; hh < 2; hh++) {
                             const int cc = (p0 >> 3) + hh;   // 16-byte chunk (8 columns)
@@ -1011,23 +1073,19 @@ __global__ void __launch_bounds__(THREADS, 1)
                                 const int cidx = 8 * hh + 2 * e2;
                                 pk[e2] = pack_bf16(fmaf(Dh, xf.x, y2[cidx]), fmaf(Dh, xf.y, y2[cidx + 1]));
                             }
-                            *reinterpret_cast<uint4 *>(yt + t * 128 + ((cc ^ (t & 7)) << 4)) =
-                                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                            *reinterpret_cast<uint4 *>(yrow + 8 * cc) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                         }
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (l32 == 0) mbar_arrive(bar(B_YTAKEN));
-                fence_async_smem();
                 named_bar(2, EPI_THREADS);
                 if (et == 0) {
-                    tma_store4(&map_y, 0, (int)h, (int)(t_beg + (int64_t)c * QT), (int)b, sbase + L::OFF_YT);
                     mbar_arrive(bar(B_XEMPTY + sx));
                     mbar_arrive(bar(B_CEMPTY + scf));
                 }
             }
-            if (et == 0) tma_store_wait_all();
             // final state: h_{T-1} = g after the last chunk (no lookahead there)
             if (!*abort_flag && a.h_out && last_seg) {
                 float *ho = a.h_out + (lane_id * N + n) * P + cb0;
@@ -1047,7 +1105,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int n = et & (N - 1), half = et >> 7;
         const int c = nchunks - 1;
         const int Lc = (int)(t_end - t_beg - (int64_t)c * QT);
-        const uint8_t *xr = sm + L::OFF_X + (c % NX) * L::SZ_X;
+        const uint8_t *xr = sm + L::OFF_X + (c % L::NXR) * L::SZ_X;
         const int t = Lc - 1;
         float *uo = a.prevBx_out + (lane_id * N + n) * P;
         for (int cc = 4 * half; cc < 4 * half + 4; cc++) {
@@ -1193,7 +1251,7 @@ template <int R>
 static cudaError_t launch_tc_r(const ScanArgs &a, cudaStream_t s) {
     using namespace tc;
     constexpr int QT = Q / R;
-    CUtensorMap mx, mb, mc, mth, my;
+    CUtensorMap mx, mb, mc, mth;
     const int64_t rk = R > 1 ? R : 0;
     if (!make_map(&mx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P, a.H, a.T, a.Bt, P, QT, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&mb, a.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, a.H, a.T, a.Bt, N, QT, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -1201,10 +1259,11 @@ static cudaError_t launch_tc_r(const ScanArgs &a, cudaStream_t s) {
         !make_map(&mc, a.C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, a.H, a.T, a.Bt, N, QT, CU_TENSOR_MAP_SWIZZLE_NONE,
                   rk) ||
         !make_map(&mth, a.theta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, NP2, a.H, a.T, a.Bt, NP2, QT,
-                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&my, a.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P, a.H, a.T, a.Bt, P, QT, CU_TENSOR_MAP_SWIZZLE_128B))
+                  CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     TcArgs t;
+    t.y = a.y;
+    t.theta = a.theta;
     t.dt = a.dt; t.A = a.A; t.lam = a.lam; t.D = a.D;
     t.Wx = a.Wx; t.Wy = a.Wy;
     t.h0 = a.h0; t.prevBx0 = a.prevBx0; t.angle0 = a.angle0;
@@ -1223,7 +1282,7 @@ static cudaError_t launch_tc_r(const ScanArgs &a, cudaStream_t s) {
     constexpr int SMEM = smem_bytes<R>();
     if (pl.nseg > 1) {
         cudaFuncSetAttribute(k_scan_tc<true, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-        k_scan_tc<true, R><<<(unsigned)(lanes * (pl.nseg - 1)), THREADS, SMEM, s>>>(mx, mb, mc, mth, my, t);
+        k_scan_tc<true, R><<<(unsigned)(lanes * (pl.nseg - 1)), THREADS, SMEM, s>>>(mx, mb, mc, mth, t);
         count_launch();
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         k_seg_combine<<<dim3((unsigned)lanes, NP2 * P / 256), 256, 0, s>>>(t);
@@ -1231,7 +1290,7 @@ static cudaError_t launch_tc_r(const ScanArgs &a, cudaStream_t s) {
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     cudaFuncSetAttribute(k_scan_tc<false, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-    k_scan_tc<false, R><<<(unsigned)(lanes * pl.nseg), THREADS, SMEM, s>>>(mx, mb, mc, mth, my, t);
+    k_scan_tc<false, R><<<(unsigned)(lanes * pl.nseg), THREADS, SMEM, s>>>(mx, mb, mc, mth, t);
     count_launch();
     return cudaGetLastError();
 }
