@@ -64,6 +64,7 @@ constexpr int NWARPS = 19, THREADS = NWARPS * 32;
 constexpr int W_TMA = 0, W_MMA = 1, W_COEF = 2, W_PREP0 = 3, NPREP = 8, W_EPI0 = 11;
 constexpr int PREP_THREADS = NPREP * 32;          // 256
 constexpr int EPI_THREADS = 256;                  // two warps per TMEM lane quarter
+constexpr int EPI_WARPS = EPI_THREADS / 32;
 
 // ---- shared-memory map (bytes from a 1024-aligned base) ------------------
 // Rank R: a chunk holds QT = Q / R tokens and Q rows (token, rank) of B and C;
@@ -206,12 +207,37 @@ __device__ __forceinline__ bool wait_bar_spin(uint32_t bar, uint32_t parity, vol
                                               int site) {
     return mbar_try_spin(bar, parity) || wait_bar_slow(bar, parity, abort_flag, err, site, true);
 }
+// Bounded waits taken by every lane of a converged warp, with one warp-wide
+// outcome.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag, int *err,
+                                          int site);
+__device__ __forceinline__ bool warp_wait_spin(uint32_t bar, uint32_t parity, volatile int *abort_flag, int *err,
+                                               int site) {
+    const bool ok = wait_bar_spin(bar, parity, abort_flag, err, site);
+    return __all_sync(0xffffffffu, ok);
+}
 
 // Bounded wait on an mbarrier phase.  Returns false when the kernel is
 // aborting (this wait timed out, or another thread's did).
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag, int *err,
                                          int site) {
     return mbar_try(bar, parity) || wait_bar_slow(bar, parity, abort_flag, err, site, false);
+}
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag, int *err,
+                                          int site) {
+    const bool ok = wait_bar(bar, parity, abort_flag, err, site);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// One lane of a converged warp (elect.sync): the lane that issues a UMMA, a
+// commit or a TMA copy, while the whole warp computes the (warp-uniform)
+// operands.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile(
+        "{\n .reg .b32 rx;\n .reg .pred px;\n elect.sync rx|px, 0xffffffff;\n selp.b32 %0, 1, 0, px;\n}"
+        : "=r"(pred));
+    return pred != 0;
 }
 
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
@@ -373,15 +399,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(bar(B_BFULL + i), 1);
             mbar_init(bar(B_BEMPTY + i), 1);
         }
-        // x tiles are released by the Xw builder, the intra UMMA and the output
-        // writer (state-only pass: the Xw builder alone)
+        // x tiles are released by the Xw builder, the intra UMMA and each of the
+        // eight output-writing warps (state-only pass: the Xw builder alone);
+        // coefficients by the rotation group and each epilogue warp
         for (int i = 0; i < L::NXR; i++) {
             mbar_init(bar(B_XFULL + i), 1);
-            mbar_init(bar(B_XEMPTY + i), SO ? 1 : 3);
+            mbar_init(bar(B_XEMPTY + i), SO ? 1 : 2 + EPI_WARPS);
         }
         for (int i = 0; i < NC; i++) {
             mbar_init(bar(B_CFULL + i), 1);
-            mbar_init(bar(B_CEMPTY + i), 2);
+            mbar_init(bar(B_CEMPTY + i), 1 + EPI_WARPS);
         }
         for (int i = 0; i < 2; i++) {
             mbar_init(bar(B_OPSREADY + i), 1);
@@ -426,7 +453,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (warp == W_TMA) {
         // ------------------------------------------------------------ producer
-        if (l32 == 0) {
+        // converged warp, warp-uniform coordinates, one elected lane issues
+        {
             // B and C of a chunk: rows (token, rank) -- a 4-D box (N, H, T, Bt)
             // for SISO, a 5-D box (N, R, H, T, Bt) for MIMO
             auto load_bc = [&](uint32_t dst, const CUtensorMap *m, int t0, uint32_t fb) {
@@ -448,22 +476,31 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tma_prefetch4(&map_th, 0, (int)h, t0, (int)b);
                 tma_prefetch4(&map_x, 0, (int)h, t0, (int)b);
             };
-            for (int c = 1; c < PFD; c++) prefetch(c);
+            if (elect_one())
+                for (int c = 1; c < PFD; c++) prefetch(c);
+            __syncwarp();
             int issued = 0;
             for (int c = 0; c < nchunks; c++) {
                 const int sb = c % NB, kb = c / NB, sx = c % L::NXR, kx = c / L::NXR;
                 const int t0 = (int)(t_beg + (int64_t)c * QT);
-                prefetch(c + PFD);
-                if (kb > 0 && !wait_bar(bar(B_BEMPTY + sb), (kb - 1) & 1, abort_flag, a.err, 1)) break;
+                if (elect_one()) prefetch(c + PFD);
+                __syncwarp();
+                if (kb > 0 && !warp_wait(bar(B_BEMPTY + sb), (kb - 1) & 1, abort_flag, a.err, 1)) break;
                 const uint32_t st = sbase + L::OFF_BCT + sb * L::SZ_BCT;
                 const uint32_t fb = bar(B_BFULL + sb);
-                mbar_expect_tx(fb, SO ? SZ_BC : L::SZ_BCT);
-                load_bc(st, &map_b, t0, fb);
-                if (!SO) load_bc(st + SZ_BC, &map_c, t0, fb);
-                if (kx > 0 && !wait_bar(bar(B_XEMPTY + sx), (kx - 1) & 1, abort_flag, a.err, 2)) break;
+                if (elect_one()) {
+                    mbar_expect_tx(fb, SO ? SZ_BC : L::SZ_BCT);
+                    load_bc(st, &map_b, t0, fb);
+                    if (!SO) load_bc(st + SZ_BC, &map_c, t0, fb);
+                }
+                __syncwarp();
+                if (kx > 0 && !warp_wait(bar(B_XEMPTY + sx), (kx - 1) & 1, abort_flag, a.err, 2)) break;
                 const uint32_t xb = bar(B_XFULL + sx);
-                mbar_expect_tx(xb, L::SZ_X);
-                tma_load4(sbase + L::OFF_X + sx * L::SZ_X, &map_x, 0, (int)h, t0, (int)b, xb);
+                if (elect_one()) {
+                    mbar_expect_tx(xb, L::SZ_X);
+                    tma_load4(sbase + L::OFF_X + sx * L::SZ_X, &map_x, 0, (int)h, t0, (int)b, xb);
+                }
+                __syncwarp();
                 issued = c + 1;
             }
             // never leave loads in flight into shared memory at exit
@@ -780,7 +817,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else if (warp == W_MMA) {
         // ------------------------------------------------------------ MMA issue
-        if (l32 == 0) {
+        // The whole warp walks the chunks converged, so the descriptors are
+        // warp-uniform; one elected lane issues each UMMA and commit.
+        {
             const uint32_t id_kk = idesc(64, 64, 0, 0);    // D1 = Cbar . Bsc^T
             const uint32_t id_kmn = idesc(64, 64, 0, 1);   // D2, D3: B operand MN-major
             const uint32_t id_st = idesc(128, 64, 1, 1);   // D4: A and B MN-major
@@ -808,48 +847,65 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint64_t d_bsc_mn = d_bsc_mn0 + ob * STEP_BC, d_xw = d_xw0 + ob * STEP_XP;
                 const uint64_t dx = (R == 1) ? d_x0 + (uint64_t)sx * STEP_X : d_xr0 + ob * STEP_XP;
                 const uint64_t dg = d_gb0 + ((c + 1) & 1) * STEP_GB;   // state after chunk c-1
-                if (!wait_bar_spin(bar(B_OPSREADY + ob), (c >> 1) & 1, abort_flag, a.err, 10)) break;
+                if (!warp_wait_spin(bar(B_OPSREADY + ob), (c >> 1) & 1, abort_flag, a.err, 10)) break;
                 if (SO) {
                     // state-only pass: the chunk-state UMMA alone
-                    if (!wait_bar_spin(bar(B_STTAKEN), c & 1, abort_flag, a.err, 12)) break;
+                    if (!warp_wait_spin(bar(B_STTAKEN), c & 1, abort_flag, a.err, 12)) break;
                     tc_fence_after();
+                    if (elect_one()) {
+                        for (int kk = 0; kk < Q / 16; kk++)
+                            umma(tmem + COL_D4, d_bsc_mn + kstep_mn(kk), d_xw + kstep_mn(kk), id_st, kk > 0);
+                        umma_commit(bar(B_STFULL));
+                        umma_commit(bar(B_OPSFREE + ob));
+                    }
+                    __syncwarp();
+                    continue;
+                }
+                if (c > 0 && !warp_wait_spin(bar(B_STAKEN), (c - 1) & 1, abort_flag, a.err, 11)) break;
+                tc_fence_after();
+                if (elect_one()) {
+#pragma unroll 1
+                    for (int kk = 0; kk < N / 16; kk++)
+                        umma(tmem + COL_D1, d_cb_k + kstep_k(kk), d_bsc_k + kstep_k(kk), id_kk, kk > 0);
+                    umma_commit(bar(B_SFULL));
+                }
+                __syncwarp();
+                if (!warp_wait_spin(bar(B_STTAKEN), c & 1, abort_flag, a.err, 12)) break;
+                tc_fence_after();
+                if (elect_one()) {
+#pragma unroll 1
                     for (int kk = 0; kk < Q / 16; kk++)
                         umma(tmem + COL_D4, d_bsc_mn + kstep_mn(kk), d_xw + kstep_mn(kk), id_st, kk > 0);
                     umma_commit(bar(B_STFULL));
-                    umma_commit(bar(B_OPSFREE + ob));
-                    continue;
                 }
-                if (c > 0 && !wait_bar_spin(bar(B_STAKEN), (c - 1) & 1, abort_flag, a.err, 11)) break;
+                __syncwarp();
+                if (c > 0 && !warp_wait_spin(bar(B_YTAKEN), (c - 1) & 1, abort_flag, a.err, 13)) break;
                 tc_fence_after();
+                if (elect_one()) {
 #pragma unroll 1
-                for (int kk = 0; kk < N / 16; kk++)
-                    umma(tmem + COL_D1, d_cb_k + kstep_k(kk), d_bsc_k + kstep_k(kk), id_kk, kk > 0);
-                umma_commit(bar(B_SFULL));
-                if (!wait_bar_spin(bar(B_STTAKEN), c & 1, abort_flag, a.err, 12)) break;
+                    for (int kk = 0; kk < N / 16; kk++)
+                        umma(tmem + COL_D3, d_cb_k + kstep_k(kk), dg + kstep_mn(kk), id_kmn, kk > 0);
+                }
+                __syncwarp();
+                if (!warp_wait_spin(bar(B_SPFULL), c & 1, abort_flag, a.err, 14)) break;
                 tc_fence_after();
+                if (elect_one()) {
 #pragma unroll 1
-                for (int kk = 0; kk < Q / 16; kk++)
-                    umma(tmem + COL_D4, d_bsc_mn + kstep_mn(kk), d_xw + kstep_mn(kk), id_st, kk > 0);
-                umma_commit(bar(B_STFULL));
-                if (c > 0 && !wait_bar_spin(bar(B_YTAKEN), (c - 1) & 1, abort_flag, a.err, 13)) break;
-                tc_fence_after();
-#pragma unroll 1
-                for (int kk = 0; kk < N / 16; kk++)
-                    umma(tmem + COL_D3, d_cb_k + kstep_k(kk), dg + kstep_mn(kk), id_kmn, kk > 0);
-                if (!wait_bar_spin(bar(B_SPFULL), c & 1, abort_flag, a.err, 14)) break;
-                tc_fence_after();
-#pragma unroll 1
-                for (int kk = 0; kk < Q / 16; kk++)
-                    umma(tmem + COL_D2, d_sp + (uint64_t)((kk * 32) >> 4), dx + kstep_mn(kk), id_kmn, kk > 0);
-                umma_commit(bar(B_YFULL));
-                umma_commit(bar(B_OPSFREE + ob));      // every operand of chunk c has been read
-                umma_commit(bar(B_XEMPTY + sx));
+                    for (int kk = 0; kk < Q / 16; kk++)
+                        umma(tmem + COL_D2, d_sp + (uint64_t)((kk * 32) >> 4), dx + kstep_mn(kk), id_kmn, kk > 0);
+                    umma_commit(bar(B_YFULL));
+                    umma_commit(bar(B_OPSFREE + ob));  // every operand of chunk c has been read
+                    umma_commit(bar(B_XEMPTY + sx));
+                }
+                __syncwarp();
             }
             // drain: every MMA issued so far has completed before TMEM is freed
-            umma_commit(bar(B_DRAIN));
+            if (elect_one()) umma_commit(bar(B_DRAIN));
+            __syncwarp();
             const long long t0 = clock64();
             while (!mbar_try(bar(B_DRAIN), 0) && clock64() - t0 < WAIT_LIMIT_CYCLES) {
             }
+            __syncwarp();
         }
     } else {
         // ------------------------------------------------------------- epilogue
@@ -867,11 +923,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         const float Dh = a.D[h];
         uint8_t *sp = sm + L::OFF_SP;
         __nv_bfloat16 *yg = static_cast<__nv_bfloat16 *>(a.y);
-        // one thread waits, the group meets at a named barrier and leaves together
+        // each warp waits on its own (no group barrier): a warp that gives up
+        // leaves its loop, and the others give up at their next wait
         auto group_wait = [&](int bi, uint32_t parity, int site) -> bool {
-            bool fail = false;
-            if (et == 0) fail = !wait_bar(bar(bi), parity, abort_flag, a.err, site);
-            return !named_bar_or(2, EPI_THREADS, fail);
+            return warp_wait(bar(bi), parity, abort_flag, a.err, site);
         };
         auto store_g = [&](const float *gv, int slot) {
             uint8_t *gb = sm + L::OFF_GB + slot * SZ_GB;
@@ -916,9 +971,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                 fold_state(cf, g);
                 tc_fence_before();
                 __syncwarp();
-                if (l32 == 0) mbar_arrive(bar(B_STTAKEN));
-                named_bar(2, EPI_THREADS);
-                if (et == 0) mbar_arrive(bar(B_CEMPTY + scf));
+                if (l32 == 0) {
+                    mbar_arrive(bar(B_STTAKEN));
+                    mbar_arrive(bar(B_CEMPTY + scf));
+                }
             }
             if (!*abort_flag) {
                 float *go = slot_out + SLOT_G + n * P + cb0;
@@ -1079,9 +1135,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (l32 == 0) mbar_arrive(bar(B_YTAKEN));
-                named_bar(2, EPI_THREADS);
-                if (et == 0) {
+                if (l32 == 0) {
+                    mbar_arrive(bar(B_YTAKEN));
                     mbar_arrive(bar(B_XEMPTY + sx));
                     mbar_arrive(bar(B_CEMPTY + scf));
                 }
