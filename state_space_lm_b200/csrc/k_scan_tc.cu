@@ -329,6 +329,31 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v) {
 #pragma unroll
     for (int i = 0; i < 16; i++) v[i] = __uint_as_float(r[i]);
 }
+// 32 fp32 columns of 16 TMEM lanes (the rows of an M=64 accumulator in this
+// warp's lane quarter), spread over the 32 threads: thread t gets, for each
+// group i of 8 columns, v[4i], v[4i+1] = (lane t/4, columns 8i + 2(t%4) + 0, 1)
+// and v[4i+2], v[4i+3] = (lane t/4 + 8, the same columns).
+__device__ __forceinline__ void tmem_ld16x256b_x4(uint32_t taddr, float *v) {
+    uint32_t r[16];
+    __syncwarp();
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 16; i++) v[i] = __uint_as_float(r[i]);
+}
+// The same for 16 columns (two groups of 8).
+__device__ __forceinline__ void tmem_ld16x256b_x2(uint32_t taddr, float *v) {
+    uint32_t r[8];
+    __syncwarp();
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 8; i++) v[i] = __uint_as_float(r[i]);
+}
 __device__ __forceinline__ void tmem_wait_ld() {
     __syncwarp();
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
@@ -690,7 +715,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const bool last_chunk = last_seg && (c == nchunks - 1);
             auto rotate_tokens = [&](auto generic) {
                 constexpr bool G = decltype(generic)::value;
-#pragma unroll 1
+#pragma unroll
                 for (int u = 0; u < TPT; u++) {
                     const int i = i0 + u;
                     float d[4] = {dph[0][0], dph[0][1], dph[0][2], dph[0][3]};
@@ -916,9 +941,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int cb0 = 32 * ch;
         const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
         const int n = 32 * q + l32;                  // state row owned by this thread
-        const int trow = 16 * q + l32;               // score/output row (valid for l32 < 16)
-        const int ttok = trow / R;                   // its token
-        const bool rowv = l32 < 16;
+        // score / output rows (M=64 accumulators, 16 lanes per quarter): this
+        // thread holds rows ra and rb = ra + 8, two adjacent columns per group
+        // of 8 (the 16x256b load layout)
+        const int ra = 16 * q + (l32 >> 2), rb = ra + 8;
+        const int ta = ra / R, tb = rb / R;          // their tokens
+        const int cq = 2 * (l32 & 3);                // column offset inside a group of 8
         const int et = tid - W_EPI0 * 32;            // 0..255
         const float Dh = a.D[h];
         uint8_t *sp = sm + L::OFF_SP;
@@ -1020,56 +1048,44 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint8_t *xr = sm + L::OFF_X + sx * L::SZ_X;
                 if (!(ok = group_wait(B_CFULL + scf, kc & 1, 20))) break;
                 const bool unsafe = cf[CF_SCAL + 1] != 0.f;
-                // ---- masked scores S' (rows of D1, my 32 columns) ----
+                // ---- masked scores S' (rows ra, rb of D1; my 32 columns) ----
                 if (!(ok = group_wait(B_SFULL, c & 1, 21))) break;
                 tc_fence_after();
                 {
-                    const int t = ttok;
-                    const float rt = rowv ? cf[CF_R + t] : 0.f;
-                    const float gt = rowv ? cf[CF_GAM + t] : 0.f;
+                    const float rta = cf[CF_R + ta], gta = cf[CF_GAM + ta];
+                    const float rtb = cf[CF_R + tb], gtb = cf[CF_GAM + tb];
 #pragma unroll 1
-                    for (int c16 = 0; c16 < 2; c16++) {
-                        const int s0 = cb0 + 16 * c16;
-                        float v[16];
-                        tmem_ld16(tl + COL_D1 + s0, v);
+                    for (int hf = 0; hf < 2; hf++) {
+                        const int c0 = cb0 + 16 * hf;
+                        float v[8];
+                        tmem_ld16x256b_x2(tl + COL_D1 + c0, v);
                         tmem_wait_ld();
-                        if (rowv) {
-                            // column factors of the 16/R tokens of these columns
-                            float wm[16 / R];
 #pragma unroll
-                            for (int k4 = 0; k4 < 16 / R; k4 += 4) {
-                                const float4 w4 = *reinterpret_cast<const float4 *>(cf + CF_WM + s0 / R + k4);
-                                wm[k4] = w4.x; wm[k4 + 1] = w4.y; wm[k4 + 2] = w4.z; wm[k4 + 3] = w4.w;
-                            }
-#pragma unroll
-                            for (int k2 = 0; k2 < 16 / R; k2++) {
-                                const int s2 = s0 / R + k2;  // token of columns k2*R .. k2*R+R-1
-                                const float m = s2 < t ? rt * wm[k2] : (s2 == t ? rt * gt : 0.f);
-#pragma unroll
-                                for (int r2 = 0; r2 < R; r2++) v[k2 * R + r2] *= m;
-                            }
-#pragma unroll
-                            for (int hh = 0; hh < 2; hh++) {
-                                const int cc = (s0 >> 3) + hh;
-                                uint4 pk;
-                                pk.x = pack_bf16(v[8 * hh], v[8 * hh + 1]);
-                                pk.y = pack_bf16(v[8 * hh + 2], v[8 * hh + 3]);
-                                pk.z = pack_bf16(v[8 * hh + 4], v[8 * hh + 5]);
-                                pk.w = pack_bf16(v[8 * hh + 6], v[8 * hh + 7]);
-                                *reinterpret_cast<uint4 *>(sp + trow * 128 + ((cc ^ (trow & 7)) << 4)) = pk;
-                            }
+                        for (int i = 0; i < 2; i++) {
+                            const int col = c0 + 8 * i + cq;
+                            const int s0 = col / R, s1 = (col + 1) / R;   // tokens of the two columns
+                            const float w0 = cf[CF_WM + s0], w1 = cf[CF_WM + s1];
+                            v[4 * i + 0] *= s0 < ta ? rta * w0 : (s0 == ta ? rta * gta : 0.f);
+                            v[4 * i + 1] *= s1 < ta ? rta * w1 : (s1 == ta ? rta * gta : 0.f);
+                            v[4 * i + 2] *= s0 < tb ? rtb * w0 : (s0 == tb ? rtb * gtb : 0.f);
+                            v[4 * i + 3] *= s1 < tb ? rtb * w1 : (s1 == tb ? rtb * gtb : 0.f);
+                            const int cc = col >> 3;
+                            *reinterpret_cast<uint32_t *>(sp + ra * 128 + ((cc ^ (ra & 7)) << 4) + 2 * cq) =
+                                pack_bf16(v[4 * i], v[4 * i + 1]);
+                            *reinterpret_cast<uint32_t *>(sp + rb * 128 + ((cc ^ (rb & 7)) << 4) + 2 * cq) =
+                                pack_bf16(v[4 * i + 2], v[4 * i + 3]);
                         }
                     }
-                    if (unsafe && rowv) {
+                    if (unsafe) {
                         // exact path: the scores below the diagonal were stored
                         // unscaled; give each its factor e^{cum_t - cum_s} w_s here
-                        const float c2t = cf[CF_C2 + t];
 #pragma unroll 1
-                        for (int col = cb0; col < cb0 + 32; col++) {
-                            const int s2 = col / R;
+                        for (int k = 0; k < 16; k++) {
+                            const int row = (k & 2) ? rb : ra, t = row / R;
+                            const int col = cb0 + 8 * (k >> 2) + cq + (k & 1), s2 = col / R;
                             if (s2 < t) {
-                                __nv_bfloat16 *pv = reinterpret_cast<__nv_bfloat16 *>(sp + sw128(trow, col));
-                                const float m = exp2f(c2t - cf[CF_C2 + s2]) * cf[CF_W + s2];
+                                __nv_bfloat16 *pv = reinterpret_cast<__nv_bfloat16 *>(sp + sw128(row, col));
+                                const float m = exp2f(cf[CF_C2 + t] - cf[CF_C2 + s2]) * cf[CF_W + s2];
                                 *pv = __float2bfloat16_rn(__bfloat162float(*pv) * m);
                             }
                         }
@@ -1093,43 +1109,45 @@ __global__ void __launch_bounds__(THREADS, 1)
                 // ---- outputs y_t = sum_r W_y[r] (D2 + e^{cum_t} D3)_{(t,r)} + D x_t ----
                 if (!(ok = group_wait(B_YFULL, c & 1, 22))) break;
                 tc_fence_after();
-                const float ect = rowv ? cf[CF_EC + ttok] : 0.f;
-                const int rr = trow % R;
+                {
+                    const float eca = cf[CF_EC + ta], ecb = cf[CF_EC + tb];
+                    const int64_t tc0 = t_beg + (int64_t)c * QT;
 #pragma unroll 1
-                for (int c16 = 0; c16 < 2; c16++) {
-                    const int p0 = cb0 + 16 * c16;
-                    float y2[16], y3[16];
-                    tmem_ld16(tl + COL_D2 + p0, y2);
-                    tmem_ld16(tl + COL_D3 + p0, y3);
-                    tmem_wait_ld();
+                    for (int hf = 0; hf < 2; hf++) {
+                        const int c0 = cb0 + 16 * hf;        // 16 columns: two groups of 8
+                        float y2[8], y3[8];
+                        tmem_ld16x256b_x2(tl + COL_D2 + c0, y2);
+                        tmem_ld16x256b_x2(tl + COL_D3 + c0, y3);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; e++) {
-                        float v = fmaf(ect, y3[e], y2[e]);
-                        if (R > 1) {
-                            // contract the R rows of a token (adjacent lanes) with W_y
-                            v *= wys[rr * P + p0 + e];
+                        for (int i = 0; i < 2; i++) {
 #pragma unroll
-                            for (int o = 1; o < R; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                        }
-                        y2[e] = v;
-                    }
-                    const int64_t tglob = t_beg + (int64_t)c * QT + ttok;
-                    if (rowv && rr == 0 && tglob < t_end) {
-                        const int t = ttok;
-                        __nv_bfloat16 *yrow = yg + ((b * Tn + tglob) * H + h) * P;
+                            for (int j = 0; j < 4; j++) {
+                                float v = fmaf((j & 2) ? ecb : eca, y3[4 * i + j], y2[4 * i + j]);
+                                if (R > 1) {
+                                    // contract the R rows of a token (threads l32 ^ 4, ^ 8) with W_y
+                                    const int row = (j & 2) ? rb : ra;
+                                    v *= wys[(row % R) * P + c0 + 8 * i + cq + (j & 1)];
 #pragma unroll
-                        for (int hh = 0; hh < 2; hh++) {
-                            const int cc = (p0 >> 3) + hh;   // 16-byte chunk (8 columns)
-                            const uint4 xv = *reinterpret_cast<const uint4 *>(xr + t * 128 + ((cc ^ (t & 7)) << 4));
-                            const uint32_t xw4[4] = {xv.x, xv.y, xv.z, xv.w};
-                            uint32_t pk[4];
-#pragma unroll
-                            for (int e2 = 0; e2 < 4; e2++) {
-                                const float2 xf = unpack_bf16(xw4[e2]);
-                                const int cidx = 8 * hh + 2 * e2;
-                                pk[e2] = pack_bf16(fmaf(Dh, xf.x, y2[cidx]), fmaf(Dh, xf.y, y2[cidx + 1]));
+                                    for (int o = 4; o < 4 * R; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                                }
+                                y2[4 * i + j] = v;
                             }
-                            *reinterpret_cast<uint4 *>(yrow + 8 * cc) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        }
+#pragma unroll
+                        for (int hb = 0; hb < 2; hb++) {
+                            const int row = hb ? rb : ra, t = row / R;
+                            if (row % R == 0 && tc0 + t < t_end) {
+                                __nv_bfloat16 *yrow = yg + ((b * Tn + tc0 + t) * H + h) * P;
+#pragma unroll
+                                for (int i = 0; i < 2; i++) {
+                                    const int col = c0 + 8 * i + cq, cc = col >> 3;
+                                    const float2 xf = unpack_bf16(*reinterpret_cast<const uint32_t *>(
+                                        xr + t * 128 + ((cc ^ (t & 7)) << 4) + 2 * cq));
+                                    *reinterpret_cast<uint32_t *>(yrow + col) = pack_bf16(
+                                        fmaf(Dh, xf.x, y2[4 * i + 2 * hb]), fmaf(Dh, xf.y, y2[4 * i + 2 * hb + 1]));
+                                }
+                            }
                         }
                     }
                 }

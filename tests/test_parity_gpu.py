@@ -179,11 +179,25 @@ def test_siso_empty_sequence_passes_state_through():
     assert torch.equal(hf.cpu(), h0) and torch.equal(uf.cpu(), u0) and torch.equal(af.cpu(), a0)
 
 
-def test_siso_deterministic():
-    inp = gen.scan_inputs(2, 200, 4, 64, 128, dtype=BF16, seed=7)
+@pytest.mark.parametrize("case", ["siso", "mimo_r4", "siso_segmented"])
+def test_tc_scan_deterministic(case):
+    """The scans use no atomics on the data path: two calls on the same
+    inputs agree bit for bit (a race between warps or CTAs would show here)."""
+    if case == "mimo_r4":
+        inp = gen.scan_inputs(2, 200, 4, 64, 128, rank=4, dtype=BF16, seed=8)
+    elif case == "siso_segmented":
+        inp = gen.scan_inputs(1, 3000, 2, 64, 128, dtype=BF16, seed=9, dt_shift=-4.0)
+    else:
+        inp = gen.scan_inputs(2, 200, 4, 64, 128, dtype=BF16, seed=7)
     d = cuda(inp)
-    a = m3.siso_chunked_fwd(d["x"], d["dt"], d["A"], d["lam"], d["theta"], d["B"], d["C"], d["D"], 64)
-    b = m3.siso_chunked_fwd(d["x"], d["dt"], d["A"], d["lam"], d["theta"], d["B"], d["C"], d["D"], 64)
+
+    def run():
+        if case == "mimo_r4":
+            return m3.mimo_chunked_fwd(d["x"], d["dt"], d["A"], d["lam"], d["theta"], d["B"], d["C"], d["D"], 64,
+                                       W_x=d["Wx"], W_y=d["Wy"])
+        return m3.siso_chunked_fwd(d["x"], d["dt"], d["A"], d["lam"], d["theta"], d["B"], d["C"], d["D"], 64)
+
+    a, b = run(), run()
     for u, v in zip(a, b):
         assert torch.equal(u, v)
 
