@@ -24,28 +24,29 @@
 // One CTA owns one (b, h) lane -- or one segment of it, see below -- and
 // walks its chunks in order.  Per chunk four UMMAs (tcgen05.mma kind::f16,
 // bf16 operands in shared memory, fp32 accumulators in tensor memory):
-//   D1 = Cbar . Bsc^T             scores            M=64  N=64  K=128
+//   D1 = Cbar . Bbar^T            scores            M=64  N=64  K=128
 //   D3 = Cbar . g_in              inter-chunk term  M=64  N=64  K=128
 //   D2 = S' . X                   intra-chunk term  M=64  N=64  K=64
-//   D4 = Bsc^T . Xw               chunk state       M=128 N=64  K=64
-// The decay mask is split into a row factor and a column factor: Bsc holds
-// e_s Bbar_s with e_s = e^{cum_end - cum_s}, the masking multiplies row t by
-// r_t = e^{cum_t - cum_end} and column s by w_s (gamma_t on the diagonal), and
-// Xw holds w_s x_s, so D4 is the chunk's state contribution directly.  When a
-// chunk's log-decay range exceeds 60 the factors could leave the fp32 range;
-// such a chunk uses Bsc = Bbar, an exact per-element mask
-// e^{cum_t - cum_s} w_s and Xw = e^{cum_end - cum_s} w_s x_s instead.
+//   D4 = Bbar^T . Xw              chunk state       M=128 N=64  K=64
+// With e_s = e^{cum_end - cum_s}, Xw holds e_s w_s x_s, so D4 is the chunk's
+// state contribution directly, and the decay mask is split into a row factor
+// r_t = e^{cum_t - cum_end} and a column factor e_s w_s (gamma_t on the
+// diagonal, zero above it), applied to D1 in the epilogue.  When a chunk's
+// log-decay range exceeds 60 the two factors could leave the fp32 range; such
+// a chunk's scores instead get the exact factor e^{cum_t - cum_s} w_s one by
+// one.
 //
 // Long sequences over few lanes are cut into segments of whole chunks: a
 // state-only pass computes every segment's end state from a zero start in
 // its own angle frame, a small combine kernel chains the segments, and the
 // full pass then runs all segments in parallel from their entering states.
 //
-// Warp roles (19 warps): 0 TMA producer, 1 MMA issuer (and TMEM owner),
+// Warp roles (20 warps): 0 TMA producer, 1 MMA issuer (and TMEM owner),
 // 2 per-token coefficients, 3-10 rotation (QkNorm, bias, RoPE; each thread 4
-// pairs x 4 tokens with 16-byte shared-memory accesses) and the Xw scaling,
-// 11-18 epilogue (two warps per TMEM lane quarter, each owning 32 of the 64
-// columns: masked scores, fp32 state in registers, outputs).  Inputs stream
+// pairs x 4 tokens with 16-byte shared-memory accesses), 11-18 epilogue (two
+// warps per TMEM lane quarter, each owning 32 of the 64 columns: masked
+// scores, fp32 state in registers, outputs), 19 the X operands (Xw, and the
+// rank-expanded X_r for MIMO).  Inputs stream
 // through two rings: B, C, theta (released once rotated) and x (released
 // once the outputs are written).  Every wait is bounded: past ~1 s the kernel
 // records an error, stops issuing work, drains what it has in flight and
@@ -60,8 +61,8 @@ namespace tc {
 template <bool V> struct BoolC { static constexpr bool value = V; };
 
 constexpr int Q = 64, P = 64, N = 128, NP2 = 64;
-constexpr int NWARPS = 19, THREADS = NWARPS * 32;
-constexpr int W_TMA = 0, W_MMA = 1, W_COEF = 2, W_PREP0 = 3, NPREP = 8, W_EPI0 = 11;
+constexpr int NWARPS = 20, THREADS = NWARPS * 32;
+constexpr int W_TMA = 0, W_MMA = 1, W_COEF = 2, W_PREP0 = 3, NPREP = 8, W_EPI0 = 11, W_XB = 19;
 constexpr int PREP_THREADS = NPREP * 32;          // 256
 constexpr int EPI_THREADS = 256;                  // two warps per TMEM lane quarter
 constexpr int EPI_WARPS = EPI_THREADS / 32;
@@ -75,8 +76,8 @@ constexpr int NB = 2, NX = 3, NC = 4;             // ring depths: B/C, x, coeffi
 constexpr int SZ_BC = Q * N * 2;                  // 16 KB, bf16, row-major (TMA)
 constexpr int SZ_SP = Q * Q * 2, SZ_GB = N * P * 2;
 // per-chunk coefficient buffer (a ring of NC), floats; per token of the chunk
-constexpr int CF_W = 0, CF_GAM = Q, CF_E = 2 * Q, CF_R = 3 * Q, CF_EC = 4 * Q, CF_XS = 5 * Q,
-              CF_C2 = 6 * Q, CF_DT = 7 * Q, CF_WM = 8 * Q, CF_SCAL = 9 * Q, CF_FLOATS = 9 * Q + 8;
+constexpr int CF_W = 0, CF_GAM = Q, CF_R = 2 * Q, CF_EC = 3 * Q, CF_XS = 4 * Q, CF_C2 = 5 * Q, CF_DT = 6 * Q,
+              CF_WM = 7 * Q, CF_SCAL = 8 * Q, CF_FLOATS = 8 * Q + 8;
 template <int R>
 struct Lay {
     static constexpr int QT = Q / R;
@@ -85,8 +86,8 @@ struct Lay {
     static constexpr int SZ_BCT = 2 * SZ_BC;                  // one B/C stage
     static constexpr int OFF_BCT = 0;                         // NB x [B | C]
     static constexpr int OFF_X = OFF_BCT + NB * SZ_BCT;       // NX x [QT][P]
-    static constexpr int OFF_BSC = ((OFF_X + NXR * SZ_X + 1023) / 1024) * 1024;   // 2 x [2 atoms][Q rows][64]
-    static constexpr int OFF_CB = OFF_BSC + 2 * Q * N * 2;    // 2 x [2 atoms][Q rows][64] bf16, SW128
+    static constexpr int OFF_BB = ((OFF_X + NXR * SZ_X + 1023) / 1024) * 1024;   // 2 x [2 atoms][Q rows][64]
+    static constexpr int OFF_CB = OFF_BB + 2 * Q * N * 2;    // 2 x [2 atoms][Q rows][64] bf16, SW128
     static constexpr int OFF_SP = OFF_CB + 2 * Q * N * 2;     // [Q][Q] bf16, SW128
     static constexpr int OFF_XW = OFF_SP + SZ_SP;             // 2 x [Q rows][P] bf16, SW128
     static constexpr int OFF_XR = OFF_XW + 2 * Q * P * 2;     // 2 x [Q rows][P] bf16, SW128 (R > 1)
@@ -424,19 +425,21 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(bar(B_BFULL + i), 1);
             mbar_init(bar(B_BEMPTY + i), 1);
         }
-        // x tiles are released by the Xw builder, the intra UMMA and each of the
-        // eight output-writing warps (state-only pass: the Xw builder alone);
-        // coefficients by the rotation group and each epilogue warp
+        // x tiles are released by the X-operand warp, the intra UMMA and each
+        // of the eight output-writing warps (state-only pass: the X-operand
+        // warp alone); coefficients by the rotation group, the X-operand warp
+        // and each epilogue warp; a chunk's operands are ready once both the
+        // rotation group and the X-operand warp have written theirs
         for (int i = 0; i < L::NXR; i++) {
             mbar_init(bar(B_XFULL + i), 1);
             mbar_init(bar(B_XEMPTY + i), SO ? 1 : 2 + EPI_WARPS);
         }
         for (int i = 0; i < NC; i++) {
             mbar_init(bar(B_CFULL + i), 1);
-            mbar_init(bar(B_CEMPTY + i), 1 + EPI_WARPS);
+            mbar_init(bar(B_CEMPTY + i), 2 + EPI_WARPS);
         }
         for (int i = 0; i < 2; i++) {
-            mbar_init(bar(B_OPSREADY + i), 1);
+            mbar_init(bar(B_OPSREADY + i), 2);
             mbar_init(bar(B_OPSFREE + i), 1);
         }
         mbar_init(bar(B_SFULL), 1);
@@ -599,17 +602,18 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int u = 0; u < 2; u++) {
                 const int i = l32 + 32 * u;
                 if (i < QT) {
-                    const float e = exp2f(cend - la[u]);
-                    // mask factors: row r_t and column w_s, or ones when the chunk
-                    // takes the exact path (the scores then get e^{cum_t-cum_s} w_s
-                    // one by one)
+                    // e_s = e^{cum_end - cum_s} goes into the X operand of the
+                    // chunk-state UMMA (Xw = e_s w_s x_s) and into the mask's
+                    // column factor; the mask is r_t * (e_s w_s), or ones when the
+                    // chunk takes the exact path (the scores then get
+                    // e^{cum_t - cum_s} w_s one by one)
+                    const float ew = exp2f(cend - la[u]) * wv[u];
                     cf[CF_W + i] = wv[u];
-                    cf[CF_WM + i] = unsafe ? 1.f : wv[u];
+                    cf[CF_WM + i] = unsafe ? 1.f : ew;
                     cf[CF_GAM + i] = gv[u];
-                    cf[CF_E + i] = unsafe ? 1.f : e;
                     cf[CF_R + i] = unsafe ? 1.f : exp2f(la[u] - cend);
                     cf[CF_EC + i] = exp2f(la[u]);
-                    cf[CF_XS + i] = unsafe ? e * wv[u] : wv[u];
+                    cf[CF_XS + i] = ew;
                     cf[CF_C2 + i] = la[u];
                     cf[CF_DT + i] = dl[u];
                 }
@@ -649,17 +653,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         };
         load_theta(0);
         for (int c = 0; c < nchunks; c++) {
-            const int sb = c % NB, kb = c / NB, sx = c % L::NXR, kx = c / L::NXR, scf = c % NC, kc = c / NC;
+            const int sb = c % NB, kb = c / NB, scf = c % NC, kc = c / NC;
             const int ob = c & 1;                  // operand buffer
             bool fail = false;
             if (pt == 0) {
                 fail = !(wait_bar(bar(B_BFULL + sb), kb & 1, abort_flag, a.err, 4) &&
-                         wait_bar(bar(B_XFULL + sx), kx & 1, abort_flag, a.err, 5) &&
                          wait_bar(bar(B_CFULL + scf), kc & 1, abort_flag, a.err, 6) &&
                          (c < 2 || wait_bar(bar(B_OPSFREE + ob), ((c >> 1) - 1) & 1, abort_flag, a.err, 7)));
             }
             if (named_bar_or(1, PREP_THREADS, fail)) break;
-            uint8_t *bsc = sm + L::OFF_BSC + ob * (Q * N * 2);
+            uint8_t *bbar = sm + L::OFF_BB + ob * (Q * N * 2);
             uint8_t *cb = sm + L::OFF_CB + ob * (Q * N * 2);
             const float *cf = coef0 + scf * CF_FLOATS;
             const uint8_t *stg = sm + L::OFF_BCT + sb * L::SZ_BCT;
@@ -730,7 +733,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                         phi[q] += d[q];
                         sincos_rr(phi[q], &sn[q], &cs[q]);
                     }
-                    const float e = cf[CF_E + i];
 #pragma unroll 1
                     for (int r = 0; r < R; r++) {
                         const int row = i * R + r;
@@ -757,7 +759,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                                     if (nr.biasC) { cv.x += nr.biasC[bo]; cv.y += nr.biasC[bo + 1]; }
                                 }
                                 const float rb0 = cs[q] * bv.x - sn[q] * bv.y, rb1 = sn[q] * bv.x + cs[q] * bv.y;
-                                pbw[q] = pack_bf16(rb0 * e, rb1 * e);
+                                pbw[q] = pack_bf16(rb0, rb1);
                                 if (!SO) pcw[q] = pack_bf16(cs[q] * cv.x - sn[q] * cv.y, sn[q] * cv.x + cs[q] * cv.y);
                                 else pcw[q] = 0u;
                                 if (last_chunk && i == Lc - 1) {
@@ -769,7 +771,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                             oc = make_uint4(pcw[0], pcw[1], pcw[2], pcw[3]);
                         }
                         const uint32_t off = atom + (uint32_t)(row * 128 + ((chk ^ (row & 7)) << 4));
-                        *reinterpret_cast<uint4 *>(bsc + off) = ob;
+                        *reinterpret_cast<uint4 *>(bbar + off) = ob;
                         if (!SO) *reinterpret_cast<uint4 *>(cb + off) = oc;
                     }
                 }
@@ -777,6 +779,33 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (has_norm || has_bias) rotate_tokens(BoolC<true>{});
             else rotate_tokens(BoolC<false>{});
             load_theta(c + 1);                     // in flight while the X operands are built
+            fence_async_smem();
+            named_bar(1, PREP_THREADS);
+            if (tg == 15) {
+                // the last token group ends at the chunk's last token
+                *reinterpret_cast<float4 *>(phic + 4 * j4) = make_float4(phi[0], phi[1], phi[2], phi[3]);
+                if (last_chunk && a.angle_out)
+                    *reinterpret_cast<float4 *>(a.angle_out + lane_id * NP2 + 4 * j4) =
+                        make_float4(phi[0], phi[1], phi[2], phi[3]);
+                if (SO && c == nchunks - 1)
+                    *reinterpret_cast<float4 *>(slot_out + SLOT_PHIL + 4 * j4) =
+                        make_float4(phi[0], phi[1], phi[2], phi[3]);
+            }
+            if (pt == 0) {
+                mbar_arrive(bar(B_OPSREADY + ob));
+                mbar_arrive(bar(B_BEMPTY + sb));
+                mbar_arrive(bar(B_CEMPTY + scf));
+            }
+        }
+    } else if (warp == W_XB) {
+        // ------------------------------------------------------ X operands
+        for (int c = 0; c < nchunks; c++) {
+            const int sx = c % L::NXR, kx = c / L::NXR, scf = c % NC, kc = c / NC, ob = c & 1;
+            if (!(warp_wait(bar(B_XFULL + sx), kx & 1, abort_flag, a.err, 8) &&
+                  warp_wait(bar(B_CFULL + scf), kc & 1, abort_flag, a.err, 9) &&
+                  (c < 2 || warp_wait(bar(B_OPSFREE + ob), ((c >> 1) - 1) & 1, abort_flag, a.err, 15))))
+                break;
+            const float *cf = coef0 + scf * CF_FLOATS;
             // the X operands, 16-byte vectors of 128-byte rows (a vector keeps its
             // place under the swizzle, so its row is its index / 8):
             //   SISO:  Xw = diag(xs) x
@@ -785,8 +814,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint8_t *xt = sm + L::OFF_X + sx * L::SZ_X;
                 uint4 *dw = reinterpret_cast<uint4 *>(sm + L::OFF_XW + ob * (Q * P * 2));
                 uint4 *dr = reinterpret_cast<uint4 *>(sm + L::OFF_XR + ob * (Q * P * 2));
-#pragma unroll
-                for (int v = pt; v < Q * P / 8; v += PREP_THREADS) {
+#pragma unroll 4
+                for (int v = l32; v < Q * P / 8; v += 32) {
                     const int row = v >> 3, pc = v & 7;
                     const int sq = row / R;                       // token of the row
                     const float sc = cf[CF_XS + sq];
@@ -822,20 +851,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
             }
             fence_async_smem();
-            named_bar(1, PREP_THREADS);
-            if (tg == 15) {
-                // the last token group ends at the chunk's last token
-                *reinterpret_cast<float4 *>(phic + 4 * j4) = make_float4(phi[0], phi[1], phi[2], phi[3]);
-                if (last_chunk && a.angle_out)
-                    *reinterpret_cast<float4 *>(a.angle_out + lane_id * NP2 + 4 * j4) =
-                        make_float4(phi[0], phi[1], phi[2], phi[3]);
-                if (SO && c == nchunks - 1)
-                    *reinterpret_cast<float4 *>(slot_out + SLOT_PHIL + 4 * j4) =
-                        make_float4(phi[0], phi[1], phi[2], phi[3]);
-            }
-            if (pt == 0) {
+            __syncwarp();
+            if (l32 == 0) {
                 mbar_arrive(bar(B_OPSREADY + ob));
-                mbar_arrive(bar(B_BEMPTY + sb));
                 mbar_arrive(bar(B_XEMPTY + sx));
                 mbar_arrive(bar(B_CEMPTY + scf));
             }
@@ -845,16 +863,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         // The whole warp walks the chunks converged, so the descriptors are
         // warp-uniform; one elected lane issues each UMMA and commit.
         {
-            const uint32_t id_kk = idesc(64, 64, 0, 0);    // D1 = Cbar . Bsc^T
+            const uint32_t id_kk = idesc(64, 64, 0, 0);    // D1 = Cbar . Bbar^T
             const uint32_t id_kmn = idesc(64, 64, 0, 1);   // D2, D3: B operand MN-major
             const uint32_t id_st = idesc(128, 64, 1, 1);   // D4: A and B MN-major
             // Descriptors are built once; a K-step of a UMMA only moves the start
             // address field (16-byte units, low bits of the descriptor).
             // (a buffer switch adds its byte offset / 16 to the start field)
             const uint64_t d_sp = sdesc(sbase + L::OFF_SP, 16, 1024);
-            const uint64_t d_bsc_k0 = sdesc(sbase + L::OFF_BSC, 16, 1024);
+            const uint64_t d_bb_k0 = sdesc(sbase + L::OFF_BB, 16, 1024);
             const uint64_t d_cb_k0 = sdesc(sbase + L::OFF_CB, 16, 1024);
-            const uint64_t d_bsc_mn0 = sdesc(sbase + L::OFF_BSC, Q * 128, 1024);
+            const uint64_t d_bb_mn0 = sdesc(sbase + L::OFF_BB, Q * 128, 1024);
             const uint64_t d_xw0 = sdesc(sbase + L::OFF_XW, Q * 128, 1024);
             const uint64_t d_xr0 = sdesc(sbase + L::OFF_XR, Q * 128, 1024);
             const uint64_t d_gb0 = sdesc(sbase + L::OFF_GB, N * 128, 1024);
@@ -868,8 +886,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             auto kstep_mn = [](int kk) { return (uint64_t)((kk * 2048) >> 4); };
             for (int c = 0; c < nchunks; c++) {
                 const int sx = c % L::NXR, ob = c & 1;
-                const uint64_t d_bsc_k = d_bsc_k0 + ob * STEP_BC, d_cb_k = d_cb_k0 + ob * STEP_BC;
-                const uint64_t d_bsc_mn = d_bsc_mn0 + ob * STEP_BC, d_xw = d_xw0 + ob * STEP_XP;
+                const uint64_t d_bb_k = d_bb_k0 + ob * STEP_BC, d_cb_k = d_cb_k0 + ob * STEP_BC;
+                const uint64_t d_bb_mn = d_bb_mn0 + ob * STEP_BC, d_xw = d_xw0 + ob * STEP_XP;
                 const uint64_t dx = (R == 1) ? d_x0 + (uint64_t)sx * STEP_X : d_xr0 + ob * STEP_XP;
                 const uint64_t dg = d_gb0 + ((c + 1) & 1) * STEP_GB;   // state after chunk c-1
                 if (!warp_wait_spin(bar(B_OPSREADY + ob), (c >> 1) & 1, abort_flag, a.err, 10)) break;
@@ -879,7 +897,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     tc_fence_after();
                     if (elect_one()) {
                         for (int kk = 0; kk < Q / 16; kk++)
-                            umma(tmem + COL_D4, d_bsc_mn + kstep_mn(kk), d_xw + kstep_mn(kk), id_st, kk > 0);
+                            umma(tmem + COL_D4, d_bb_mn + kstep_mn(kk), d_xw + kstep_mn(kk), id_st, kk > 0);
                         umma_commit(bar(B_STFULL));
                         umma_commit(bar(B_OPSFREE + ob));
                     }
@@ -891,7 +909,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (elect_one()) {
 #pragma unroll 1
                     for (int kk = 0; kk < N / 16; kk++)
-                        umma(tmem + COL_D1, d_cb_k + kstep_k(kk), d_bsc_k + kstep_k(kk), id_kk, kk > 0);
+                        umma(tmem + COL_D1, d_cb_k + kstep_k(kk), d_bb_k + kstep_k(kk), id_kk, kk > 0);
                     umma_commit(bar(B_SFULL));
                 }
                 __syncwarp();
@@ -900,7 +918,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (elect_one()) {
 #pragma unroll 1
                     for (int kk = 0; kk < Q / 16; kk++)
-                        umma(tmem + COL_D4, d_bsc_mn + kstep_mn(kk), d_xw + kstep_mn(kk), id_st, kk > 0);
+                        umma(tmem + COL_D4, d_bb_mn + kstep_mn(kk), d_xw + kstep_mn(kk), id_st, kk > 0);
                     umma_commit(bar(B_STFULL));
                 }
                 __syncwarp();
@@ -1065,10 +1083,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                             const int col = c0 + 8 * i + cq;
                             const int s0 = col / R, s1 = (col + 1) / R;   // tokens of the two columns
                             const float w0 = cf[CF_WM + s0], w1 = cf[CF_WM + s1];
-                            v[4 * i + 0] *= s0 < ta ? rta * w0 : (s0 == ta ? rta * gta : 0.f);
-                            v[4 * i + 1] *= s1 < ta ? rta * w1 : (s1 == ta ? rta * gta : 0.f);
-                            v[4 * i + 2] *= s0 < tb ? rtb * w0 : (s0 == tb ? rtb * gtb : 0.f);
-                            v[4 * i + 3] *= s1 < tb ? rtb * w1 : (s1 == tb ? rtb * gtb : 0.f);
+                            v[4 * i + 0] *= s0 < ta ? rta * w0 : (s0 == ta ? gta : 0.f);
+                            v[4 * i + 1] *= s1 < ta ? rta * w1 : (s1 == ta ? gta : 0.f);
+                            v[4 * i + 2] *= s0 < tb ? rtb * w0 : (s0 == tb ? gtb : 0.f);
+                            v[4 * i + 3] *= s1 < tb ? rtb * w1 : (s1 == tb ? gtb : 0.f);
                             const int cc = col >> 3;
                             *reinterpret_cast<uint32_t *>(sp + ra * 128 + ((cc ^ (ra & 7)) << 4) + 2 * cq) =
                                 pack_bf16(v[4 * i], v[4 * i + 1]);
@@ -1173,7 +1191,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncthreads();
     // prev_Bx = sum_r Bbar_{T-1,r} X_{T-1,r}^T (rotated, unscaled B rows kept by
     // the rotation warps; X_{T-1,r} = W_x[r] x_{T-1})
-    if (!SO && last_seg && !*abort_flag && a.prevBx_out && warp >= W_EPI0) {
+    if (!SO && last_seg && !*abort_flag && a.prevBx_out && warp >= W_EPI0 && warp < W_EPI0 + EPI_WARPS) {
         const int et = tid - W_EPI0 * 32;
         const int n = et & (N - 1), half = et >> 7;
         const int c = nchunks - 1;
