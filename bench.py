@@ -154,14 +154,15 @@ def source_hash(paths):
     return h.hexdigest()[:16]
 
 
-def traffic_record(kernel, src_paths):
-    """DRAM bytes per launch from a committed ncu summary, only if the kernel's
-    sources are unchanged since the counters were taken."""
+def traffic_record(key, src_paths):
+    """DRAM bytes per launch of a kernel on one workload ("kernel:workload")
+    from a committed ncu summary, only if the kernel's sources are unchanged
+    since the counters were taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
-        rec = json.load(f).get(kernel)
+        rec = json.load(f).get(key)
     if not rec or rec.get("source_hash") != source_hash(src_paths):
         return None
     return rec
@@ -428,7 +429,7 @@ def run_ours(args, world, rank, local):
 
     peaks, peak_kind = load_peaks()
     achieved = w.bytes / kernel_s / 1e9
-    tr = traffic_record(w.kernel, w.srcs)
+    tr = traffic_record(w.kernel + ":" + w.c["name"], w.srcs)
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": round(achieved / peaks["hbm_gbs"], 4),
             "traffic": (tr["dram_bytes_per_launch"] if tr else None),

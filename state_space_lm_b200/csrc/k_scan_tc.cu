@@ -113,8 +113,10 @@ enum {
     B_OPSFREE = B_OPSREADY + 2,     // 2: the UMMAs reading them are done
     B_SFULL = B_OPSFREE + 2,
     B_STAKEN, B_SPFULL,             // scores in TMEM / read / masked scores written
-    B_YFULL, B_YTAKEN,              // output accumulators done / read
-    B_STFULL, B_STTAKEN,            // chunk state done / folded into the state
+    B_YFULL,                        // output accumulators done
+    B_YTAKEN,                       // 2: inter-chunk accumulator (double-buffered) read
+    B_STFULL = B_YTAKEN + 2,        // chunk state done
+    B_STTAKEN,                      // chunk state folded into the state
     B_DRAIN,
     NBAR
 };
@@ -123,8 +125,10 @@ constexpr int smem_bytes() { return Lay<R>::OFF_BAR + NBAR * 8 + 16 + 1024; }   
 static_assert(smem_bytes<1>() <= 227 * 1024 && smem_bytes<2>() <= 227 * 1024 && smem_bytes<4>() <= 227 * 1024,
               "shared memory budget");
 
-constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t COL_D1 = 0, COL_D2 = 64, COL_D3 = 128, COL_D4 = 192;
+// D3 is double-buffered (chunk c uses COL_D3 + (c & 1) * D3_STRIDE), so the
+// inter-chunk UMMA of chunk c does not wait for the outputs of chunk c-1
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t COL_D1 = 0, COL_D2 = 64, COL_D3 = 128, COL_D4 = 192, D3_STRIDE = 128;
 
 struct TcArgs {
     void *y;               // (Bt, T, H, P) bf16
@@ -447,6 +451,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_init(bar(B_SPFULL), 8);
         mbar_init(bar(B_YFULL), 1);
         mbar_init(bar(B_YTAKEN), 8);
+        mbar_init(bar(B_YTAKEN + 1), 8);
         mbar_init(bar(B_STFULL), 1);
         mbar_init(bar(B_STTAKEN), 8);
         mbar_init(bar(B_DRAIN), 1);
@@ -922,12 +927,18 @@ __global__ void __launch_bounds__(THREADS, 1)
                     umma_commit(bar(B_STFULL));
                 }
                 __syncwarp();
-                if (c > 0 && !warp_wait_spin(bar(B_YTAKEN), (c - 1) & 1, abort_flag, a.err, 13)) break;
+                // D3 buffer c & 1 was last read by the outputs of chunk c - 2
+                if (c > 1 && !warp_wait_spin(bar(B_YTAKEN + (c & 1)), ((c >> 1) - 1) & 1, abort_flag, a.err, 13))
+                    break;
                 tc_fence_after();
                 if (elect_one()) {
+                    const uint32_t d3 = tmem + COL_D3 + (uint32_t)(c & 1) * D3_STRIDE;
 #pragma unroll 1
                     for (int kk = 0; kk < N / 16; kk++)
-                        umma(tmem + COL_D3, d_cb_k + kstep_k(kk), dg + kstep_mn(kk), id_kmn, kk > 0);
+                        umma(d3, d_cb_k + kstep_k(kk), dg + kstep_mn(kk), id_kmn, kk > 0);
+                    // SISO: B, C and Xw of chunk c are read by now (the intra UMMA
+                    // reads the x tile and the scores only)
+                    if (R == 1) umma_commit(bar(B_OPSFREE + ob));
                 }
                 __syncwarp();
                 if (!warp_wait_spin(bar(B_SPFULL), c & 1, abort_flag, a.err, 14)) break;
@@ -937,7 +948,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     for (int kk = 0; kk < Q / 16; kk++)
                         umma(tmem + COL_D2, d_sp + (uint64_t)((kk * 32) >> 4), dx + kstep_mn(kk), id_kmn, kk > 0);
                     umma_commit(bar(B_YFULL));
-                    umma_commit(bar(B_OPSFREE + ob));  // every operand of chunk c has been read
+                    if (R > 1) umma_commit(bar(B_OPSFREE + ob));   // X_r is read by the intra UMMA
                     umma_commit(bar(B_XEMPTY + sx));
                 }
                 __syncwarp();
@@ -1135,7 +1146,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         const int c0 = cb0 + 16 * hf;        // 16 columns: two groups of 8
                         float y2[8], y3[8];
                         tmem_ld16x256b_x2(tl + COL_D2 + c0, y2);
-                        tmem_ld16x256b_x2(tl + COL_D3 + c0, y3);
+                        tmem_ld16x256b_x2(tl + COL_D3 + (uint32_t)(c & 1) * D3_STRIDE + c0, y3);
                         tmem_wait_ld();
 #pragma unroll
                         for (int i = 0; i < 2; i++) {
@@ -1172,7 +1183,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (l32 == 0) {
-                    mbar_arrive(bar(B_YTAKEN));
+                    mbar_arrive(bar(B_YTAKEN + (c & 1)));
                     mbar_arrive(bar(B_XEMPTY + sx));
                     mbar_arrive(bar(B_CEMPTY + scf));
                 }
