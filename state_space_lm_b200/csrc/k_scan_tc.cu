@@ -429,14 +429,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(bar(B_BFULL + i), 1);
             mbar_init(bar(B_BEMPTY + i), 1);
         }
-        // x tiles are released by the X-operand warp, the intra UMMA and each
-        // of the eight output-writing warps (state-only pass: the X-operand
-        // warp alone); coefficients by the rotation group, the X-operand warp
+        // x tiles are released by the X-operand warp, the intra UMMA and (MIMO)
+        // each of the eight output-writing warps (state-only pass: the
+        // X-operand warp alone); coefficients by the rotation group, the X-operand warp
         // and each epilogue warp; a chunk's operands are ready once both the
         // rotation group and the X-operand warp have written theirs
         for (int i = 0; i < L::NXR; i++) {
             mbar_init(bar(B_XFULL + i), 1);
-            mbar_init(bar(B_XEMPTY + i), SO ? 1 : 2 + EPI_WARPS);
+            mbar_init(bar(B_XEMPTY + i), SO ? 1 : (R == 1 ? 2 : 2 + EPI_WARPS));
         }
         for (int i = 0; i < NC; i++) {
             mbar_init(bar(B_CFULL + i), 1);
@@ -711,9 +711,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             {
                 const float4 p0 = *reinterpret_cast<const float4 *>(phic + 4 * j4);
                 phi[0] = p0.x; phi[1] = p0.y; phi[2] = p0.z; phi[3] = p0.w;
-                for (int g2 = 0; g2 < tg; g2++) {
-                    const float4 pg = *reinterpret_cast<const float4 *>(part + g2 * NP2 + 4 * j4);
-                    phi[0] += pg.x; phi[1] += pg.y; phi[2] += pg.z; phi[3] += pg.w;
+                // unrolled and predicated, so the loads of all earlier groups
+                // are in flight together (the sum keeps its order)
+#pragma unroll
+                for (int g2 = 0; g2 < 15; g2++) {
+                    if (g2 < tg) {
+                        const float4 pg = *reinterpret_cast<const float4 *>(part + g2 * NP2 + 4 * j4);
+                        phi[0] += pg.x; phi[1] += pg.y; phi[2] += pg.z; phi[3] += pg.w;
+                    }
                 }
             }
             // pass 2: rotate my tokens (the same angles for every rank).  The
@@ -1098,6 +1103,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                             v[4 * i + 1] *= s1 < ta ? rta * w1 : (s1 == ta ? gta : 0.f);
                             v[4 * i + 2] *= s0 < tb ? rtb * w0 : (s0 == tb ? gtb : 0.f);
                             v[4 * i + 3] *= s1 < tb ? rtb * w1 : (s1 == tb ? gtb : 0.f);
+                            if (R == 1) {
+                                // SISO: the skip D x_t rides on the intra UMMA as D on the
+                                // diagonal of the scores (its B operand is x itself)
+                                v[4 * i + 0] += s0 == ta ? Dh : 0.f;
+                                v[4 * i + 1] += s1 == ta ? Dh : 0.f;
+                                v[4 * i + 2] += s0 == tb ? Dh : 0.f;
+                                v[4 * i + 3] += s1 == tb ? Dh : 0.f;
+                            }
                             const int cc = col >> 3;
                             *reinterpret_cast<uint32_t *>(sp + ra * 128 + ((cc ^ (ra & 7)) << 4) + 2 * cq) =
                                 pack_bf16(v[4 * i], v[4 * i + 1]);
@@ -1171,10 +1184,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                                 for (int i = 0; i < 2; i++) {
                                     const int col = c0 + 8 * i + cq, cc = col >> 3;
-                                    const float2 xf = unpack_bf16(*reinterpret_cast<const uint32_t *>(
-                                        xr + t * 128 + ((cc ^ (t & 7)) << 4) + 2 * cq));
-                                    *reinterpret_cast<uint32_t *>(yrow + col) = pack_bf16(
-                                        fmaf(Dh, xf.x, y2[4 * i + 2 * hb]), fmaf(Dh, xf.y, y2[4 * i + 2 * hb + 1]));
+                                    float y0 = y2[4 * i + 2 * hb], y1 = y2[4 * i + 2 * hb + 1];
+                                    if (R > 1) {   // SISO has D x in the intra term already
+                                        const float2 xf = unpack_bf16(*reinterpret_cast<const uint32_t *>(
+                                            xr + t * 128 + ((cc ^ (t & 7)) << 4) + 2 * cq));
+                                        y0 = fmaf(Dh, xf.x, y0);
+                                        y1 = fmaf(Dh, xf.y, y1);
+                                    }
+                                    *reinterpret_cast<uint32_t *>(yrow + col) = pack_bf16(y0, y1);
                                 }
                             }
                         }
@@ -1184,7 +1201,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 __syncwarp();
                 if (l32 == 0) {
                     mbar_arrive(bar(B_YTAKEN + (c & 1)));
-                    mbar_arrive(bar(B_XEMPTY + sx));
+                    if (R > 1) mbar_arrive(bar(B_XEMPTY + sx));
                     mbar_arrive(bar(B_CEMPTY + scf));
                 }
             }
