@@ -96,8 +96,8 @@ struct Lay {
     static constexpr int OFF_BLAST = OFF_COEF + NC * CF_FLOATS * 4;  // fp32 [R][N]
     static constexpr int OFF_WXY = OFF_BLAST + R * N * 4;            // fp32 [2][R][P] (R > 1)
     static constexpr int OFF_PHIC = OFF_WXY + (R > 1 ? 2 * R * P * 4 : 0);  // fp32 [NP2]
-    static constexpr int OFF_PART = OFF_PHIC + NP2 * 4;       // fp32 [16][NP2] token-group angle sums
-    static constexpr int OFF_INV = OFF_PART + 16 * NP2 * 4;   // fp32 [2][Q] QkNorm inverse RMS
+    static constexpr int OFF_PART = OFF_PHIC + NP2 * 4;       // fp32 [8][NP2] per-warp angle sums
+    static constexpr int OFF_INV = OFF_PART + 8 * NP2 * 4;    // fp32 [2][Q] QkNorm inverse RMS
     static constexpr int OFF_BAR = OFF_INV + 2 * Q * 4;       // mbarriers
 };
 
@@ -380,12 +380,12 @@ __device__ __forceinline__ uint32_t sw128(int row, int col) {
 
 // sin/cos with Cody-Waite reduction to [-pi, pi] (2 pi split into an exactly
 // representable head and a tail), then the hardware approximation there.
-__device__ __forceinline__ void sincos_rr(float x, float *s, float *c) {
-    const float k = rintf(x * 0.15915494309189535f);
-    float r = fmaf(-k, 6.28125f, x);
-    r = fmaf(-k, 1.9353071795864769e-3f, r);
-    __sincosf(r, s, c);
+constexpr float INV_2PI = 0.15915494309189535f, TWO_PI_HI = 6.28125f, TWO_PI_LO = 1.9353071795864769e-3f;
+__device__ __forceinline__ float reduce_2pi(float x) {
+    const float k = rintf(x * INV_2PI);
+    return fmaf(-k, TWO_PI_LO, fmaf(-k, TWO_PI_HI, x));
 }
+__device__ __forceinline__ void sincos_rr(float x, float *s, float *c) { __sincosf(reduce_2pi(x), s, c); }
 
 // SO (state only): the first pass over all but the last segment of each lane;
 // it loads x, B, theta (no C), runs only the chunk-state UMMA, starts from a
@@ -691,9 +691,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                     if (l32 == 0) inv[r] = rsqrtf(ss / N + nr.eps);
                 }
             }
-            // pass 1: angle increments of my token group
+            // pass 1: angle increments of my token group, then the angle entering
+            // it: the chunk's entering angle + the earlier warps' sums + (second
+            // token group of a warp) the first group's sum
             float dph[TPT][4];
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            float amax = 0.f;                      // bound on my angle's drift inside the chunk
 #pragma unroll
             for (int u = 0; u < TPT; u++) {
                 const float d = cf[CF_DT + i0 + u];
@@ -704,30 +707,46 @@ __global__ void __launch_bounds__(THREADS, 1)
                 dph[u][3] = d * t4.w;
 #pragma unroll
                 for (int q = 0; q < 4; q++) acc[q] += dph[u][q];
+                amax += fmaxf(fmaxf(fabsf(dph[u][0]), fabsf(dph[u][1])), fmaxf(fabsf(dph[u][2]), fabsf(dph[u][3])));
             }
-            *reinterpret_cast<float4 *>(part + tg * NP2 + 4 * j4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            const int wp = pt >> 5;
+            float first[4];                        // the warp's first token group's sums
+#pragma unroll
+            for (int q = 0; q < 4; q++) first[q] = __shfl_sync(0xffffffffu, acc[q], l32 & 15);
+            if (l32 >= 16)
+                *reinterpret_cast<float4 *>(part + wp * NP2 + 4 * j4) =
+                    make_float4(first[0] + acc[0], first[1] + acc[1], first[2] + acc[2], first[3] + acc[3]);
             named_bar(1, PREP_THREADS);
             float phi[4];
             {
                 const float4 p0 = *reinterpret_cast<const float4 *>(phic + 4 * j4);
                 phi[0] = p0.x; phi[1] = p0.y; phi[2] = p0.z; phi[3] = p0.w;
-                // unrolled and predicated, so the loads of all earlier groups
-                // are in flight together (the sum keeps its order)
 #pragma unroll
-                for (int g2 = 0; g2 < 15; g2++) {
-                    if (g2 < tg) {
-                        const float4 pg = *reinterpret_cast<const float4 *>(part + g2 * NP2 + 4 * j4);
+                for (int w2 = 0; w2 < NPREP - 1; w2++) {
+                    if (w2 < wp) {
+                        const float4 pg = *reinterpret_cast<const float4 *>(part + w2 * NP2 + 4 * j4);
                         phi[0] += pg.x; phi[1] += pg.y; phi[2] += pg.z; phi[3] += pg.w;
                     }
                 }
+                if (l32 >= 16) {
+#pragma unroll
+                    for (int q = 0; q < 4; q++) phi[q] += first[q];
+                }
             }
+            // sin/cos of a small angle need no range reduction per token: reduce
+            // the entering angle once and advance the reduced copy, unless some
+            // increment is large (then every token reduces its own angle)
+            const bool fast = !__any_sync(0xffffffffu, amax > 256.f);
+            float phr[4];
+#pragma unroll
+            for (int q = 0; q < 4; q++) phr[q] = reduce_2pi(phi[q]);
             // pass 2: rotate my tokens (the same angles for every rank).  The
             // token loop stays rolled (a small hot loop); the QkNorm / bias
             // variant is a separate copy of it, so the plain one carries none
             // of that code.
             const bool last_chunk = last_seg && (c == nchunks - 1);
-            auto rotate_tokens = [&](auto generic) {
-                constexpr bool G = decltype(generic)::value;
+            auto rotate_tokens = [&](auto generic, auto fast_sc) {
+                constexpr bool G = decltype(generic)::value, F = decltype(fast_sc)::value;
 #pragma unroll
                 for (int u = 0; u < TPT; u++) {
                     const int i = i0 + u;
@@ -740,8 +759,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                     float sn[4], cs[4];
 #pragma unroll
                     for (int q = 0; q < 4; q++) {
-                        phi[q] += d[q];
-                        sincos_rr(phi[q], &sn[q], &cs[q]);
+                        if (F) {
+                            phr[q] += d[q];
+                            __sincosf(phr[q], &sn[q], &cs[q]);
+                        } else {
+                            phi[q] += d[q];
+                            sincos_rr(phi[q], &sn[q], &cs[q]);
+                        }
                     }
 #pragma unroll 1
                     for (int r = 0; r < R; r++) {
@@ -786,8 +810,15 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                 }
             };
-            if (has_norm || has_bias) rotate_tokens(BoolC<true>{});
-            else rotate_tokens(BoolC<false>{});
+            if (has_norm || has_bias) {
+                rotate_tokens(BoolC<true>{}, BoolC<false>{});
+            } else if (fast) {
+                rotate_tokens(BoolC<false>{}, BoolC<true>{});
+#pragma unroll
+                for (int q = 0; q < 4; q++) phi[q] += acc[q];   // the exact angle after my tokens
+            } else {
+                rotate_tokens(BoolC<false>{}, BoolC<false>{});
+            }
             load_theta(c + 1);                     // in flight while the X operands are built
             fence_async_smem();
             named_bar(1, PREP_THREADS);
