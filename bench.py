@@ -93,7 +93,7 @@ class ClockSampler:
         "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
     }
 
-    def __init__(self, device_index, period_s=0.002):
+    def __init__(self, device_index, period_s=0.0005):
         self.period = period_s
         self.samples = []
         self.reasons = 0
