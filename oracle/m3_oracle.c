@@ -527,3 +527,109 @@ int m3o_step_decode(const double *x, const double *dt, const double *A,
     free(h1); free(u1); free(a1);
     return rc;
 }
+
+/* One MIMO decode step (rank R, W_x/W_y may be NULL for all ones): the MIMO
+ * loop body for a single token, carrying (h, prev_Bx, angle) in place
+ * (dotLLM "Mamba-3 MIMO streaming decode": the state is rank-summed and the
+ * angle rank-free).  Per-token inputs are shaped as a one-token sequence. */
+int m3o_mimo_step_decode(const double *x, const double *dt, const double *A,
+                         const double *lam, const double *theta, const double *B,
+                         const double *C, const double *D, const double *Wx,
+                         const double *Wy, const m3o_bcnorm *nrm, m3o_dims d,
+                         double *h, double *prevBx, double *angle, double *y, int nthreads)
+{
+    if (!h || !prevBx || !angle) return -1;
+    d.seqlen = 1;
+    long lanes = d.batch * d.nheads, NP = d.dstate * d.headdim;
+    double *h1 = (double *)malloc(sizeof(double) * (lanes * NP + 1));
+    double *u1 = (double *)malloc(sizeof(double) * (lanes * NP + 1));
+    double *a1 = (double *)malloc(sizeof(double) * (lanes * (d.dstate / 2) + 1));
+    int rc = m3o_mimo_loop(x, dt, A, lam, theta, B, C, D, Wx, Wy, nrm, h, prevBx, angle,
+                           d, y, h1, u1, a1, nthreads);
+    if (rc >= 0) {
+        memcpy(h, h1, sizeof(double) * lanes * NP);
+        memcpy(prevBx, u1, sizeof(double) * lanes * NP);
+        memcpy(angle, a1, sizeof(double) * lanes * (d.dstate / 2));
+    }
+    free(h1); free(u1); free(a1);
+    return rc;
+}
+
+/* One decode step on the factored previous-input state (torchmamba "Models":
+ * the SISO cache carries (angle, ssm, x_prev, b_prev); dotLLM "Mamba-3 MIMO
+ * streaming decode": per-rank key/value states instead of their product).
+ * The previous token's input term is rebuilt from its factors,
+ *   U_prev[n][p] = sum_r b_prev[r][n] W_x[h,r,p] x_prev[p],
+ * the step is the MIMO recurrence for one token (rank 1 with W = 1 is the
+ * SISO step), and afterwards b_prev <- B_rot_{t,r}, x_prev <- x_t.
+ * In/out: h (Bt,H,N,P), bprev (Bt,H,R,N), xprev (Bt,H,P), angle (Bt,H,N/2).
+ * Inputs: x (Bt,H,P), dt/lam (Bt,H), theta (Bt,H,N/2), B/C (Bt,H,R,N),
+ * W_x/W_y (H,R,P) or NULL.  Output y (Bt,H,P). */
+int m3o_step_decode_factored(const double *x, const double *dt, const double *A,
+                             const double *lam, const double *theta, const double *B,
+                             const double *C, const double *D, const double *Wx,
+                             const double *Wy, const m3o_bcnorm *nrm, m3o_dims d,
+                             double *h, double *bprev, double *xprev, double *angle,
+                             double *y)
+{
+    if (!h || !bprev || !xprev || !angle || !x || !dt || !A || !lam || !theta || !B || !C || !D || !y)
+        return -1;
+    if (d.batch < 0 || d.nheads < 0 || d.headdim <= 0 || d.dstate <= 0 || d.dstate % 2 || d.rank < 1)
+        return -1;
+    long H = d.nheads, P = d.headdim, N = d.dstate, R = d.rank, NP = N * P;
+    double *tmp = (double *)malloc(sizeof(double) * N);
+    double *Bb = (double *)malloc(sizeof(double) * R * N);
+    double *Cb = (double *)malloc(sizeof(double) * R * N);
+    double *Xr = (double *)malloc(sizeof(double) * R * P);
+    double *Xp = (double *)malloc(sizeof(double) * R * P);
+    for (long lane = 0; lane < d.batch * H; lane++) {
+        long hh = lane % H;
+        double dl = dt[lane], lm = lam[lane];
+        double al = exp(dl * A[hh]);
+        double be = (1.0 - lm) * dl * al;
+        double ga = lm * dl;
+        double *phi = angle + lane * (N / 2);
+        for (long i = 0; i < N / 2; i++) phi[i] += dl * theta[lane * (N / 2) + i];
+        const double *xt = x + lane * P;
+        double *xo = xprev + lane * P;
+        for (long r = 0; r < R; r++) {
+            long off = (lane * R + r) * N;
+            bc_prepare(B + off, N, nrm ? nrm->normw_B : NULL,
+                       nrm && nrm->bias_B ? nrm->bias_B + (hh * R + r) * N : NULL, nrm ? nrm->eps : 0.0, tmp);
+            rotate_pairs(tmp, phi, N, Bb + r * N);
+            bc_prepare(C + off, N, nrm ? nrm->normw_C : NULL,
+                       nrm && nrm->bias_C ? nrm->bias_C + (hh * R + r) * N : NULL, nrm ? nrm->eps : 0.0, tmp);
+            rotate_pairs(tmp, phi, N, Cb + r * N);
+            for (long p = 0; p < P; p++) {
+                double w = Wx ? Wx[(hh * R + r) * P + p] : 1.0;
+                Xr[r * P + p] = w * xt[p];
+                Xp[r * P + p] = w * xo[p];
+            }
+        }
+        double *hs = h + lane * NP;
+        const double *bp = bprev + lane * R * N;
+        for (long n = 0; n < N; n++)
+            for (long p = 0; p < P; p++) {
+                double up = 0.0, ut = 0.0;
+                for (long r = 0; r < R; r++) {
+                    up += bp[r * N + n] * Xp[r * P + p];
+                    ut += Bb[r * N + n] * Xr[r * P + p];
+                }
+                hs[n * P + p] = al * hs[n * P + p] + be * up + ga * ut;
+            }
+        double *yt = y + lane * P;
+        for (long p = 0; p < P; p++) {
+            double acc = 0.0;
+            for (long r = 0; r < R; r++) {
+                double yr = 0.0;
+                for (long n = 0; n < N; n++) yr += Cb[r * N + n] * hs[n * P + p];
+                acc += (Wy ? Wy[(hh * R + r) * P + p] : 1.0) * yr;
+            }
+            yt[p] = acc + D[hh] * xt[p];
+        }
+        memcpy(bprev + lane * R * N, Bb, sizeof(double) * R * N);
+        memcpy(xo, xt, sizeof(double) * P);
+    }
+    free(tmp); free(Bb); free(Cb); free(Xr); free(Xp);
+    return 0;
+}

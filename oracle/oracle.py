@@ -64,7 +64,7 @@ class _Norm(ctypes.Structure):
 def _open(path):
     lib = ctypes.CDLL(path)
     for name in ("m3o_discretize", "m3o_rope_bc", "m3o_siso_loop", "m3o_mimo_loop",
-                 "m3o_siso_chunked", "m3o_step_decode"):
+                 "m3o_siso_chunked", "m3o_step_decode", "m3o_mimo_step_decode", "m3o_step_decode_factored"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -224,3 +224,43 @@ def step_decode(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, prevBx, angle, nor
     if rc < 0:
         raise ValueError("oracle rejected the arguments")
     return y[:, 0], h, prevBx, angle
+
+
+def mimo_step_decode(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, prevBx, angle, Wx=None, Wy=None,
+                     norm=None, nthreads=0):
+    """One rank-R MIMO decode step on the full previous-input state.  B_t, C_t
+    (Bt,H,R,N).  Returns y_t (Bt,H,P), h, prev_Bx, angle (new arrays)."""
+    x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, Wx, Wy = (
+        _f64(a) for a in (x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, Wx, Wy))
+    h, prevBx, angle = (np.array(a, dtype=np.float64, copy=True) for a in (h, prevBx, angle))
+    Bt, H, P = x_t.shape
+    R, N = B_t.shape[-2], B_t.shape[-1]
+    y = np.empty((Bt, 1, H, P))
+    nptr, keep = _norm(norm)
+    rc = _load().m3o_mimo_step_decode(_p(x_t), _p(dt_t), _p(A), _p(lam_t), _p(theta_t), _p(B_t),
+                                      _p(C_t), _p(D), _p(Wx), _p(Wy), nptr, _dims(Bt, 1, H, P, N, R),
+                                      _p(h), _p(prevBx), _p(angle), _p(y), int(nthreads))
+    if rc < 0:
+        raise ValueError("oracle rejected the arguments")
+    return y[:, 0], h, prevBx, angle
+
+
+def step_decode_factored(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, bprev, xprev, angle,
+                         Wx=None, Wy=None, norm=None):
+    """One decode step on the factored previous-input state: bprev (Bt,H,R,N)
+    is the rotated B of the previous token per rank and xprev (Bt,H,P) its x.
+    B_t, C_t (Bt,H,R,N) (R = 1 for SISO).  Returns y_t, h, bprev, xprev, angle
+    (new arrays)."""
+    x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, Wx, Wy = (
+        _f64(a) for a in (x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, Wx, Wy))
+    h, bprev, xprev, angle = (np.array(a, dtype=np.float64, copy=True) for a in (h, bprev, xprev, angle))
+    Bt, H, P = x_t.shape
+    R, N = B_t.shape[-2], B_t.shape[-1]
+    y = np.empty((Bt, H, P))
+    nptr, keep = _norm(norm)
+    rc = _load().m3o_step_decode_factored(_p(x_t), _p(dt_t), _p(A), _p(lam_t), _p(theta_t), _p(B_t),
+                                          _p(C_t), _p(D), _p(Wx), _p(Wy), nptr, _dims(Bt, 1, H, P, N, R),
+                                          _p(h), _p(bprev), _p(xprev), _p(angle), _p(y))
+    if rc < 0:
+        raise ValueError("oracle rejected the arguments")
+    return y, h, bprev, xprev, angle

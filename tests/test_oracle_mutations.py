@@ -27,6 +27,9 @@ MUTATIONS = [
      "double al = exp(-dl * J->A[h]);\n        double be = (1.0 - lm) * dl * al;\n        double ga = lm * dl;\n        for (long i = 0; i < N / 2; i++) phi[i] += dl * J->theta[bth * (N / 2) + i];\n        bc_prepare"),
     ("MIMO contract without W_y", "acc += (J->Wy ? J->Wy[(h * R + r) * P + p] : 1.0) * yr;", "acc += yr;"),
     ("chunk lookahead dropped", "sg = (1.0 - J->lam[nx]) * J->dt[nx];", "sg = 0.0;"),
+    ("factored decode: previous term from the current x", "up += bp[r * N + n] * Xp[r * P + p];",
+     "up += bp[r * N + n] * Xr[r * P + p];"),
+    ("factored decode: b_prev not advanced", "memcpy(bprev + lane * R * N, Bb, sizeof(double) * R * N);", ""),
 ]
 
 PIN_CASES = [
@@ -38,6 +41,8 @@ PIN_CASES = [
     lambda o: pins.test_mimo_is_r2_siso_calls(o),
     lambda o: pins.test_split_schedules_siso(o, [2, 4]),
     lambda o: pins.test_chunked_equals_loop(o, 4, 37),
+    lambda o: pins.test_factored_decode_from_zero_equals_mimo_loop(o, 3),
+    lambda o: pins.test_mimo_decode_steps_equal_mimo_loop(o),
 ]
 
 

@@ -19,6 +19,10 @@ oracle's code:
 * split schedules: prefill + decode reproduces the one-shot scan (dotLLM pull
   request, "Mamba-3 streaming decode" and "MIMO streaming decode": schedules
   2+2+2, 1+1+1+1+1+1, 3+3, 4+2, 2+4, 1+2+3, 5+1);
+* MIMO decode steps, and decode steps on the factored previous-input state
+  (previous token's rotated B per rank and its x), reproduce the one-shot
+  MIMO scan (dotLLM pull request, "MIMO streaming decode"; TorchMamba README,
+  "Models": cache of angle, ssm, x_prev, b_prev);
 * chunked fp64 form equals the loop (ats-v2 README, "Mamba uses a chunked
   parallel scan": exact at float64);
 * rotation invariance and the trapezoid weights' sum.
@@ -316,6 +320,95 @@ def test_prefill_then_decode_steps(oracle_mod):
                                              h, u, a)
         ys.append(yt[:, None])
     close(np.concatenate(ys, 1), y1)
+    close(h, h1)
+    close(u, u1)
+    close(a, a1)
+
+
+# ----------------------------------------------------------------------------
+# MIMO decode, and decode on the factored previous-input state (dotLLM pull
+# request, "Mamba-3 MIMO streaming decode"; TorchMamba README, "Models": the
+# cache carries (angle, ssm, x_prev, b_prev)) == the one-shot MIMO scan
+# ----------------------------------------------------------------------------
+def _mimo_inputs(rng, Bt, T, H, P, N, R):
+    inp = rnd_inputs(rng, Bt=Bt, T=T, H=H, P=P, N=N, R=R)
+    if R == 1:   # the factored step takes B, C with an explicit rank axis
+        inp["B"], inp["C"] = inp["B"][:, :, :, None], inp["C"][:, :, :, None]
+    Wx = 1 + 0.3 * rng.standard_normal((H, R, P))
+    Wy = 1 + 0.3 * rng.standard_normal((H, R, P))
+    return inp, Wx, Wy
+
+
+def _tok(inp, t):
+    return [inp[k][:, t] for k in ("x", "dt")] + [inp["A"]] + [inp[k][:, t] for k in ("lam", "theta", "B", "C")] + [inp["D"]]
+
+
+def _outer(bprev, xprev, Wx):
+    """prev_Bx rebuilt from its factors: sum_r b_prev[r] (W_x[r] x_prev)^T."""
+    return np.einsum("bhrn,hrp,bhp->bhnp", bprev, Wx, xprev)
+
+
+@pytest.mark.parametrize("R", [1, 3])
+def test_factored_decode_from_zero_equals_mimo_loop(oracle_mod, R):
+    rng = np.random.default_rng(40 + R)
+    Bt, T, H, P, N = 2, 7, 2, 3, 6
+    inp, Wx, Wy = _mimo_inputs(rng, Bt, T, H, P, N, R)
+    y1, h1, u1, a1 = oracle_mod.mimo_loop(**inp, Wx=Wx, Wy=Wy)
+    h, bp, xp, a = np.zeros((Bt, H, N, P)), np.zeros((Bt, H, R, N)), np.zeros((Bt, H, P)), np.zeros((Bt, H, N // 2))
+    for t in range(T):
+        yt, h, bp, xp, a = oracle_mod.step_decode_factored(*_tok(inp, t), h, bp, xp, a, Wx=Wx, Wy=Wy)
+        close(yt, y1[:, t])
+    close(h, h1)
+    close(_outer(bp, xp, Wx), u1)
+    close(a, a1)
+
+
+def test_factored_decode_after_prefill(oracle_mod):
+    """Schedule 4 + 3: a prefill by the loop, then decode steps on the factored
+    state taken from the prefill's last token (its rotated B and its x)."""
+    rng = np.random.default_rng(44)
+    Bt, T, H, P, N, R, k = 2, 7, 3, 4, 8, 2, 4
+    inp, Wx, Wy = _mimo_inputs(rng, Bt, T, H, P, N, R)
+    y1, h1, u1, a1 = oracle_mod.mimo_loop(**inp, Wx=Wx, Wy=Wy)
+    pre = {kk: (v[:, :k] if kk in ("x", "dt", "lam", "theta", "B", "C") else v) for kk, v in inp.items()}
+    _, h, u, a = oracle_mod.mimo_loop(**pre, Wx=Wx, Wy=Wy)
+    Br, _, _ = oracle_mod.rope_bc(pre["B"], pre["C"], pre["theta"], pre["dt"])
+    bp, xp = Br[:, k - 1], inp["x"][:, k - 1]
+    close(_outer(bp, xp, Wx), u)       # the factors rebuild the prefill's prev_Bx
+    for t in range(k, T):
+        yt, h, bp, xp, a = oracle_mod.step_decode_factored(*_tok(inp, t), h, bp, xp, a, Wx=Wx, Wy=Wy)
+        close(yt, y1[:, t])
+    close(h, h1)
+    close(a, a1)
+
+
+def test_factored_decode_r1_equals_siso_decode(oracle_mod):
+    rng = np.random.default_rng(45)
+    Bt, T, H, P, N = 1, 6, 2, 5, 4
+    inp = rnd_inputs(rng, Bt=Bt, T=T, H=H, P=P, N=N)
+    h, u, a = np.zeros((Bt, H, N, P)), np.zeros((Bt, H, N, P)), np.zeros((Bt, H, N // 2))
+    hf, bp, xp, af = h.copy(), np.zeros((Bt, H, 1, N)), np.zeros((Bt, H, P)), a.copy()
+    for t in range(T):
+        ys, h, u, a = oracle_mod.step_decode(inp["x"][:, t], inp["dt"][:, t], inp["A"], inp["lam"][:, t],
+                                             inp["theta"][:, t], inp["B"][:, t], inp["C"][:, t], inp["D"],
+                                             h, u, a)
+        yf, hf, bp, xp, af = oracle_mod.step_decode_factored(
+            inp["x"][:, t], inp["dt"][:, t], inp["A"], inp["lam"][:, t], inp["theta"][:, t],
+            inp["B"][:, t, :, None], inp["C"][:, t, :, None], inp["D"], hf, bp, xp, af)
+        close(yf, ys)
+    close(hf, h)
+    close(_outer(bp, xp, np.ones((H, 1, P))), u)
+
+
+def test_mimo_decode_steps_equal_mimo_loop(oracle_mod):
+    rng = np.random.default_rng(46)
+    Bt, T, H, P, N, R = 2, 6, 2, 4, 6, 4
+    inp, Wx, Wy = _mimo_inputs(rng, Bt, T, H, P, N, R)
+    y1, h1, u1, a1 = oracle_mod.mimo_loop(**inp, Wx=Wx, Wy=Wy)
+    h, u, a = np.zeros((Bt, H, N, P)), np.zeros((Bt, H, N, P)), np.zeros((Bt, H, N // 2))
+    for t in range(T):
+        yt, h, u, a = oracle_mod.mimo_step_decode(*_tok(inp, t), h, u, a, Wx=Wx, Wy=Wy)
+        close(yt, y1[:, t])
     close(h, h1)
     close(u, u1)
     close(a, a1)
