@@ -196,10 +196,17 @@ def scan_flops(c):
 
 
 def decode_bytes(c):
-    Bt, H, P, N = c["batch"], c["nheads"], c["headdim"], c["dstate"]
+    """Algorithmic bytes of one decode step: the carried state read and written
+    once, the per-token inputs read once, y written once (W_x, W_y once per
+    head)."""
+    Bt, H, P, N, R = c["batch"], c["nheads"], c["headdim"], c["dstate"], c["rank"]
     es = 2
-    per_lane = 2 * 2 * N * P * 4 + 2 * (N // 2) * 4 + es * P + 2 * es * N + 8 + 4 * (N // 2) + es * P
-    return Bt * H * per_lane
+    if c.get("state") == "factored":   # h, b_prev (R, N), x_prev (P)
+        state = 2 * N * P * 4 + 2 * R * N * 4 + 2 * P * 4
+    else:                              # h, prev_Bx
+        state = 2 * 2 * N * P * 4
+    per_lane = state + 2 * (N // 2) * 4 + es * P + 2 * es * R * N + 8 + 4 * (N // 2) + es * P
+    return Bt * H * per_lane + (2 * H * R * P * 4 if R > 1 else 0)
 
 
 class ScanWorkload:
@@ -278,10 +285,11 @@ class ScanWorkload:
 
 
 class DecodeWorkload:
-    """Decode steps of the SISO scan: every step advances all (batch, head)
-    lanes by one token.  The carried state comes from a seeded prefill (a
-    chunked forward over the first ``seqlen`` tokens, untimed); the per-step
-    inputs of every step are drawn up front and resident in HBM."""
+    """Decode steps: every step advances all (batch, head) lanes by one token.
+    The carried state comes from a seeded prefill (a chunked forward over the
+    first ``seqlen`` tokens, untimed; for the factored state, its last token's
+    rotated B and x); the per-step inputs of every step are drawn up front and
+    resident in HBM."""
 
     def __init__(self, idx, device, nsteps):
         from state_space_lm_b200 import m3
@@ -293,31 +301,56 @@ class DecodeWorkload:
         g = inp.pop("generator")
         self.host_prefill = inp
         d = {k: v.to(device) for k, v in inp.items() if isinstance(v, torch.Tensor)}
-        _, self.h, self.u, self.a = m3.siso_chunked_fwd(d["x"], d["dt"], d["A"], d["lam"], d["theta"], d["B"],
-                                                        d["C"], d["D"], c["chunk"])
+        R = c["rank"]
+        self.factored = c.get("state") == "factored"
+        self.Wx, self.Wy = d.get("Wx"), d.get("Wy")
+        if R == 1:
+            _, self.h, self.u, self.a = m3.siso_chunked_fwd(d["x"], d["dt"], d["A"], d["lam"], d["theta"],
+                                                            d["B"], d["C"], d["D"], c["chunk"])
+        else:
+            _, self.h, self.u, self.a = m3.mimo_chunked_fwd(d["x"], d["dt"], d["A"], d["lam"], d["theta"],
+                                                            d["B"], d["C"], d["D"], c["chunk"], W_x=self.Wx,
+                                                            W_y=self.Wy)
+        if self.factored:
+            Br, _, _ = m3.rope_bc(d["B"], d["C"], d["theta"], d["dt"])
+            last = Br[:, -1]
+            self.bp = (last[:, :, None] if R == 1 else last).float().contiguous()
+            self.xp = d["x"][:, -1].float().contiguous()
+            self.u = None
         self.A, self.D = d["A"], d["D"]
-        self.steps_host = [gen.decode_step_inputs(g, Bt, H, P, N) for _ in range(nsteps)]
+        self.steps_host = [gen.decode_step_inputs(g, Bt, H, P, N, rank=R, rank_axis=self.factored)
+                           for _ in range(nsteps)]
         self.steps_dev = [{k: v.to(device) for k, v in st.items()} for st in self.steps_host]
         self.y = torch.empty(Bt, H, P, device=device, dtype=torch.bfloat16)
         self.i = 0
         self.units = Bt                           # one token per sequence per step
         self.bytes = decode_bytes(c)
         self.flops = 0
-        self.kernel = self.kernel_label = "k_decode"
+        self.kernel = self.kernel_label = "k_decode_gen" if (self.factored or R > 1) else "k_decode"
         self.srcs = [os.path.join(ROOT, "state_space_lm_b200", "csrc", "k_decode.cu")]
-        self.input_bytes = 2 * Bt * H * N * P * 4
+        self.input_bytes = (1 if self.factored else 2) * Bt * H * N * P * 4
 
     def step(self, dev=None, out=None, stream=None):
         st = self.steps_dev[self.i % len(self.steps_dev)] if dev is None else dev
         self.i += 1
-        self.m3.step_decode(st["x"], st["dt"], self.A, st["lam"], st["theta"], st["B"], st["C"], self.D,
-                            self.h, self.u, self.a, y_out=self.y if out is None else out, stream=stream)
+        y = self.y if out is None else out
+        if self.factored:
+            self.m3.step_decode_factored(st["x"], st["dt"], self.A, st["lam"], st["theta"], st["B"], st["C"],
+                                         self.D, self.h, self.bp, self.xp, self.a, W_x=self.Wx, W_y=self.Wy,
+                                         y_out=y, stream=stream)
+        elif self.c["rank"] > 1:
+            self.m3.mimo_step_decode(st["x"], st["dt"], self.A, st["lam"], st["theta"], st["B"], st["C"], self.D,
+                                     self.h, self.u, self.a, W_x=self.Wx, W_y=self.Wy, y_out=y, stream=stream)
+        else:
+            self.m3.step_decode(st["x"], st["dt"], self.A, st["lam"], st["theta"], st["B"], st["C"], self.D,
+                                self.h, self.u, self.a, y_out=y, stream=stream)
 
     def config(self):
         c = self.c
         return {"workload": c["name"], "batch": c["batch"], "nheads": c["nheads"], "headdim": c["headdim"],
                 "dstate": c["dstate"], "prefill": c["seqlen"], "decode_steps_per_call": 1,
-                "inputs": "x/B/C bf16, dt/lam/theta fp32 per step; fp32 state h, prev_Bx, angle",
+                "rank": c["rank"], "state": "factored (h, b_prev, x_prev)" if self.factored else "full (h, prev_Bx)",
+                "inputs": "x/B/C bf16, dt/lam/theta fp32 per step; fp32 state and angle",
                 "l2": "state larger than L2 (%.0f MB vs 126 MB), no flush" % (self.input_bytes / 1e6)}
 
 
@@ -358,7 +391,7 @@ def run_ours(args, world, rank, local):
     from state_space_lm_b200 import build, m3
     if not os.path.exists(build.LIB):
         raise SystemExit("CUDA library not built: run python -m state_space_lm_b200.build")
-    if args.config == 4:
+    if args.config >= 4:
         w = DecodeWorkload(args.config, device, args.steps + args.warmup)
     else:
         w = ScanWorkload(args.config, device)
@@ -513,7 +546,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=1, choices=[0, 1, 2, 3, 4])
+    ap.add_argument("--config", type=int, default=1, choices=[0, 1, 2, 3, 4, 5, 6])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

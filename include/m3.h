@@ -166,6 +166,44 @@ m3_status m3_step_decode(const void *x_t, const float *dt_t, const float *A,
                          const m3_bcnorm *norm, m3_dims d, float *h, float *prevBx,
                          float *angle, void *y_t, void *stream);
 
+/* S5 for rank R -- one MIMO decode step on the full previous-input state.
+ * (dotLLM pull request, "Mamba-3 MIMO streaming decode": the state is summed
+ * over ranks, the angle is rank-free; TorchMamba README, "Models": rank-R
+ * update on a shared (N,P) state.)
+ *   X_r = W_x[r] x_t,  U_t = sum_r Bbar_r X_r^T
+ *   h <- alpha h + beta prevBx + gamma U_t,  prevBx <- U_t
+ *   y_t = sum_r W_y[r] (Cbar_r^T h) + D x_t
+ * Arguments as m3_step_decode plus W_x, W_y (nheads, rank, headdim) fp32,
+ * each NULL for all ones; B_t, C_t are (batch, nheads, rank, dstate);
+ * QkNorm/bias as in m3_bcnorm (bias (nheads, rank, dstate)).
+ * 1 <= d.rank <= 8 and headdim a multiple of 4 (else M3_ERR_UNSUPPORTED). */
+m3_status m3_mimo_step_decode(const void *x_t, const float *dt_t, const float *A,
+                              const float *lam_t, const float *theta_t, const void *B_t,
+                              const void *C_t, const float *D, const float *W_x,
+                              const float *W_y, m3_dtype dtype, const m3_bcnorm *norm,
+                              m3_dims d, float *h, float *prevBx, float *angle, void *y_t,
+                              void *stream);
+
+/* One decode step on the factored previous-input state, any rank (rank 1 with
+ * NULL W_x, W_y is the SISO step).  Instead of prevBx (dstate x headdim per
+ * lane) the caller carries the previous token's factors (TorchMamba README,
+ * "Models": the cache (angle, ssm, x_prev, b_prev)):
+ *   b_prev (batch, nheads, rank, dstate) fp32: the rotated (QkNorm/bias'd) B
+ *          of the previous token, per rank;
+ *   x_prev (batch, nheads, headdim) fp32: the previous token's x;
+ * and the previous-input term sum_r b_prev[r] (W_x[r] x_prev)^T is rebuilt on
+ * the fly, so a step reads and writes only h among the (N, P) states -- about
+ * half the bytes of m3_step_decode.  b_prev and x_prev are updated in place
+ * (to this token's rotated B and x_t); zeros start a sequence with no
+ * previous token.  All other arguments, limits and errors as
+ * m3_mimo_step_decode. */
+m3_status m3_step_decode_factored(const void *x_t, const float *dt_t, const float *A,
+                                  const float *lam_t, const float *theta_t, const void *B_t,
+                                  const void *C_t, const float *D, const float *W_x,
+                                  const float *W_y, m3_dtype dtype, const m3_bcnorm *norm,
+                                  m3_dims d, float *h, float *b_prev, float *x_prev,
+                                  float *angle, void *y_t, void *stream);
+
 /* Size in bytes of the scratch buffer built into the library for
  * m3_siso_chunked_fwd_noalloc (32 MiB). */
 #define M3_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)

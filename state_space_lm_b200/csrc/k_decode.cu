@@ -141,4 +141,187 @@ cudaError_t launch_decode(const DecodeArgs &a, m3_dtype dt, cudaStream_t s) {
     return dt == M3_BF16 ? launch_decode_t<__nv_bfloat16>(a, s) : launch_decode_t<float>(a, s);
 }
 
+// ---------------------------------------------------------------------------
+// Rank-R decode step, on the full previous-input state (prev_Bx, N x P per
+// lane) or on its factors (dotLLM pull request, "Mamba-3 MIMO streaming
+// decode": the state is summed over ranks and the angle is rank-free;
+// TorchMamba README, "Models": the cache (angle, ssm, x_prev, b_prev)):
+//   X_r = W_x[r] x_t,  U_t = sum_r Bbar_r X_r^T
+//   U_prev = prev_Bx  or  sum_r b_prev[r] (W_x[r] x_prev)^T   (factored)
+//   h <- alpha h + beta U_prev + gamma U_t
+//   y = sum_r W_y[r] (Cbar_r^T h) + D x_t
+//   prev_Bx <- U_t   or   b_prev <- Bbar, x_prev <- x_t      (factored)
+// One CTA per (b, h) lane; rank bound RT (R <= RT, the rest predicated off);
+// threads stream 4-wide rows of h (and prev_Bx).  The factored form reads and
+// writes only h, so a step moves about half the bytes of the full form.
+// ---------------------------------------------------------------------------
+template <typename T, int RT, bool FACT>
+__global__ void __launch_bounds__(256) k_decode_gen(DecodeArgs a) {
+    constexpr int VEC = 4;
+    const int64_t lane = blockIdx.x, h = lane % a.H;
+    const int P = (int)a.P, N = (int)a.N, NP2 = N / 2, R = (int)a.R;
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const T *x = static_cast<const T *>(a.x);
+    const T *Bg = static_cast<const T *>(a.B);
+    const T *Cg = static_cast<const T *>(a.C);
+    T *y = static_cast<T *>(a.y);
+
+    extern __shared__ float sm[];
+    float *Bb = sm;                 // RT x N  rotated B of this token
+    float *Cb = Bb + RT * N;        // RT x N  rotated C
+    float *Pb = Cb + RT * N;        // RT x N  b_prev (factored form)
+    float *red = Pb + RT * N;       // 32
+    float *ypart = red + 32;        // ngroups x RT x P
+
+    const float dl = a.dt[lane], lm = a.lam[lane];
+    const float al = expf(dl * a.A[h]);
+    const float be = (1.f - lm) * dl * al;
+    const float ga = lm * dl;
+
+    // QkNorm inverse RMS per rank
+    float invB[RT], invC[RT];
+#pragma unroll
+    for (int r = 0; r < RT; r++) { invB[r] = 1.f; invC[r] = 1.f; }
+    if (a.nrm.wB || a.nrm.wC) {
+#pragma unroll
+        for (int r = 0; r < RT; r++) {
+            if (r >= R) break;
+            float sb = 0.f, sc = 0.f;
+            for (int n = tid; n < N; n += nt) {
+                const float vb = ldf(Bg, (lane * R + r) * N + n), vc = ldf(Cg, (lane * R + r) * N + n);
+                sb += vb * vb;
+                sc += vc * vc;
+            }
+            sb = block_sum(sb, red);
+            __syncthreads();
+            sc = block_sum(sc, red);
+            __syncthreads();
+            invB[r] = rsqrtf(sb / N + a.nrm.eps);
+            invC[r] = rsqrtf(sc / N + a.nrm.eps);
+        }
+    }
+    if (FACT)
+        for (int k = tid; k < R * N; k += nt) Pb[k] = a.bprev[lane * R * N + k];
+    for (int j = tid; j < NP2; j += nt) {
+        const float phi = a.angle[lane * NP2 + j] + dl * a.theta[lane * NP2 + j];
+        a.angle[lane * NP2 + j] = phi;
+        float sn, cn;
+        sincosf(phi, &sn, &cn);
+#pragma unroll
+        for (int r = 0; r < RT; r++) {
+            if (r >= R) break;
+            const int64_t o = (lane * R + r) * N + 2 * j;
+            float b0 = ldf(Bg, o), b1 = ldf(Bg, o + 1), c0 = ldf(Cg, o), c1 = ldf(Cg, o + 1);
+            if (a.nrm.wB) { b0 *= invB[r] * a.nrm.wB[2 * j]; b1 *= invB[r] * a.nrm.wB[2 * j + 1]; }
+            if (a.nrm.wC) { c0 *= invC[r] * a.nrm.wC[2 * j]; c1 *= invC[r] * a.nrm.wC[2 * j + 1]; }
+            const int64_t bo = (h * R + r) * N + 2 * j;
+            if (a.nrm.biasB) { b0 += a.nrm.biasB[bo]; b1 += a.nrm.biasB[bo + 1]; }
+            if (a.nrm.biasC) { c0 += a.nrm.biasC[bo]; c1 += a.nrm.biasC[bo + 1]; }
+            Bb[r * N + 2 * j] = cn * b0 - sn * b1;
+            Bb[r * N + 2 * j + 1] = sn * b0 + cn * b1;
+            Cb[r * N + 2 * j] = cn * c0 - sn * c1;
+            Cb[r * N + 2 * j + 1] = sn * c0 + cn * c1;
+        }
+    }
+    __syncthreads();
+
+    const int PV = P / VEC;              // vectors per state row
+    const int ngroups = nt / PV;         // rows streamed concurrently
+    const int pv = tid % PV, ng = tid / PV;
+    float xv[VEC], X[RT][VEC], Xp[RT][VEC], Y[RT][VEC];
+#pragma unroll
+    for (int k = 0; k < VEC; k++) xv[k] = ldf(x, lane * P + pv * VEC + k);
+#pragma unroll
+    for (int r = 0; r < RT; r++) {
+#pragma unroll
+        for (int k = 0; k < VEC; k++) {
+            const int p = pv * VEC + k;
+            const float w = (r < R && a.Wx) ? a.Wx[(h * R + r) * P + p] : 1.f;
+            X[r][k] = r < R ? w * xv[k] : 0.f;
+            Xp[r][k] = (FACT && r < R) ? w * a.xprev[lane * P + p] : 0.f;
+            Y[r][k] = 0.f;
+        }
+    }
+    if (ng < ngroups) {
+        float4 *hp = reinterpret_cast<float4 *>(a.h + lane * (int64_t)N * P);
+        float4 *up = FACT ? nullptr : reinterpret_cast<float4 *>(a.prevBx + lane * (int64_t)N * P);
+#pragma unroll 2
+        for (int n = ng; n < N; n += ngroups) {
+            float4 hq = hp[n * PV + pv];
+            float hv[VEC] = {hq.x, hq.y, hq.z, hq.w}, uv[VEC], ut[VEC];
+            if (!FACT) {
+                const float4 uq = up[n * PV + pv];
+                uv[0] = uq.x; uv[1] = uq.y; uv[2] = uq.z; uv[3] = uq.w;
+            }
+#pragma unroll
+            for (int k = 0; k < VEC; k++) {
+                ut[k] = 0.f;
+                if (FACT) uv[k] = 0.f;
+            }
+#pragma unroll
+            for (int r = 0; r < RT; r++) {
+                const float bn = Bb[r * N + n], pn = FACT ? Pb[r * N + n] : 0.f;
+#pragma unroll
+                for (int k = 0; k < VEC; k++) {
+                    ut[k] = fmaf(bn, X[r][k], ut[k]);
+                    if (FACT) uv[k] = fmaf(pn, Xp[r][k], uv[k]);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < VEC; k++) hv[k] = al * hv[k] + be * uv[k] + ga * ut[k];
+#pragma unroll
+            for (int r = 0; r < RT; r++) {
+                const float cn = Cb[r * N + n];
+#pragma unroll
+                for (int k = 0; k < VEC; k++) Y[r][k] = fmaf(cn, hv[k], Y[r][k]);
+            }
+            hp[n * PV + pv] = make_float4(hv[0], hv[1], hv[2], hv[3]);
+            if (!FACT) up[n * PV + pv] = make_float4(ut[0], ut[1], ut[2], ut[3]);
+        }
+#pragma unroll
+        for (int r = 0; r < RT; r++)
+#pragma unroll
+            for (int k = 0; k < VEC; k++) ypart[(ng * RT + r) * P + pv * VEC + k] = Y[r][k];
+    }
+    __syncthreads();
+    for (int p = tid; p < P; p += nt) {
+        float s = 0.f;
+        for (int r = 0; r < R; r++) {
+            float yr = 0.f;
+            for (int g = 0; g < ngroups; g++) yr += ypart[(g * RT + r) * P + p];
+            s += (a.Wy ? a.Wy[(h * R + r) * P + p] : 1.f) * yr;
+        }
+        const float xp_new = ldf(x, lane * P + p);
+        stf(y, lane * P + p, s + a.D[h] * xp_new);
+        if (FACT) a.xprev[lane * P + p] = xp_new;
+    }
+    if (FACT)
+        for (int k = tid; k < R * N; k += nt) a.bprev[lane * R * N + k] = Bb[k];
+}
+
+template <typename T, int RT>
+static cudaError_t launch_decode_gen_rt(const DecodeArgs &a, bool factored, cudaStream_t s) {
+    const int threads = 256;
+    const int ngroups = threads / (int)(a.P / 4);
+    const size_t smem = sizeof(float) * (3 * RT * a.N + 32 + (size_t)ngroups * RT * a.P);
+    if (factored) k_decode_gen<T, RT, true><<<(unsigned)(a.Bt * a.H), threads, smem, s>>>(a);
+    else k_decode_gen<T, RT, false><<<(unsigned)(a.Bt * a.H), threads, smem, s>>>(a);
+    count_launch();
+    return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_decode_gen_t(const DecodeArgs &a, bool factored, cudaStream_t s) {
+    if (a.R <= 1) return launch_decode_gen_rt<T, 1>(a, factored, s);
+    if (a.R <= 2) return launch_decode_gen_rt<T, 2>(a, factored, s);
+    if (a.R <= 4) return launch_decode_gen_rt<T, 4>(a, factored, s);
+    return launch_decode_gen_rt<T, 8>(a, factored, s);
+}
+
+cudaError_t launch_decode_gen(const DecodeArgs &a, m3_dtype dt, bool factored, cudaStream_t s) {
+    if (a.Bt * a.H == 0) return cudaSuccess;
+    return dt == M3_BF16 ? launch_decode_gen_t<__nv_bfloat16>(a, factored, s)
+                         : launch_decode_gen_t<float>(a, factored, s);
+}
+
 }  // namespace m3

@@ -222,4 +222,52 @@ m3_status m3_step_decode(const void *x_t, const float *dt_t, const float *A, con
     return launched(launch_decode(a, dtype, (cudaStream_t)stream));
 }
 
+namespace {
+// Shared validation of the rank-R decode entry points.
+m3_status decode_gen(const void *x_t, const float *dt_t, const float *A, const float *lam_t, const float *theta_t,
+                     const void *B_t, const void *C_t, const float *D, const float *W_x, const float *W_y,
+                     m3_dtype dtype, const m3_bcnorm *norm, m3_dims d, float *h, float *prevBx, float *b_prev,
+                     float *x_prev, float *angle, void *y_t, void *stream, bool factored) {
+    m3_status st;
+    if ((st = check_dtype(dtype)) != M3_OK) return st;
+    if ((st = check_core_dims(d, false)) != M3_OK) return st;
+    if (d.rank < 1) return M3_ERR_INVALID_ARG;
+    if (d.rank > kMaxRank || d.headdim % 4) return M3_ERR_UNSUPPORTED;
+    M3_REQ(A); M3_REQ(D);
+    M3_OPT(W_x); M3_OPT(W_y);
+    if (d.batch > 0) {
+        M3_REQ(x_t); M3_REQ(dt_t); M3_REQ(lam_t); M3_REQ(theta_t); M3_REQ(B_t); M3_REQ(C_t);
+        M3_REQ(h); M3_REQ(angle); M3_REQ(y_t);
+        if (factored) { M3_REQ(b_prev); M3_REQ(x_prev); }
+        else M3_REQ(prevBx);
+    }
+    NormArgs nrm;
+    if ((st = read_norm(norm, nrm)) != M3_OK) return st;
+    if (d.batch == 0) return M3_OK;
+    DecodeArgs a;
+    a.x = x_t; a.B = B_t; a.C = C_t; a.dt = dt_t; a.A = A; a.lam = lam_t; a.theta = theta_t; a.D = D;
+    a.nrm = nrm; a.h = h; a.prevBx = prevBx; a.angle = angle; a.y = y_t;
+    a.Bt = d.batch; a.H = d.nheads; a.P = d.headdim; a.N = d.dstate;
+    a.Wx = W_x; a.Wy = W_y; a.bprev = b_prev; a.xprev = x_prev; a.R = d.rank;
+    return launched(launch_decode_gen(a, dtype, factored, (cudaStream_t)stream));
+}
+}  // namespace
+
+m3_status m3_mimo_step_decode(const void *x_t, const float *dt_t, const float *A, const float *lam_t,
+                              const float *theta_t, const void *B_t, const void *C_t, const float *D,
+                              const float *W_x, const float *W_y, m3_dtype dtype, const m3_bcnorm *norm,
+                              m3_dims d, float *h, float *prevBx, float *angle, void *y_t, void *stream) {
+    return decode_gen(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, W_x, W_y, dtype, norm, d, h, prevBx, nullptr,
+                      nullptr, angle, y_t, stream, false);
+}
+
+m3_status m3_step_decode_factored(const void *x_t, const float *dt_t, const float *A, const float *lam_t,
+                                  const float *theta_t, const void *B_t, const void *C_t, const float *D,
+                                  const float *W_x, const float *W_y, m3_dtype dtype, const m3_bcnorm *norm,
+                                  m3_dims d, float *h, float *b_prev, float *x_prev, float *angle, void *y_t,
+                                  void *stream) {
+    return decode_gen(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, W_x, W_y, dtype, norm, d, h, nullptr, b_prev,
+                      x_prev, angle, y_t, stream, true);
+}
+
 }  // extern "C"

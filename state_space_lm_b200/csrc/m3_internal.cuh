@@ -53,6 +53,10 @@ struct DecodeArgs {
     float *h, *prevBx, *angle;
     void *y;
     int64_t Bt, H, P, N;
+    // rank-R and factored-state decode (k_decode_gen)
+    const float *Wx = nullptr, *Wy = nullptr;   // (H, R, P), NULL = ones
+    float *bprev = nullptr, *xprev = nullptr;   // factored previous-input state
+    int64_t R = 1;
 };
 
 struct RopeArgs {
@@ -73,6 +77,8 @@ cudaError_t launch_scan_simt(const ScanArgs &a, m3_dtype dt, cudaStream_t s);
 size_t scan_simt_smem_bytes(int64_t P, int64_t N, int64_t R, int Q);
 int scan_simt_chunk(int64_t P, int64_t N, int64_t R, int64_t chunk);
 cudaError_t launch_decode(const DecodeArgs &a, m3_dtype dt, cudaStream_t s);
+// rank R (1..8), full (prevBx) or factored (bprev, xprev) previous-input state; headdim % 4 == 0
+cudaError_t launch_decode_gen(const DecodeArgs &a, m3_dtype dt, bool factored, cudaStream_t s);
 // tensor-core SISO scan (bf16, headdim 64, dState 128, chunk 64)
 bool scan_tc_supported(const ScanArgs &a, m3_dtype dt);
 cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s);

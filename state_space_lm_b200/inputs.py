@@ -38,6 +38,12 @@ CONFIGS = {
             headdim=64, dstate=128, rank=1, chunk=128, dtype="bf16", dt_shift=-4.0),
     4: dict(name="decode_512xh16_p64_n128", batch=512, seqlen=256, nheads=16, headdim=64,
             dstate=128, rank=1, chunk=64, dtype="bf16", dt_shift=-2.0, steps=1024),
+    # decode on the factored previous-input state (b_prev, x_prev), SISO and rank 4
+    5: dict(name="decode_factored_512xh16_p64_n128", batch=512, seqlen=256, nheads=16, headdim=64,
+            dstate=128, rank=1, chunk=64, dtype="bf16", dt_shift=-2.0, steps=1024, state="factored"),
+    6: dict(name="decode_factored_mimo_r4_512xh16_p64_n128", batch=512, seqlen=256, nheads=16,
+            headdim=64, dstate=128, rank=4, chunk=64, dtype="bf16", dt_shift=-2.0, steps=1024,
+            state="factored"),
 }
 
 _DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}
@@ -101,26 +107,27 @@ def scan_inputs(batch, seqlen, nheads, headdim, dstate, rank=1, dtype="bf16",
 
 
 def decode_step_inputs(generator, batch, nheads, headdim, dstate, dtype="bf16",
-                       dt_shift=-2.0):
-    """Per-token inputs of one SISO decode step, drawn from ``generator``:
+                       dt_shift=-2.0, rank=1, rank_axis=False):
+    """Per-token inputs of one decode step, drawn from ``generator``:
     x_t (Bt,H,P), dt_t (Bt,H), lam_t (Bt,H), theta_t (Bt,H,N/2), B_t and C_t
-    (Bt,H,N)."""
+    (Bt,H,N), or (Bt,H,R,N) when rank > 1 or rank_axis."""
     g = generator
     sdt = _DTYPES[dtype]
     Bt, H, P, N = batch, nheads, headdim, dstate
+    bc = (Bt, H, rank, N) if (rank > 1 or rank_axis) else (Bt, H, N)
     out = {}
     out["x"] = _normal(g, (Bt, H, P)).to(sdt)
     out["dt"] = torch.nn.functional.softplus(_normal(g, (Bt, H)) + dt_shift).float()
     out["lam"] = torch.sigmoid(_normal(g, (Bt, H))).float()
     out["theta"] = _uniform(g, (Bt, H, N // 2), -math.pi / 8, math.pi / 8).float()
-    out["B"] = (_normal(g, (Bt, H, N)) / math.sqrt(N)).to(sdt)
-    out["C"] = (_normal(g, (Bt, H, N)) / math.sqrt(N)).to(sdt)
+    out["B"] = (_normal(g, bc) / math.sqrt(N)).to(sdt)
+    out["C"] = (_normal(g, bc) / math.sqrt(N)).to(sdt)
     return out
 
 
 def config_inputs(idx, seed=None, **overrides):
-    """Inputs of workload ``idx`` (0-3: one chunked-scan call; 4: the prefill of
-    the decode workload -- its steps come from ``decode_step_inputs`` with the
+    """Inputs of workload ``idx`` (0-3: one chunked-scan call; 4-6: the prefill
+    of a decode workload -- its steps come from ``decode_step_inputs`` with the
     returned generator)."""
     c = dict(CONFIGS[idx])
     c.update(overrides)

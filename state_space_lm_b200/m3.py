@@ -22,7 +22,8 @@ _DTYPE = {torch.float32: M3_F32, torch.bfloat16: M3_BF16}
 ABI_FUNCTIONS = (
     "m3_get_limits", "m3_discretize", "m3_rope_bc", "m3_siso_chunked_fwd",
     "m3_mimo_chunked_fwd", "m3_step_decode", "m3_workspace_bytes", "m3_status_string",
-    "m3_launch_count", "m3_device_error", "m3_siso_chunked_fwd_noalloc",
+    "m3_launch_count", "m3_device_error", "m3_siso_chunked_fwd_noalloc", "m3_mimo_step_decode",
+    "m3_step_decode_factored",
 )
 
 
@@ -93,6 +94,12 @@ def lib():
     L.m3_step_decode.restype = ctypes.c_int
     L.m3_step_decode.argtypes = [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int,
                                  ctypes.POINTER(BcNorm), Dims, _VP, _VP, _VP, _VP, _VP]
+    for fn in (L.m3_mimo_step_decode, L.m3_step_decode_factored):
+        fn.restype = ctypes.c_int
+    L.m3_mimo_step_decode.argtypes = [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int,
+                                      ctypes.POINTER(BcNorm), Dims, _VP, _VP, _VP, _VP, _VP]
+    L.m3_step_decode_factored.argtypes = [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int,
+                                          ctypes.POINTER(BcNorm), Dims, _VP, _VP, _VP, _VP, _VP, _VP]
     _lib = L
     return L
 
@@ -246,4 +253,38 @@ def step_decode(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, prevBx, angle, nor
                                 _ptr(B_t), _ptr(C_t), _ptr(D), _DTYPE[x_t.dtype], nptr, d, _ptr(h),
                                 _ptr(prevBx), _ptr(angle), _ptr(y), _stream(stream)),
            "m3_step_decode")
+    return y
+
+
+def mimo_step_decode(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, prevBx, angle, W_x=None, W_y=None,
+                     norm=None, y_out=None, stream=None):
+    """S5 for rank R: one decode step on the full previous-input state.  B_t, C_t
+    (Bt,H,R,N); h, prevBx, angle updated in place; returns y_t (Bt,H,P)."""
+    Bt, H, P = x_t.shape
+    R, N = B_t.shape[-2], B_t.shape[-1]
+    y = torch.empty_like(x_t) if y_out is None else y_out
+    d = Dims(Bt, 1, H, P, N, R, 1)
+    nptr, keep = _norm(norm)
+    _check(lib().m3_mimo_step_decode(_ptr(x_t), _ptr(dt_t), _ptr(A), _ptr(lam_t), _ptr(theta_t), _ptr(B_t),
+                                     _ptr(C_t), _ptr(D), _ptr(W_x), _ptr(W_y), _DTYPE[x_t.dtype], nptr, d,
+                                     _ptr(h), _ptr(prevBx), _ptr(angle), _ptr(y), _stream(stream)),
+           "m3_mimo_step_decode")
+    return y
+
+
+def step_decode_factored(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, b_prev, x_prev, angle, W_x=None,
+                         W_y=None, norm=None, y_out=None, stream=None):
+    """One decode step on the factored previous-input state (any rank; B_t, C_t
+    (Bt,H,R,N)).  h, b_prev (Bt,H,R,N), x_prev (Bt,H,P) and angle are updated in
+    place; returns y_t (Bt,H,P)."""
+    Bt, H, P = x_t.shape
+    R, N = B_t.shape[-2], B_t.shape[-1]
+    y = torch.empty_like(x_t) if y_out is None else y_out
+    d = Dims(Bt, 1, H, P, N, R, 1)
+    nptr, keep = _norm(norm)
+    _check(lib().m3_step_decode_factored(_ptr(x_t), _ptr(dt_t), _ptr(A), _ptr(lam_t), _ptr(theta_t),
+                                         _ptr(B_t), _ptr(C_t), _ptr(D), _ptr(W_x), _ptr(W_y),
+                                         _DTYPE[x_t.dtype], nptr, d, _ptr(h), _ptr(b_prev), _ptr(x_prev),
+                                         _ptr(angle), _ptr(y), _stream(stream)),
+           "m3_step_decode_factored")
     return y

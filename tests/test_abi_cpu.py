@@ -117,6 +117,28 @@ def test_decode_rope_discretize_validation(L):
     assert L.m3_discretize(FAKE, FAKE, FAKE, dims(nheads=0), FAKE, FAKE, FAKE, None) == m3.M3_ERR_INVALID_ARG
 
 
+def test_rank_decode_validation(L):
+    def full(d, Wx=None, h=FAKE, u=FAKE, dtype=m3.M3_BF16):
+        return L.m3_mimo_step_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, Wx, None, dtype, None, d,
+                                     h, u, FAKE, FAKE, None)
+
+    def fact(d, bp=FAKE, xp=FAKE, Wy=None):
+        return L.m3_step_decode_factored(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, Wy, m3.M3_BF16,
+                                         None, d, FAKE, bp, xp, FAKE, FAKE, None)
+
+    assert full(dims(rank=0)) == m3.M3_ERR_INVALID_ARG
+    assert full(dims(rank=9)) == m3.M3_ERR_UNSUPPORTED
+    assert full(dims(rank=2, headdim=6)) == m3.M3_ERR_UNSUPPORTED     # rows are streamed 4-wide
+    assert full(dims(rank=2), Wx=MIS) == m3.M3_ERR_INVALID_ARG
+    assert full(dims(rank=2), u=None) == m3.M3_ERR_INVALID_ARG         # the full state needs prev_Bx
+    assert full(dims(rank=2), h=MIS) == m3.M3_ERR_INVALID_ARG
+    assert full(dims(rank=2), dtype=5) == m3.M3_ERR_INVALID_ARG
+    assert fact(dims(dstate=5)) == m3.M3_ERR_INVALID_ARG
+    assert fact(dims(rank=1), bp=None) == m3.M3_ERR_INVALID_ARG        # the factored state needs b_prev
+    assert fact(dims(rank=3), xp=MIS) == m3.M3_ERR_INVALID_ARG
+    assert fact(dims(rank=3), Wy=MIS) == m3.M3_ERR_INVALID_ARG
+
+
 def test_workspace_query(L):
     for which in (m3.M3_WS_SISO, m3.M3_WS_MIMO):
         n = m3.workspace_bytes(which, dims(), m3.M3_BF16)

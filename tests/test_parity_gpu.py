@@ -308,6 +308,120 @@ def test_decode_norm_bias():
 
 
 # ----------------------------------------------------------------------------
+# S5 for rank R, and decode on the factored previous-input state
+# ----------------------------------------------------------------------------
+def _mimo_w(g, H, R, P):
+    w = lambda: (1.0 + 0.3 * torch.randn(H, R, P, generator=g, dtype=torch.float64)).float()
+    return w(), w()
+
+
+def _dec_step(st, d, R):
+    """Per-token device inputs (B, C with the rank axis) of one decode step."""
+    ds = cuda(st)
+    return (ds["x"], ds["dt"], d["A"], ds["lam"], ds["theta"], ds["B"], ds["C"], d["D"])
+
+
+def _dec_step_f64(st, inp):
+    return (to_f64(st["x"]), to_f64(st["dt"]), to_f64(inp["A"]), to_f64(st["lam"]), to_f64(st["theta"]),
+            to_f64(st["B"]), to_f64(st["C"]), to_f64(inp["D"]))
+
+
+@pytest.mark.parametrize("dtype", [FP32, BF16])
+@pytest.mark.parametrize("R", [2, 4])
+def test_mimo_decode_steps(dtype, R):
+    Bt, H, P, N, steps = 3, 2, 16, 8, 6
+    inp = gen.scan_inputs(Bt, 1, H, P, N, rank=R, dtype=dtype, seed=90 + R)
+    d = cuda(inp)
+    g = torch.Generator().manual_seed(190 + R)
+    Wx, Wy = _mimo_w(g, H, R, P)
+    h0, u0, a0 = _states(Bt, H, N, P, 91 + R)
+    h, u, a = h0.cuda(), u0.cuda(), a0.cuda()
+    rh, ru, ra = to_f64(h0), to_f64(u0), to_f64(a0)
+    tol = _tol(dtype)
+    for _ in range(steps):
+        st = gen.decode_step_inputs(g, Bt, H, P, N, dtype=dtype, rank=R)
+        y = m3.mimo_step_decode(*_dec_step(st, d, R), h, u, a, W_x=Wx.cuda(), W_y=Wy.cuda())
+        ry, rh, ru, ra = oracle.mimo_step_decode(*_dec_step_f64(st, inp), rh, ru, ra, Wx=to_f64(Wx),
+                                                 Wy=to_f64(Wy))
+        assert relerr(y, ry) <= tol
+    assert relerr(h, rh) <= tol and relerr(u, ru) <= tol and relerr(a, ra) <= 1e-5
+
+
+@pytest.mark.parametrize("dtype", [FP32, BF16])
+@pytest.mark.parametrize("R", [1, 3, 4])
+def test_factored_decode_steps(dtype, R):
+    Bt, H, P, N, steps = 3, 2, 16, 8, 6
+    inp = gen.scan_inputs(Bt, 1, H, P, N, rank=max(R, 2), dtype=dtype, seed=95 + R)
+    d = cuda(inp)
+    g = torch.Generator().manual_seed(195 + R)
+    Wx, Wy = _mimo_w(g, H, R, P)
+    h0, _, a0 = _states(Bt, H, N, P, 96 + R)
+    bp0 = (torch.randn(Bt, H, R, N, generator=g, dtype=torch.float64) / N ** 0.5).float()
+    xp0 = torch.randn(Bt, H, P, generator=g, dtype=torch.float64).float()
+    h, bp, xp, a = h0.cuda(), bp0.cuda(), xp0.cuda(), a0.cuda()
+    rh, rbp, rxp, ra = to_f64(h0), to_f64(bp0), to_f64(xp0), to_f64(a0)
+    tol = _tol(dtype)
+    for _ in range(steps):
+        st = gen.decode_step_inputs(g, Bt, H, P, N, dtype=dtype, rank=R, rank_axis=True)
+        y = m3.step_decode_factored(*_dec_step(st, d, R), h, bp, xp, a, W_x=Wx.cuda(), W_y=Wy.cuda())
+        ry, rh, rbp, rxp, ra = oracle.step_decode_factored(*_dec_step_f64(st, inp), rh, rbp, rxp, ra,
+                                                           Wx=to_f64(Wx), Wy=to_f64(Wy))
+        assert relerr(y, ry) <= tol
+    assert relerr(h, rh) <= tol and relerr(bp, rbp) <= tol and relerr(a, ra) <= 1e-5
+    assert relerr(xp, rxp) == 0.0          # x_prev is x_t itself
+
+
+def test_factored_decode_norm_bias():
+    Bt, H, P, N, R = 2, 2, 8, 8, 2
+    inp = gen.scan_inputs(Bt, 1, H, P, N, rank=R, dtype=FP32, seed=98, bcnorm=True)
+    g = torch.Generator().manual_seed(198)
+    Wx, Wy = _mimo_w(g, H, R, P)
+    h0, _, a0 = _states(Bt, H, N, P, 99)
+    bp0 = torch.randn(Bt, H, R, N, generator=g, dtype=torch.float64).float()
+    xp0 = torch.randn(Bt, H, P, generator=g, dtype=torch.float64).float()
+    d = cuda(inp)
+    h, bp, xp, a = h0.cuda(), bp0.cuda(), xp0.cuda(), a0.cuda()
+    tok = lambda k: d[k][:, 0].contiguous()
+    y = m3.step_decode_factored(tok("x"), tok("dt"), d["A"], tok("lam"), tok("theta"), tok("B"), tok("C"), d["D"],
+                                h, bp, xp, a, W_x=Wx.cuda(), W_y=Wy.cuda(), norm=norm_dev(inp))
+    f = lambda k: to_f64(inp[k][:, 0])
+    ry, rh, rbp, rxp, ra = oracle.step_decode_factored(f("x"), f("dt"), to_f64(inp["A"]), f("lam"), f("theta"),
+                                                       f("B"), f("C"), to_f64(inp["D"]), to_f64(h0), to_f64(bp0),
+                                                       to_f64(xp0), to_f64(a0), Wx=to_f64(Wx), Wy=to_f64(Wy),
+                                                       norm=norm_f64(inp))
+    for got, ref in ((y, ry), (h, rh), (bp, rbp), (a, ra)):
+        assert relerr(got, ref) <= 1e-5
+
+
+@pytest.mark.parametrize("R", [1, 2])
+def test_prefill_then_factored_decode(R):
+    """A chunked prefill on the GPU, its last token's rotated B (m3_rope_bc)
+    and x as the factored state, then decode steps: equal to the one-shot
+    oracle scan over prefill + decoded tokens."""
+    Bt, H, P, N, T0, steps = 2, 3, 16, 8, 11, 5
+    T = T0 + steps
+    full = gen.scan_inputs(Bt, T, H, P, N, rank=R, dtype=FP32, seed=101 + R, mimo_weights=True)
+    pre = {k: (v[:, :T0].contiguous() if k in ("x", "dt", "lam", "theta", "B", "C") else v)
+           for k, v in full.items() if isinstance(v, torch.Tensor)}
+    d = cuda(pre)
+    _, h, _, a = m3.mimo_chunked_fwd(d["x"], d["dt"], d["A"], d["lam"], d["theta"], d["B"], d["C"], d["D"], 4,
+                                     W_x=d["Wx"], W_y=d["Wy"])
+    Br, _, _ = m3.rope_bc(d["B"], d["C"], d["theta"], d["dt"])
+    bp = Br[:, T0 - 1].float().contiguous()
+    xp = d["x"][:, T0 - 1].float().contiguous()
+    ys = []
+    fd = cuda(full)
+    for t in range(T0, T):
+        tk = lambda k: fd[k][:, t].contiguous()
+        ys.append(m3.step_decode_factored(tk("x"), tk("dt"), fd["A"], tk("lam"), tk("theta"), tk("B"), tk("C"),
+                                          fd["D"], h, bp, xp, a, W_x=fd["Wx"], W_y=fd["Wy"]))
+    ref = oracle.mimo_loop(**{k: to_f64(full[k]) for k in ("x", "dt", "A", "lam", "theta", "B", "C", "D")},
+                           Wx=to_f64(full["Wx"]), Wy=to_f64(full["Wy"]))
+    assert relerr(torch.stack(ys, 1), ref[0][:, T0:]) <= 1e-5
+    assert relerr(h, ref[1]) <= 1e-5 and relerr(a, ref[3]) <= 1e-5
+
+
+# ----------------------------------------------------------------------------
 # full-size workloads, sampled lanes (the launch configuration the bench times)
 # ----------------------------------------------------------------------------
 def _full_scan(idx):
@@ -373,4 +487,44 @@ def test_full_size_decode_sampled_lanes():
         assert relerr(ys[li_], ry[0, T0:, 0]) <= 2e-2
         assert relerr(h[b, hh], rh[0, 0]) <= 2e-2
         assert relerr(u[b, hh], ru[0, 0]) <= 2e-2
+        assert relerr(a[b, hh], ra[0, 0]) <= 1e-5
+
+
+def test_full_size_factored_decode_sampled_lanes():
+    """Decode workload shape, factored state: prefill, b_prev from the prefill's
+    last rotated B (m3_rope_bc), then 64 steps; sampled lanes against the
+    oracle's one-shot loop over prefill + steps."""
+    c = gen.CONFIGS[4]
+    Bt, H, P, N = c["batch"], c["nheads"], c["headdim"], c["dstate"]
+    inp = gen.config_inputs(4)
+    d = cuda(inp)
+    T0 = c["seqlen"]
+    _, h, _, a = m3.siso_chunked_fwd(d["x"], d["dt"], d["A"], d["lam"], d["theta"], d["B"], d["C"], d["D"],
+                                     c["chunk"])
+    Br, _, _ = m3.rope_bc(d["B"], d["C"], d["theta"], d["dt"])
+    bp = Br[:, T0 - 1, :, None].float().contiguous()          # (Bt, H, 1, N)
+    xp = d["x"][:, T0 - 1].float().contiguous()
+    lanes = sample_lanes(Bt, H)
+    g = inp["generator"]
+    seq = {k: [] for k in ("x", "dt", "lam", "theta", "B", "C")}
+    ys = []
+    for s in range(64):
+        st = gen.decode_step_inputs(g, Bt, H, P, N, rank_axis=True)
+        ds = cuda(st)
+        y = m3.step_decode_factored(ds["x"], ds["dt"], d["A"], ds["lam"], ds["theta"], ds["B"], ds["C"], d["D"],
+                                    h, bp, xp, a)
+        ys.append(torch.stack([y[b, hh] for (b, hh) in lanes]).cpu())
+        for k in seq:
+            v = st[k][:, :, 0] if k in ("B", "C") else st[k]
+            seq[k].append(torch.stack([v[b, hh] for (b, hh) in lanes]))
+    torch.cuda.synchronize()
+    ys = torch.stack(ys, 1)
+    for li_, (b, hh) in enumerate(lanes):
+        li = lane_inputs(inp, b, hh)
+        for k in seq:
+            steps = torch.stack([v[li_] for v in seq[k]])[None, :, None]
+            li[k] = np.concatenate([li[k], to_f64(steps)], axis=1)
+        ry, rh, _, ra = oracle.siso_loop(**li)
+        assert relerr(ys[li_], ry[0, T0:, 0]) <= 2e-2
+        assert relerr(h[b, hh], rh[0, 0]) <= 2e-2
         assert relerr(a[b, hh], ra[0, 0]) <= 1e-5
