@@ -200,6 +200,10 @@ __global__ void __launch_bounds__(256) k_decode_gen(DecodeArgs a) {
             invC[r] = rsqrtf(sc / N + a.nrm.eps);
         }
     }
+    const int PV = P / VEC;              // vectors per state row
+    const int ngroups = nt / PV;         // rows streamed concurrently
+    const int pv = tid % PV, ng = tid / PV;
+    float4 *hp = reinterpret_cast<float4 *>(a.h + lane * (int64_t)N * P);
     if (FACT)
         for (int k = tid; k < R * N; k += nt) Pb[k] = a.bprev[lane * R * N + k];
     for (int j = tid; j < NP2; j += nt) {
@@ -225,29 +229,35 @@ __global__ void __launch_bounds__(256) k_decode_gen(DecodeArgs a) {
     }
     __syncthreads();
 
-    const int PV = P / VEC;              // vectors per state row
-    const int ngroups = nt / PV;         // rows streamed concurrently
-    const int pv = tid % PV, ng = tid / PV;
-    float xv[VEC], X[RT][VEC], Xp[RT][VEC], Y[RT][VEC];
+    // Small ranks keep X_r = W_x[r] x (and W_x[r] x_prev) per rank; ranks 4
+    // and 8 keep W_x[r] alone and scale the rank sums by x (x_prev) after, which
+    // holds half the registers:  U_t[n][p] = x[p] sum_r Bbar_r[n] W_x[r][p].
+    constexpr bool WF = RT >= 4;
+    constexpr int RX = WF ? 1 : RT;                 // per-rank products kept
+    float xv[VEC], xq[VEC], W[RT][VEC], X[RX][VEC], Xp[RX][VEC], Y[RT][VEC];
 #pragma unroll
-    for (int k = 0; k < VEC; k++) xv[k] = ldf(x, lane * P + pv * VEC + k);
+    for (int k = 0; k < VEC; k++) {
+        xv[k] = ldf(x, lane * P + pv * VEC + k);
+        xq[k] = FACT ? a.xprev[lane * P + pv * VEC + k] : 0.f;
+    }
 #pragma unroll
     for (int r = 0; r < RT; r++) {
 #pragma unroll
         for (int k = 0; k < VEC; k++) {
             const int p = pv * VEC + k;
-            const float w = (r < R && a.Wx) ? a.Wx[(h * R + r) * P + p] : 1.f;
-            X[r][k] = r < R ? w * xv[k] : 0.f;
-            Xp[r][k] = (FACT && r < R) ? w * a.xprev[lane * P + p] : 0.f;
+            W[r][k] = r < R ? (a.Wx ? a.Wx[(h * R + r) * P + p] : 1.f) : 0.f;
             Y[r][k] = 0.f;
+            if (!WF) {
+                X[r < RX ? r : 0][k] = W[r][k] * xv[k];
+                Xp[r < RX ? r : 0][k] = W[r][k] * xq[k];
+            }
         }
     }
     if (ng < ngroups) {
-        float4 *hp = reinterpret_cast<float4 *>(a.h + lane * (int64_t)N * P);
         float4 *up = FACT ? nullptr : reinterpret_cast<float4 *>(a.prevBx + lane * (int64_t)N * P);
 #pragma unroll 2
         for (int n = ng; n < N; n += ngroups) {
-            float4 hq = hp[n * PV + pv];
+            const float4 hq = hp[n * PV + pv];
             float hv[VEC] = {hq.x, hq.y, hq.z, hq.w}, uv[VEC], ut[VEC];
             if (!FACT) {
                 const float4 uq = up[n * PV + pv];
@@ -263,8 +273,15 @@ __global__ void __launch_bounds__(256) k_decode_gen(DecodeArgs a) {
                 const float bn = Bb[r * N + n], pn = FACT ? Pb[r * N + n] : 0.f;
 #pragma unroll
                 for (int k = 0; k < VEC; k++) {
-                    ut[k] = fmaf(bn, X[r][k], ut[k]);
-                    if (FACT) uv[k] = fmaf(pn, Xp[r][k], uv[k]);
+                    ut[k] = fmaf(bn, WF ? W[r][k] : X[r < RX ? r : 0][k], ut[k]);
+                    if (FACT) uv[k] = fmaf(pn, WF ? W[r][k] : Xp[r < RX ? r : 0][k], uv[k]);
+                }
+            }
+            if (WF) {
+#pragma unroll
+                for (int k = 0; k < VEC; k++) {
+                    ut[k] *= xv[k];
+                    if (FACT) uv[k] *= xq[k];
                 }
             }
 #pragma unroll
