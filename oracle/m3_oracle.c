@@ -31,9 +31,10 @@
  *   (H,R,P);  QkNorm gain of shape (N), bias of shape (H,R,N).
  *
  * Layouts (row-major, last index fastest):
- *   x, y (Bt,T,H,P); dt, lam (Bt,T,H); A, D (H); theta (Bt,T,H,N/2);
- *   B, C (Bt,T,H,R,N) with R = 1 for SISO; W_x, W_y (H,R,P);
- *   h, prev_Bx (Bt,H,N,P); angle (Bt,H,N/2).
+ *   x, y (Bt,T,H,P); dt, lam (Bt,T,H); A, D (H); theta (Bt,T,H,K);
+ *   B, C (Bt,T,G,R,N) with R = 1 for SISO (G = H unless grouped);
+ *   W_x, W_y (H,R,P); h, prev_Bx (Bt,H,N,P); angle (Bt,H,K);
+ *   K = N/2 unless partial RoPE.
  *
  * Every function returns 0 on success, -1 on a bad argument.
  */
@@ -45,7 +46,23 @@
 
 typedef struct {
     long batch, seqlen, nheads, headdim, dstate, rank;
+    long ngroups;    /* B/C groups G (H % G == 0); 0 means G = H            */
+    long rope_pairs; /* pairs (2i, 2i+1), i < K, that rotate; 0 means N/2  */
 } m3o_dims;
+
+/* Grouped B/C (torchmamba "Models": n_groups, H % G == 0) and partial RoPE
+ * (dotLLM pull request, real-checkpoint run: num_rope_angles = 32 of
+ * d_state 128, rope_fraction 0.5).  Head h reads the B/C row of group
+ * h / (H / G); only the first K pairs rotate (theta and the angle then hold K
+ * values per head), the others pass through unrotated. */
+static long n_groups(m3o_dims d) { return d.ngroups > 0 ? d.ngroups : d.nheads; }
+static long n_pairs(m3o_dims d) { return d.rope_pairs > 0 ? d.rope_pairs : d.dstate / 2; }
+/* offset of the B/C row (rank r) read by head h at (b, t) */
+static long bc_off(m3o_dims d, long b, long t, long h, long r)
+{
+    long G = n_groups(d), R = d.rank < 1 ? 1 : d.rank;
+    return (((b * d.seqlen + t) * G + h / (d.nheads / G)) * R + r) * d.dstate;
+}
 
 typedef struct {
     const double *normw_B, *normw_C; /* (N) or NULL: QkNorm off          */
@@ -91,15 +108,17 @@ static void bc_prepare(const double *src, long N, const double *w,
         for (long n = 0; n < N; n++) dst[n] += bias[n];
 }
 
-/* Rotate adjacent pairs (2i, 2i+1) of v by the angles phi[i]. */
-static void rotate_pairs(const double *v, const double *phi, long N, double *out)
+/* Rotate adjacent pairs (2i, 2i+1), i < K, of v by the angles phi[i]; the
+ * remaining elements pass through. */
+static void rotate_pairs(const double *v, const double *phi, long K, long N, double *out)
 {
-    for (long i = 0; i < N / 2; i++) {
+    for (long i = 0; i < K; i++) {
         double c = cos(phi[i]), s = sin(phi[i]);
         double v0 = v[2 * i], v1 = v[2 * i + 1];
         out[2 * i] = c * v0 - s * v1;
         out[2 * i + 1] = s * v0 + c * v1;
     }
+    for (long n = 2 * K; n < N; n++) out[n] = v[n];
 }
 
 /* ------------------------------------------------------------------------ */
@@ -115,29 +134,32 @@ int m3o_rope_bc(const double *B, const double *C, const double *theta,
     long R = d.rank < 1 ? 1 : d.rank;
     if (!B || !C || !theta || !dt || !B_rot || !C_rot) return -1;
     if (N <= 0 || (N & 1)) return -1;
-    double *phi = (double *)malloc(sizeof(double) * (N / 2));
+    long G = n_groups(d), K = n_pairs(d);
+    if (H % G || K < 1 || K > N / 2) return -1;
+    double *phi = (double *)malloc(sizeof(double) * K);
     double *tmp = (double *)malloc(sizeof(double) * N);
     for (long b = 0; b < Bt; b++)
         for (long h = 0; h < H; h++) {
-            for (long i = 0; i < N / 2; i++)
-                phi[i] = angle0 ? angle0[(b * H + h) * (N / 2) + i] : 0.0;
+            for (long i = 0; i < K; i++)
+                phi[i] = angle0 ? angle0[(b * H + h) * K + i] : 0.0;
             for (long t = 0; t < T; t++) {
                 long bth = (b * T + t) * H + h;
-                for (long i = 0; i < N / 2; i++)
-                    phi[i] += dt[bth] * theta[bth * (N / 2) + i];
+                for (long i = 0; i < K; i++)
+                    phi[i] += dt[bth] * theta[bth * K + i];
                 for (long r = 0; r < R; r++) {
-                    long off = (bth * R + r) * N;
+                    long off = (bth * R + r) * N;          /* per-head output row */
+                    long offin = bc_off(d, b, t, h, r);    /* the group's input row */
                     const double *bb = nrm && nrm->bias_B ? nrm->bias_B + (h * R + r) * N : NULL;
                     const double *cb = nrm && nrm->bias_C ? nrm->bias_C + (h * R + r) * N : NULL;
-                    bc_prepare(B + off, N, nrm ? nrm->normw_B : NULL, bb, nrm ? nrm->eps : 0.0, tmp);
-                    rotate_pairs(tmp, phi, N, B_rot + off);
-                    bc_prepare(C + off, N, nrm ? nrm->normw_C : NULL, cb, nrm ? nrm->eps : 0.0, tmp);
-                    rotate_pairs(tmp, phi, N, C_rot + off);
+                    bc_prepare(B + offin, N, nrm ? nrm->normw_B : NULL, bb, nrm ? nrm->eps : 0.0, tmp);
+                    rotate_pairs(tmp, phi, K, N, B_rot + off);
+                    bc_prepare(C + offin, N, nrm ? nrm->normw_C : NULL, cb, nrm ? nrm->eps : 0.0, tmp);
+                    rotate_pairs(tmp, phi, K, N, C_rot + off);
                 }
             }
             if (angle_final)
-                for (long i = 0; i < N / 2; i++)
-                    angle_final[(b * H + h) * (N / 2) + i] = phi[i];
+                for (long i = 0; i < K; i++)
+                    angle_final[(b * H + h) * K + i] = phi[i];
         }
     free(phi);
     free(tmp);
@@ -170,7 +192,8 @@ static void siso_lane(const lane_job *J, long b, long h)
     long NP = N * P;
     double *hs = (double *)malloc(sizeof(double) * NP);
     double *Up = (double *)malloc(sizeof(double) * NP);
-    double *phi = (double *)malloc(sizeof(double) * (N / 2));
+    long K = n_pairs(J->d);
+    double *phi = (double *)malloc(sizeof(double) * K);
     double *tmp = (double *)malloc(sizeof(double) * N);
     double *Bb = (double *)malloc(sizeof(double) * N);
     double *Cb = (double *)malloc(sizeof(double) * N);
@@ -179,8 +202,8 @@ static void siso_lane(const lane_job *J, long b, long h)
         hs[k] = J->h0 ? J->h0[lane * NP + k] : 0.0;
         Up[k] = J->prevBx0 ? J->prevBx0[lane * NP + k] : 0.0;
     }
-    for (long i = 0; i < N / 2; i++)
-        phi[i] = J->angle0 ? J->angle0[lane * (N / 2) + i] : 0.0;
+    for (long i = 0; i < K; i++)
+        phi[i] = J->angle0 ? J->angle0[lane * K + i] : 0.0;
     const m3o_bcnorm *nr = J->nrm;
     for (long t = 0; t < T; t++) {
         long bth = (b * T + t) * H + h;
@@ -188,13 +211,13 @@ static void siso_lane(const lane_job *J, long b, long h)
         double al = exp(dl * J->A[h]);
         double be = (1.0 - lm) * dl * al;
         double ga = lm * dl;
-        for (long i = 0; i < N / 2; i++) phi[i] += dl * J->theta[bth * (N / 2) + i];
-        bc_prepare(J->B + bth * N, N, nr ? nr->normw_B : NULL,
+        for (long i = 0; i < K; i++) phi[i] += dl * J->theta[bth * K + i];
+        bc_prepare(J->B + bc_off(J->d, b, t, h, 0), N, nr ? nr->normw_B : NULL,
                    nr && nr->bias_B ? nr->bias_B + h * N : NULL, nr ? nr->eps : 0.0, tmp);
-        rotate_pairs(tmp, phi, N, Bb);
-        bc_prepare(J->C + bth * N, N, nr ? nr->normw_C : NULL,
+        rotate_pairs(tmp, phi, K, N, Bb);
+        bc_prepare(J->C + bc_off(J->d, b, t, h, 0), N, nr ? nr->normw_C : NULL,
                    nr && nr->bias_C ? nr->bias_C + h * N : NULL, nr ? nr->eps : 0.0, tmp);
-        rotate_pairs(tmp, phi, N, Cb);
+        rotate_pairs(tmp, phi, K, N, Cb);
         const double *xt = J->x + bth * P;
         for (long n = 0; n < N; n++)
             for (long p = 0; p < P; p++) {
@@ -211,7 +234,7 @@ static void siso_lane(const lane_job *J, long b, long h)
     }
     if (J->h_out) memcpy(J->h_out + lane * NP, hs, sizeof(double) * NP);
     if (J->prevBx_out) memcpy(J->prevBx_out + lane * NP, Up, sizeof(double) * NP);
-    if (J->angle_out) memcpy(J->angle_out + lane * (N / 2), phi, sizeof(double) * (N / 2));
+    if (J->angle_out) memcpy(J->angle_out + lane * K, phi, sizeof(double) * K);
     free(hs); free(Up); free(phi); free(tmp); free(Bb); free(Cb);
 }
 
@@ -232,7 +255,8 @@ static void mimo_lane(const lane_job *J, long b, long h)
     double *hs = (double *)malloc(sizeof(double) * NP);
     double *Up = (double *)malloc(sizeof(double) * NP);
     double *Ut = (double *)malloc(sizeof(double) * NP);
-    double *phi = (double *)malloc(sizeof(double) * (N / 2));
+    long K = n_pairs(J->d);
+    double *phi = (double *)malloc(sizeof(double) * K);
     double *tmp = (double *)malloc(sizeof(double) * N);
     double *Bb = (double *)malloc(sizeof(double) * R * N);
     double *Cb = (double *)malloc(sizeof(double) * R * N);
@@ -242,8 +266,8 @@ static void mimo_lane(const lane_job *J, long b, long h)
         hs[k] = J->h0 ? J->h0[lane * NP + k] : 0.0;
         Up[k] = J->prevBx0 ? J->prevBx0[lane * NP + k] : 0.0;
     }
-    for (long i = 0; i < N / 2; i++)
-        phi[i] = J->angle0 ? J->angle0[lane * (N / 2) + i] : 0.0;
+    for (long i = 0; i < K; i++)
+        phi[i] = J->angle0 ? J->angle0[lane * K + i] : 0.0;
     const m3o_bcnorm *nr = J->nrm;
     for (long t = 0; t < T; t++) {
         long bth = (b * T + t) * H + h;
@@ -251,16 +275,16 @@ static void mimo_lane(const lane_job *J, long b, long h)
         double al = exp(dl * J->A[h]);
         double be = (1.0 - lm) * dl * al;
         double ga = lm * dl;
-        for (long i = 0; i < N / 2; i++) phi[i] += dl * J->theta[bth * (N / 2) + i];
+        for (long i = 0; i < K; i++) phi[i] += dl * J->theta[bth * K + i];
         const double *xt = J->x + bth * P;
         for (long r = 0; r < R; r++) {
-            long off = (bth * R + r) * N;
+            long off = bc_off(J->d, b, t, h, r);
             bc_prepare(J->B + off, N, nr ? nr->normw_B : NULL,
                        nr && nr->bias_B ? nr->bias_B + (h * R + r) * N : NULL, nr ? nr->eps : 0.0, tmp);
-            rotate_pairs(tmp, phi, N, Bb + r * N);
+            rotate_pairs(tmp, phi, K, N, Bb + r * N);
             bc_prepare(J->C + off, N, nr ? nr->normw_C : NULL,
                        nr && nr->bias_C ? nr->bias_C + (h * R + r) * N : NULL, nr ? nr->eps : 0.0, tmp);
-            rotate_pairs(tmp, phi, N, Cb + r * N);
+            rotate_pairs(tmp, phi, K, N, Cb + r * N);
             for (long p = 0; p < P; p++)
                 Xr[r * P + p] = (J->Wx ? J->Wx[(h * R + r) * P + p] : 1.0) * xt[p];
         }
@@ -287,7 +311,7 @@ static void mimo_lane(const lane_job *J, long b, long h)
     }
     if (J->h_out) memcpy(J->h_out + lane * NP, hs, sizeof(double) * NP);
     if (J->prevBx_out) memcpy(J->prevBx_out + lane * NP, Up, sizeof(double) * NP);
-    if (J->angle_out) memcpy(J->angle_out + lane * (N / 2), phi, sizeof(double) * (N / 2));
+    if (J->angle_out) memcpy(J->angle_out + lane * K, phi, sizeof(double) * K);
     free(hs); free(Up); free(Ut); free(phi); free(tmp); free(Bb); free(Cb); free(Xr);
 }
 
@@ -313,7 +337,8 @@ static void siso_chunked_lane(const lane_job *J, long b, long h)
     const m3o_bcnorm *nr = J->nrm;
     double *Bb = (double *)malloc(sizeof(double) * T * N);
     double *Cb = (double *)malloc(sizeof(double) * T * N);
-    double *phi = (double *)malloc(sizeof(double) * (N / 2));
+    long K = n_pairs(J->d);
+    double *phi = (double *)malloc(sizeof(double) * K);
     double *tmp = (double *)malloc(sizeof(double) * N);
     double *la = (double *)malloc(sizeof(double) * T);   /* log alpha */
     double *ga = (double *)malloc(sizeof(double) * T);
@@ -321,18 +346,18 @@ static void siso_chunked_lane(const lane_job *J, long b, long h)
     double *g = (double *)malloc(sizeof(double) * NP);
     double *gn = (double *)malloc(sizeof(double) * NP);
     double *cum = (double *)malloc(sizeof(double) * Q);
-    for (long i = 0; i < N / 2; i++)
-        phi[i] = J->angle0 ? J->angle0[lane * (N / 2) + i] : 0.0;
+    for (long i = 0; i < K; i++)
+        phi[i] = J->angle0 ? J->angle0[lane * K + i] : 0.0;
     for (long t = 0; t < T; t++) {
         long bth = (b * T + t) * H + h;
         double dl = J->dt[bth];
-        for (long i = 0; i < N / 2; i++) phi[i] += dl * J->theta[bth * (N / 2) + i];
-        bc_prepare(J->B + bth * N, N, nr ? nr->normw_B : NULL,
+        for (long i = 0; i < K; i++) phi[i] += dl * J->theta[bth * K + i];
+        bc_prepare(J->B + bc_off(J->d, b, t, h, 0), N, nr ? nr->normw_B : NULL,
                    nr && nr->bias_B ? nr->bias_B + h * N : NULL, nr ? nr->eps : 0.0, tmp);
-        rotate_pairs(tmp, phi, N, Bb + t * N);
-        bc_prepare(J->C + bth * N, N, nr ? nr->normw_C : NULL,
+        rotate_pairs(tmp, phi, K, N, Bb + t * N);
+        bc_prepare(J->C + bc_off(J->d, b, t, h, 0), N, nr ? nr->normw_C : NULL,
                    nr && nr->bias_C ? nr->bias_C + h * N : NULL, nr ? nr->eps : 0.0, tmp);
-        rotate_pairs(tmp, phi, N, Cb + t * N);
+        rotate_pairs(tmp, phi, K, N, Cb + t * N);
         la[t] = dl * J->A[h];
         ga[t] = J->lam[bth] * dl;
     }
@@ -391,7 +416,7 @@ static void siso_chunked_lane(const lane_job *J, long b, long h)
                     T > 0 ? Bb[(T - 1) * N + n] * J->x[((b * T + T - 1) * H + h) * P + p]
                           : (J->prevBx0 ? J->prevBx0[lane * NP + n * P + p] : 0.0);
     }
-    if (J->angle_out) memcpy(J->angle_out + lane * (N / 2), phi, sizeof(double) * (N / 2));
+    if (J->angle_out) memcpy(J->angle_out + lane * K, phi, sizeof(double) * K);
     free(Bb); free(Cb); free(phi); free(tmp); free(la); free(ga); free(w);
     free(g); free(gn); free(cum);
 }
@@ -438,6 +463,9 @@ static int check_dims(m3o_dims d, int mimo)
     if (d.batch < 0 || d.seqlen < 0 || d.nheads <= 0 || d.headdim <= 0) return -1;
     if (d.dstate <= 0 || (d.dstate & 1)) return -1;  /* RoPE needs even N */
     if (mimo && d.rank < 1) return -1;
+    if (d.ngroups < 0 || d.rope_pairs < 0) return -1;
+    if (d.nheads % n_groups(d)) return -1;              /* H % G == 0 */
+    if (n_pairs(d) > d.dstate / 2) return -1;
     return 0;
 }
 
@@ -503,8 +531,8 @@ int m3o_siso_chunked(const double *x, const double *dt, const double *A,
 
 /* One decode step (SISO): the loop body for a single token, carrying
  * (h, prev_Bx, angle) in place.  Per-token inputs are shaped as a
- * one-token sequence: x (Bt,1,H,P), dt/lam (Bt,1,H), theta (Bt,1,H,N/2),
- * B/C (Bt,1,H,N); y (Bt,1,H,P). */
+ * one-token sequence: x (Bt,1,H,P), dt/lam (Bt,1,H), theta (Bt,1,H,K),
+ * B/C (Bt,1,G,N); y (Bt,1,H,P). */
 int m3o_step_decode(const double *x, const double *dt, const double *A,
                     const double *lam, const double *theta, const double *B,
                     const double *C, const double *D, const m3o_bcnorm *nrm,
@@ -516,13 +544,13 @@ int m3o_step_decode(const double *x, const double *dt, const double *A,
     long lanes = d.batch * d.nheads, NP = d.dstate * d.headdim;
     double *h1 = (double *)malloc(sizeof(double) * (lanes * NP + 1));
     double *u1 = (double *)malloc(sizeof(double) * (lanes * NP + 1));
-    double *a1 = (double *)malloc(sizeof(double) * (lanes * (d.dstate / 2) + 1));
+    double *a1 = (double *)malloc(sizeof(double) * (lanes * n_pairs(d) + 1));
     int rc = m3o_siso_loop(x, dt, A, lam, theta, B, C, D, nrm, h, prevBx, angle,
                            d, y, h1, u1, a1, nthreads);
     if (rc >= 0) {
         memcpy(h, h1, sizeof(double) * lanes * NP);
         memcpy(prevBx, u1, sizeof(double) * lanes * NP);
-        memcpy(angle, a1, sizeof(double) * lanes * (d.dstate / 2));
+        memcpy(angle, a1, sizeof(double) * lanes * n_pairs(d));
     }
     free(h1); free(u1); free(a1);
     return rc;
@@ -543,13 +571,13 @@ int m3o_mimo_step_decode(const double *x, const double *dt, const double *A,
     long lanes = d.batch * d.nheads, NP = d.dstate * d.headdim;
     double *h1 = (double *)malloc(sizeof(double) * (lanes * NP + 1));
     double *u1 = (double *)malloc(sizeof(double) * (lanes * NP + 1));
-    double *a1 = (double *)malloc(sizeof(double) * (lanes * (d.dstate / 2) + 1));
+    double *a1 = (double *)malloc(sizeof(double) * (lanes * n_pairs(d) + 1));
     int rc = m3o_mimo_loop(x, dt, A, lam, theta, B, C, D, Wx, Wy, nrm, h, prevBx, angle,
                            d, y, h1, u1, a1, nthreads);
     if (rc >= 0) {
         memcpy(h, h1, sizeof(double) * lanes * NP);
         memcpy(prevBx, u1, sizeof(double) * lanes * NP);
-        memcpy(angle, a1, sizeof(double) * lanes * (d.dstate / 2));
+        memcpy(angle, a1, sizeof(double) * lanes * n_pairs(d));
     }
     free(h1); free(u1); free(a1);
     return rc;
@@ -562,8 +590,8 @@ int m3o_mimo_step_decode(const double *x, const double *dt, const double *A,
  *   U_prev[n][p] = sum_r b_prev[r][n] W_x[h,r,p] x_prev[p],
  * the step is the MIMO recurrence for one token (rank 1 with W = 1 is the
  * SISO step), and afterwards b_prev <- B_rot_{t,r}, x_prev <- x_t.
- * In/out: h (Bt,H,N,P), bprev (Bt,H,R,N), xprev (Bt,H,P), angle (Bt,H,N/2).
- * Inputs: x (Bt,H,P), dt/lam (Bt,H), theta (Bt,H,N/2), B/C (Bt,H,R,N),
+ * In/out: h (Bt,H,N,P), bprev (Bt,H,R,N), xprev (Bt,H,P), angle (Bt,H,K).
+ * Inputs: x (Bt,H,P), dt/lam (Bt,H), theta (Bt,H,K), B/C (Bt,G,R,N),
  * W_x/W_y (H,R,P) or NULL.  Output y (Bt,H,P). */
 int m3o_step_decode_factored(const double *x, const double *dt, const double *A,
                              const double *lam, const double *theta, const double *B,
@@ -574,9 +602,12 @@ int m3o_step_decode_factored(const double *x, const double *dt, const double *A,
 {
     if (!h || !bprev || !xprev || !angle || !x || !dt || !A || !lam || !theta || !B || !C || !D || !y)
         return -1;
-    if (d.batch < 0 || d.nheads < 0 || d.headdim <= 0 || d.dstate <= 0 || d.dstate % 2 || d.rank < 1)
+    if (d.batch < 0 || d.nheads <= 0 || d.headdim <= 0 || d.dstate <= 0 || d.dstate % 2 || d.rank < 1)
         return -1;
-    long H = d.nheads, P = d.headdim, N = d.dstate, R = d.rank, NP = N * P;
+    if (d.ngroups < 0 || d.rope_pairs < 0 || d.nheads % n_groups(d) || n_pairs(d) > d.dstate / 2)
+        return -1;
+    d.seqlen = 1;
+    long H = d.nheads, P = d.headdim, N = d.dstate, R = d.rank, NP = N * P, K = n_pairs(d);
     double *tmp = (double *)malloc(sizeof(double) * N);
     double *Bb = (double *)malloc(sizeof(double) * R * N);
     double *Cb = (double *)malloc(sizeof(double) * R * N);
@@ -588,18 +619,18 @@ int m3o_step_decode_factored(const double *x, const double *dt, const double *A,
         double al = exp(dl * A[hh]);
         double be = (1.0 - lm) * dl * al;
         double ga = lm * dl;
-        double *phi = angle + lane * (N / 2);
-        for (long i = 0; i < N / 2; i++) phi[i] += dl * theta[lane * (N / 2) + i];
+        double *phi = angle + lane * K;
+        for (long i = 0; i < K; i++) phi[i] += dl * theta[lane * K + i];
         const double *xt = x + lane * P;
         double *xo = xprev + lane * P;
         for (long r = 0; r < R; r++) {
-            long off = (lane * R + r) * N;
+            long off = bc_off(d, lane / H, 0, hh, r);
             bc_prepare(B + off, N, nrm ? nrm->normw_B : NULL,
                        nrm && nrm->bias_B ? nrm->bias_B + (hh * R + r) * N : NULL, nrm ? nrm->eps : 0.0, tmp);
-            rotate_pairs(tmp, phi, N, Bb + r * N);
+            rotate_pairs(tmp, phi, K, N, Bb + r * N);
             bc_prepare(C + off, N, nrm ? nrm->normw_C : NULL,
                        nrm && nrm->bias_C ? nrm->bias_C + (hh * R + r) * N : NULL, nrm ? nrm->eps : 0.0, tmp);
-            rotate_pairs(tmp, phi, N, Cb + r * N);
+            rotate_pairs(tmp, phi, K, N, Cb + r * N);
             for (long p = 0; p < P; p++) {
                 double w = Wx ? Wx[(hh * R + r) * P + p] : 1.0;
                 Xr[r * P + p] = w * xt[p];

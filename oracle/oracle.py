@@ -52,7 +52,8 @@ def oracle_source_path():
 class _Dims(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_long), ("seqlen", ctypes.c_long),
                 ("nheads", ctypes.c_long), ("headdim", ctypes.c_long),
-                ("dstate", ctypes.c_long), ("rank", ctypes.c_long)]
+                ("dstate", ctypes.c_long), ("rank", ctypes.c_long),
+                ("ngroups", ctypes.c_long), ("rope_pairs", ctypes.c_long)]
 
 
 class _Norm(ctypes.Structure):
@@ -109,8 +110,9 @@ def _norm(norm):
     return ctypes.byref(s), keep + [s]
 
 
-def _dims(Bt, T, H, P, N, R=1):
-    return _Dims(Bt, T, H, P, N, R)
+def _dims(Bt, T, H, P, N, R=1, G=0, K=0):
+    """G: B/C groups (0 or H: one per head); K: rotated pairs (0 or N/2: all)."""
+    return _Dims(Bt, T, H, P, N, R, G, K)
 
 
 def discretize(dt, A, lam):
@@ -118,26 +120,30 @@ def discretize(dt, A, lam):
     dt, A, lam = _f64(dt), _f64(A), _f64(lam)
     Bt, T, H = dt.shape
     al, be, ga = (np.empty_like(dt) for _ in range(3))
-    rc = _load().m3o_discretize(_p(dt), _p(A), _p(lam), Bt, T, H, _p(al), _p(be), _p(ga))
+    L = ctypes.c_long   # long parameters: ctypes would pass a bare int as a C int
+    rc = _load().m3o_discretize(_p(dt), _p(A), _p(lam), L(Bt), L(T), L(H), _p(al), _p(be), _p(ga))
     assert rc == 0
     return al, be, ga
 
 
 def rope_bc(B, C, theta, dt, angle0=None, norm=None):
-    """B_rot, C_rot (same shape as B), angle_final (Bt,H,N/2).
+    """B_rot, C_rot per head (Bt,T,H,[R,]N), angle_final (Bt,H,K).
 
-    B, C may be (Bt,T,H,N) or (Bt,T,H,R,N)."""
+    B, C may be (Bt,T,G,N) or (Bt,T,G,R,N) with G dividing H; theta (Bt,T,H,K)
+    gives H and the number K of rotated pairs."""
     B, C, theta, dt, angle0 = _f64(B), _f64(C), _f64(theta), _f64(dt), _f64(angle0)
     if B.ndim == 4:
-        Bt, T, H, N = B.shape
+        Bt, T, G, N = B.shape
         R = 1
     else:
-        Bt, T, H, R, N = B.shape
-    Br, Cr = np.empty_like(B), np.empty_like(C)
-    ang = np.empty((Bt, H, N // 2))
+        Bt, T, G, R, N = B.shape
+    H, K = theta.shape[2], theta.shape[3]
+    shape = (Bt, T, H, N) if B.ndim == 4 else (Bt, T, H, R, N)
+    Br, Cr = np.empty(shape), np.empty(shape)
+    ang = np.empty((Bt, H, K))
     nptr, keep = _norm(norm)
     rc = _load().m3o_rope_bc(_p(B), _p(C), _p(theta), _p(dt), _p(angle0), nptr,
-                             _dims(Bt, T, H, 1, N, R), _p(Br), _p(Cr), _p(ang))
+                             _dims(Bt, T, H, 1, N, R, G, K), _p(Br), _p(Cr), _p(ang))
     assert rc == 0
     return Br, Cr, ang
 
@@ -148,14 +154,14 @@ def siso_loop(x, dt, A, lam, theta, B, C, D, h0=None, prevBx0=None, angle0=None,
     x, dt, A, lam, theta, B, C, D = (_f64(a) for a in (x, dt, A, lam, theta, B, C, D))
     h0, prevBx0, angle0 = _f64(h0), _f64(prevBx0), _f64(angle0)
     Bt, T, H, P = x.shape
-    N = B.shape[-1]
+    N, G, K = B.shape[-1], B.shape[2], theta.shape[-1]
     y = np.empty_like(x)
     hf = np.empty((Bt, H, N, P))
     uf = np.empty((Bt, H, N, P))
-    af = np.empty((Bt, H, N // 2))
+    af = np.empty((Bt, H, K))
     nptr, keep = _norm(norm)
     rc = _load().m3o_siso_loop(_p(x), _p(dt), _p(A), _p(lam), _p(theta), _p(B), _p(C), _p(D),
-                               nptr, _p(h0), _p(prevBx0), _p(angle0), _dims(Bt, T, H, P, N),
+                               nptr, _p(h0), _p(prevBx0), _p(angle0), _dims(Bt, T, H, P, N, 1, G, K),
                                _p(y), _p(hf), _p(uf), _p(af), int(nthreads))
     if rc < 0:
         raise ValueError("oracle rejected the arguments")
@@ -165,19 +171,19 @@ def siso_loop(x, dt, A, lam, theta, B, C, D, h0=None, prevBx0=None, angle0=None,
 
 def mimo_loop(x, dt, A, lam, theta, B, C, D, Wx=None, Wy=None, h0=None, prevBx0=None,
               angle0=None, norm=None, nthreads=0, return_threads=False):
-    """Sequential rank-R MIMO scan. B, C (Bt,T,H,R,N). Returns y, h, prev_Bx, angle."""
+    """Sequential rank-R MIMO scan. B, C (Bt,T,G,R,N). Returns y, h, prev_Bx, angle."""
     x, dt, A, lam, theta, B, C, D = (_f64(a) for a in (x, dt, A, lam, theta, B, C, D))
     Wx, Wy, h0, prevBx0, angle0 = (_f64(a) for a in (Wx, Wy, h0, prevBx0, angle0))
     Bt, T, H, P = x.shape
-    R, N = B.shape[-2], B.shape[-1]
+    R, N, G, K = B.shape[-2], B.shape[-1], B.shape[2], theta.shape[-1]
     y = np.empty_like(x)
     hf = np.empty((Bt, H, N, P))
     uf = np.empty((Bt, H, N, P))
-    af = np.empty((Bt, H, N // 2))
+    af = np.empty((Bt, H, K))
     nptr, keep = _norm(norm)
     rc = _load().m3o_mimo_loop(_p(x), _p(dt), _p(A), _p(lam), _p(theta), _p(B), _p(C), _p(D),
                                _p(Wx), _p(Wy), nptr, _p(h0), _p(prevBx0), _p(angle0),
-                               _dims(Bt, T, H, P, N, R), _p(y), _p(hf), _p(uf), _p(af),
+                               _dims(Bt, T, H, P, N, R, G, K), _p(y), _p(hf), _p(uf), _p(af),
                                int(nthreads))
     if rc < 0:
         raise ValueError("oracle rejected the arguments")
@@ -191,15 +197,15 @@ def siso_chunked(x, dt, A, lam, theta, B, C, D, chunk, h0=None, prevBx0=None, an
     x, dt, A, lam, theta, B, C, D = (_f64(a) for a in (x, dt, A, lam, theta, B, C, D))
     h0, prevBx0, angle0 = _f64(h0), _f64(prevBx0), _f64(angle0)
     Bt, T, H, P = x.shape
-    N = B.shape[-1]
+    N, G, K = B.shape[-1], B.shape[2], theta.shape[-1]
     y = np.empty_like(x)
     hf = np.empty((Bt, H, N, P))
     uf = np.empty((Bt, H, N, P))
-    af = np.empty((Bt, H, N // 2))
+    af = np.empty((Bt, H, K))
     nptr, keep = _norm(norm)
     rc = _load().m3o_siso_chunked(_p(x), _p(dt), _p(A), _p(lam), _p(theta), _p(B), _p(C),
                                   _p(D), nptr, _p(h0), _p(prevBx0), _p(angle0),
-                                  _dims(Bt, T, H, P, N), int(chunk), _p(y), _p(hf), _p(uf),
+                                  _dims(Bt, T, H, P, N, 1, G, K), ctypes.c_long(int(chunk)), _p(y), _p(hf), _p(uf),
                                   _p(af), int(nthreads))
     if rc < 0:
         raise ValueError("oracle rejected the arguments")
@@ -209,17 +215,17 @@ def siso_chunked(x, dt, A, lam, theta, B, C, D, chunk, h0=None, prevBx0=None, an
 def step_decode(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, prevBx, angle, norm=None,
                 nthreads=0):
     """One SISO decode step. Per-token inputs: x_t (Bt,H,P), dt_t/lam_t (Bt,H),
-    theta_t (Bt,H,N/2), B_t/C_t (Bt,H,N).  Returns y_t (Bt,H,P), h, prev_Bx, angle
+    theta_t (Bt,H,K), B_t/C_t (Bt,G,N).  Returns y_t (Bt,H,P), h, prev_Bx, angle
     (new arrays; the inputs are not modified)."""
     x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D = (
         _f64(a) for a in (x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D))
     h, prevBx, angle = (np.array(a, dtype=np.float64, copy=True) for a in (h, prevBx, angle))
     Bt, H, P = x_t.shape
-    N = B_t.shape[-1]
+    N, G, K = B_t.shape[-1], B_t.shape[1], theta_t.shape[-1]
     y = np.empty((Bt, 1, H, P))
     nptr, keep = _norm(norm)
     rc = _load().m3o_step_decode(_p(x_t), _p(dt_t), _p(A), _p(lam_t), _p(theta_t), _p(B_t),
-                                 _p(C_t), _p(D), nptr, _dims(Bt, 1, H, P, N), _p(h), _p(prevBx),
+                                 _p(C_t), _p(D), nptr, _dims(Bt, 1, H, P, N, 1, G, K), _p(h), _p(prevBx),
                                  _p(angle), _p(y), int(nthreads))
     if rc < 0:
         raise ValueError("oracle rejected the arguments")
@@ -229,16 +235,16 @@ def step_decode(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, prevBx, angle, nor
 def mimo_step_decode(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, prevBx, angle, Wx=None, Wy=None,
                      norm=None, nthreads=0):
     """One rank-R MIMO decode step on the full previous-input state.  B_t, C_t
-    (Bt,H,R,N).  Returns y_t (Bt,H,P), h, prev_Bx, angle (new arrays)."""
+    (Bt,G,R,N).  Returns y_t (Bt,H,P), h, prev_Bx, angle (new arrays)."""
     x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, Wx, Wy = (
         _f64(a) for a in (x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, Wx, Wy))
     h, prevBx, angle = (np.array(a, dtype=np.float64, copy=True) for a in (h, prevBx, angle))
     Bt, H, P = x_t.shape
-    R, N = B_t.shape[-2], B_t.shape[-1]
+    R, N, G, K = B_t.shape[-2], B_t.shape[-1], B_t.shape[1], theta_t.shape[-1]
     y = np.empty((Bt, 1, H, P))
     nptr, keep = _norm(norm)
     rc = _load().m3o_mimo_step_decode(_p(x_t), _p(dt_t), _p(A), _p(lam_t), _p(theta_t), _p(B_t),
-                                      _p(C_t), _p(D), _p(Wx), _p(Wy), nptr, _dims(Bt, 1, H, P, N, R),
+                                      _p(C_t), _p(D), _p(Wx), _p(Wy), nptr, _dims(Bt, 1, H, P, N, R, G, K),
                                       _p(h), _p(prevBx), _p(angle), _p(y), int(nthreads))
     if rc < 0:
         raise ValueError("oracle rejected the arguments")
@@ -249,17 +255,17 @@ def step_decode_factored(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, bprev, xp
                          Wx=None, Wy=None, norm=None):
     """One decode step on the factored previous-input state: bprev (Bt,H,R,N)
     is the rotated B of the previous token per rank and xprev (Bt,H,P) its x.
-    B_t, C_t (Bt,H,R,N) (R = 1 for SISO).  Returns y_t, h, bprev, xprev, angle
-    (new arrays)."""
+    B_t, C_t (Bt,G,R,N) (R = 1 for SISO); theta_t (Bt,H,K).  Returns y_t, h,
+    bprev, xprev, angle (new arrays)."""
     x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, Wx, Wy = (
         _f64(a) for a in (x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, Wx, Wy))
     h, bprev, xprev, angle = (np.array(a, dtype=np.float64, copy=True) for a in (h, bprev, xprev, angle))
     Bt, H, P = x_t.shape
-    R, N = B_t.shape[-2], B_t.shape[-1]
+    R, N, G, K = B_t.shape[-2], B_t.shape[-1], B_t.shape[1], theta_t.shape[-1]
     y = np.empty((Bt, H, P))
     nptr, keep = _norm(norm)
     rc = _load().m3o_step_decode_factored(_p(x_t), _p(dt_t), _p(A), _p(lam_t), _p(theta_t), _p(B_t),
-                                          _p(C_t), _p(D), _p(Wx), _p(Wy), nptr, _dims(Bt, 1, H, P, N, R),
+                                          _p(C_t), _p(D), _p(Wx), _p(Wy), nptr, _dims(Bt, 1, H, P, N, R, G, K),
                                           _p(h), _p(bprev), _p(xprev), _p(angle), _p(y))
     if rc < 0:
         raise ValueError("oracle rejected the arguments")

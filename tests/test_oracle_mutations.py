@@ -19,17 +19,22 @@ MUTATIONS = [
     ("dropped D skip", "yt[p] = acc + J->D[h] * xt[p];", "yt[p] = acc;"),
     ("swapped U terms", "hs[n * P + p] = al * hs[n * P + p] + be * Up[n * P + p] + ga * u;",
      "hs[n * P + p] = al * hs[n * P + p] + be * u + ga * Up[n * P + p];"),
-    ("angle without dt", "phi[i] += dl * J->theta[bth * (N / 2) + i];",
-     "phi[i] += J->theta[bth * (N / 2) + i];"),
+    ("angle without dt", "phi[i] += dl * J->theta[bth * K + i];",
+     "phi[i] += J->theta[bth * K + i];"),
     ("y from C transposed to B", "for (long n = 0; n < N; n++) acc += Cb[n] * hs[n * P + p];",
      "for (long n = 0; n < N; n++) acc += Bb[n] * hs[n * P + p];"),
-    ("alpha sign", "double al = exp(dl * J->A[h]);\n        double be = (1.0 - lm) * dl * al;\n        double ga = lm * dl;\n        for (long i = 0; i < N / 2; i++) phi[i] += dl * J->theta[bth * (N / 2) + i];\n        bc_prepare",
-     "double al = exp(-dl * J->A[h]);\n        double be = (1.0 - lm) * dl * al;\n        double ga = lm * dl;\n        for (long i = 0; i < N / 2; i++) phi[i] += dl * J->theta[bth * (N / 2) + i];\n        bc_prepare"),
+    ("alpha sign", "double al = exp(dl * J->A[h]);\n        double be = (1.0 - lm) * dl * al;\n        double ga = lm * dl;\n        for (long i = 0; i < K; i++) phi[i] += dl * J->theta[bth * K + i];\n        bc_prepare",
+     "double al = exp(-dl * J->A[h]);\n        double be = (1.0 - lm) * dl * al;\n        double ga = lm * dl;\n        for (long i = 0; i < K; i++) phi[i] += dl * J->theta[bth * K + i];\n        bc_prepare"),
     ("MIMO contract without W_y", "acc += (J->Wy ? J->Wy[(h * R + r) * P + p] : 1.0) * yr;", "acc += yr;"),
     ("chunk lookahead dropped", "sg = (1.0 - J->lam[nx]) * J->dt[nx];", "sg = 0.0;"),
     ("factored decode: previous term from the current x", "up += bp[r * N + n] * Xp[r * P + p];",
      "up += bp[r * N + n] * Xr[r * P + p];"),
     ("factored decode: b_prev not advanced", "memcpy(bprev + lane * R * N, Bb, sizeof(double) * R * N);", ""),
+    ("groups interleaved instead of contiguous", "* G + h / (d.nheads / G)) * R + r)", "* G + h % G) * R + r)"),
+    ("partial RoPE zeroes the unrotated pairs", "for (long n = 2 * K; n < N; n++) out[n] = v[n];",
+     "for (long n = 2 * K; n < N; n++) out[n] = 0.0;"),
+    ("partial RoPE rotates the last pairs", "double v0 = v[2 * i], v1 = v[2 * i + 1];\n        out[2 * i] = c * v0 - s * v1;\n        out[2 * i + 1] = s * v0 + c * v1;\n    }\n    for (long n = 2 * K; n < N; n++) out[n] = v[n];",
+     "long j = i + N / 2 - K;\n        double v0 = v[2 * j], v1 = v[2 * j + 1];\n        out[2 * j] = c * v0 - s * v1;\n        out[2 * j + 1] = s * v0 + c * v1;\n    }\n    for (long n = 0; n < N - 2 * K; n++) out[n] = v[n];"),
 ]
 
 PIN_CASES = [
@@ -43,6 +48,8 @@ PIN_CASES = [
     lambda o: pins.test_chunked_equals_loop(o, 4, 37),
     lambda o: pins.test_factored_decode_from_zero_equals_mimo_loop(o, 3),
     lambda o: pins.test_mimo_decode_steps_equal_mimo_loop(o),
+    lambda o: pins.test_grouped_partial_siso(o, 2, 1),
+    lambda o: pins.test_partial_rope_turns_only_first_pairs(o),
 ]
 
 

@@ -23,6 +23,10 @@ oracle's code:
   (previous token's rotated B per rank and its x), reproduce the one-shot
   MIMO scan (dotLLM pull request, "MIMO streaming decode"; TorchMamba README,
   "Models": cache of angle, ssm, x_prev, b_prev);
+* grouped B/C equals per-head B/C repeated over each group's heads, and
+  partial RoPE equals full RoPE with theta zero beyond the first K pairs
+  (TorchMamba README, "Models": n_groups; dotLLM pull request, real-checkpoint
+  run: num_rope_angles 32 of d_state 128);
 * chunked fp64 form equals the loop (ats-v2 README, "Mamba uses a chunked
   parallel scan": exact at float64);
 * rotation invariance and the trapezoid weights' sum.
@@ -412,6 +416,123 @@ def test_mimo_decode_steps_equal_mimo_loop(oracle_mod):
     close(h, h1)
     close(u, u1)
     close(a, a1)
+
+
+# ----------------------------------------------------------------------------
+# grouped B/C (TorchMamba README, "Models": n_groups with H % G == 0; head h
+# reads group h // (H / G)) == per-head B/C repeated over each group's heads;
+# partial RoPE (dotLLM pull request, real-checkpoint run: num_rope_angles 32
+# of d_state 128) == full RoPE with theta zero beyond the first K pairs, and
+# as complex numbers only the first K pairs turn
+# ----------------------------------------------------------------------------
+def _grouped(rng, Bt, T, H, G, P, N, R, K):
+    inp = rnd_inputs(rng, Bt=Bt, T=T, H=H, P=P, N=N, R=R)
+    shp = (Bt, T, G, N) if R == 1 else (Bt, T, G, R, N)
+    inp["B"] = rng.standard_normal(shp) / np.sqrt(N)
+    inp["C"] = rng.standard_normal(shp) / np.sqrt(N)
+    inp["theta"] = inp["theta"][..., :K]
+    return inp
+
+
+def _expand(inp, H, N):
+    """The same inputs with one B/C row per head (np.repeat over each group's
+    heads) and theta zero-padded to all N/2 pairs."""
+    G = inp["B"].shape[2]
+    out = dict(inp)
+    out["B"] = np.repeat(inp["B"], H // G, axis=2)
+    out["C"] = np.repeat(inp["C"], H // G, axis=2)
+    th = np.zeros(inp["theta"].shape[:-1] + (N // 2,))
+    th[..., :inp["theta"].shape[-1]] = inp["theta"]
+    out["theta"] = th
+    return out
+
+
+@pytest.mark.parametrize("G,K", [(1, 3), (2, 1), (6, 2), (3, 4)])
+def test_grouped_partial_siso(oracle_mod, G, K):
+    rng = np.random.default_rng(60 + 7 * G + K)
+    Bt, T, H, P, N = 2, 9, 6, 3, 8
+    inp = _grouped(rng, Bt, T, H, G, P, N, 1, K)
+    full = _expand(inp, H, N)
+    nrm = dict(normw_B=1 + 0.2 * rng.standard_normal(N), normw_C=1 + 0.2 * rng.standard_normal(N),
+               bias_B=rng.standard_normal((H, 1, N)), bias_C=rng.standard_normal((H, 1, N)), eps=1e-5)
+    a0 = rng.uniform(-2, 2, (Bt, H, K))
+    a0f = np.zeros((Bt, H, N // 2))
+    a0f[..., :K] = a0
+    got = oracle_mod.siso_loop(**inp, angle0=a0, norm=nrm)
+    ref = oracle_mod.siso_loop(**full, angle0=a0f, norm=nrm)
+    for gg, rr in zip(got[:3], ref[:3]):
+        close(gg, rr)
+    close(got[3], ref[3][..., :K])
+    close(ref[3][..., K:], 0.0)
+    ch = oracle_mod.siso_chunked(**inp, chunk=4, angle0=a0, norm=nrm)
+    for gg, rr in zip(ch, got):
+        close(gg, rr, rtol=1e-9)
+
+
+@pytest.mark.parametrize("G,K,R", [(2, 2, 2), (1, 3, 3)])
+def test_grouped_partial_mimo_and_decode(oracle_mod, G, K, R):
+    rng = np.random.default_rng(70 + G + K + R)
+    Bt, T, H, P, N = 2, 6, 4, 3, 8
+    inp = _grouped(rng, Bt, T, H, G, P, N, R, K)
+    Wx = 1 + 0.3 * rng.standard_normal((H, R, P))
+    Wy = 1 + 0.3 * rng.standard_normal((H, R, P))
+    full = _expand(inp, H, N)
+    got = oracle_mod.mimo_loop(**inp, Wx=Wx, Wy=Wy)
+    ref = oracle_mod.mimo_loop(**full, Wx=Wx, Wy=Wy)
+    for gg, rr in zip(got[:3], ref[:3]):
+        close(gg, rr)
+    close(got[3], ref[3][..., :K])
+    # decode steps, full state and factored, on the grouped partial inputs
+    h, u, a = np.zeros((Bt, H, N, P)), np.zeros((Bt, H, N, P)), np.zeros((Bt, H, K))
+    hf, bp, xp, af = h.copy(), np.zeros((Bt, H, R, N)), np.zeros((Bt, H, P)), a.copy()
+    for t in range(T):
+        yt, h, u, a = oracle_mod.mimo_step_decode(*_tok(inp, t), h, u, a, Wx=Wx, Wy=Wy)
+        close(yt, got[0][:, t])
+        yf, hf, bp, xp, af = oracle_mod.step_decode_factored(*_tok(inp, t), hf, bp, xp, af, Wx=Wx, Wy=Wy)
+        close(yf, got[0][:, t])
+    close(h, got[1])
+    close(u, got[2])
+    close(hf, got[1])
+    close(a, got[3])
+
+
+def test_grouped_partial_siso_decode(oracle_mod):
+    rng = np.random.default_rng(75)
+    Bt, T, H, G, P, N, K = 2, 5, 4, 2, 3, 8, 2
+    inp = _grouped(rng, Bt, T, H, G, P, N, 1, K)
+    y1, h1, u1, a1 = oracle_mod.siso_loop(**inp)
+    h, u, a = np.zeros((Bt, H, N, P)), np.zeros((Bt, H, N, P)), np.zeros((Bt, H, K))
+    for t in range(T):
+        yt, h, u, a = oracle_mod.step_decode(*_tok(inp, t), h, u, a)
+        close(yt, y1[:, t])
+    close(h, h1)
+    close(u, u1)
+    close(a, a1)
+
+
+def test_partial_rope_turns_only_first_pairs(oracle_mod):
+    rng = np.random.default_rng(76)
+    Bt, T, H, G, N, K = 2, 7, 4, 2, 10, 3
+    inp = _grouped(rng, Bt, T, H, G, 2, N, 1, K)
+    Br, Cr, ang = oracle_mod.rope_bc(inp["B"], inp["C"], inp["theta"], inp["dt"])
+    assert Br.shape == (Bt, T, H, N) and ang.shape == (Bt, H, K)
+    Bh = np.repeat(inp["B"], H // G, axis=2)
+    np.testing.assert_array_equal(Br[..., 2 * K:], Bh[..., 2 * K:])
+    phi = np.cumsum(inp["dt"][..., None] * inp["theta"], axis=1)
+    zb = (Bh[..., 0:2 * K:2] + 1j * Bh[..., 1:2 * K:2]) * np.exp(1j * phi)
+    close(Br[..., 0:2 * K:2] + 1j * Br[..., 1:2 * K:2], zb)
+    close(ang, phi[:, -1])
+
+
+def test_bad_groups_and_pairs(oracle_mod):
+    rng = np.random.default_rng(77)
+    inp = _grouped(rng, 1, 3, 6, 4, 2, 8, 1, 2)     # 6 heads, 4 groups
+    with pytest.raises(ValueError):
+        oracle_mod.siso_loop(**inp)
+    inp = _grouped(rng, 1, 3, 6, 3, 2, 8, 1, 4)
+    inp["theta"] = np.zeros((1, 3, 6, 5))            # 5 pairs of 4 available
+    with pytest.raises(ValueError):
+        oracle_mod.siso_loop(**inp)
 
 
 # ----------------------------------------------------------------------------
