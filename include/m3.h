@@ -6,8 +6,9 @@
  *
  *   alpha_t = exp(dt_t A_h)            beta_t = (1 - lam_t) dt_t alpha_t
  *   gamma_t = lam_t dt_t
- *   Phi_t   = Phi_{t-1} + dt_t theta_t          (per rotation pair i < N/2)
- *   Bbar_t  = R(Phi_t) B_t,  Cbar_t = R(Phi_t) C_t   (pairs (2i, 2i+1))
+ *   Phi_t   = Phi_{t-1} + dt_t theta_t          (per rotation pair i < K)
+ *   Bbar_t  = R(Phi_t) B_t,  Cbar_t = R(Phi_t) C_t   (pairs (2i, 2i+1), i < K;
+ *                                                     elements 2K.. pass through)
  *   U_t     = Bbar_t x_t^T                      (N x P)
  *   h_t     = alpha_t h_{t-1} + beta_t U_{t-1} + gamma_t U_t
  *   y_t     = Cbar_t^T h_t + D_h x_t
@@ -17,15 +18,19 @@
  *
  * Layouts: row-major, last index fastest, all buffers contiguous.
  *   x, y        (batch, seqlen, nheads, headdim)         M3_F32 or M3_BF16
- *   B, C        (batch, seqlen, nheads, dstate)          same dtype as x
- *               (batch, seqlen, nheads, rank, dstate)    MIMO
+ *   B, C        (batch, seqlen, ngroups, dstate)         same dtype as x
+ *               (batch, seqlen, ngroups, rank, dstate)   MIMO
  *   dt, lam     (batch, seqlen, nheads)                  fp32, post-activation
  *                                                        (dt > 0, 0 <= lam <= 1)
- *   theta       (batch, seqlen, nheads, dstate/2)        fp32
+ *   theta       (batch, seqlen, nheads, K)               fp32
  *   A, D        (nheads)                                 fp32
  *   W_x, W_y    (nheads, rank, headdim)                  fp32 (MIMO)
  *   h, prev_Bx  (batch, nheads, dstate, headdim)         fp32
- *   angle       (batch, nheads, dstate/2)                fp32
+ *   angle       (batch, nheads, K)                       fp32
+ * G = ngroups B/C groups (TorchMamba README, "Models": n_groups, with
+ * nheads % G == 0): head h reads the B/C row of group h / (nheads / G).
+ * K = rotated pairs (partial RoPE; dotLLM pull request, real-checkpoint run:
+ * num_rope_angles 32 of dstate 128).  Defaults G = nheads, K = dstate/2.
  *
  * Ownership and execution: the caller owns every buffer (device memory,
  * including the workspace).  The library never allocates, frees or
@@ -61,9 +66,12 @@ typedef enum { M3_F32 = 0, M3_BF16 = 1 } m3_dtype;
 
 /* Problem sizes.  rank is ignored by the SISO entry points (taken as 1);
  * chunk is the chunk length of the chunked algorithm (>= 1); seqlen is
- * ignored by m3_step_decode. */
+ * ignored by the decode steps.  ngroups: B/C groups G (0 = nheads; else
+ * nheads % ngroups == 0).  rope_pairs: rotated pairs K (0 = dstate/2; else
+ * 1 <= K <= dstate/2).  Anything else is M3_ERR_INVALID_ARG. */
 typedef struct {
     int64_t batch, seqlen, nheads, headdim, dstate, rank, chunk;
+    int64_t ngroups, rope_pairs;
 } m3_dims;
 
 /* Optional QkNorm + BC-bias applied to B and C before the rotation
@@ -97,12 +105,13 @@ m3_status m3_discretize(const float *dt, const float *A, const float *lam, m3_di
 /* S2 -- QkNorm + BC-bias + data-dependent RoPE.  (dotLLM pull request,
  * "Stage A: Mamba3QkNorm, Mamba3DataRoPE"; TorchMamba README, "Math notes":
  * accumulated data-dependent pairwise rotations, Props. 2-4.)
- * In: B, C (batch, seqlen, nheads, [rank,] dstate) of `dtype` (rank axis
- * present when d.rank > 1); theta, dt; angle0 (batch, nheads, dstate/2) or
- * NULL for zeros; norm or NULL.
- * Out: B_rot, C_rot (same shape and dtype as B; values rotated in fp32 and
- * rounded to nearest-even on store); angle_final (batch, nheads, dstate/2)
- * or NULL.  Every rank uses the same angle. */
+ * In: B, C (batch, seqlen, ngroups, [rank,] dstate) of `dtype` (rank axis
+ * present when d.rank > 1); theta, dt; angle0 (batch, nheads, K) or NULL for
+ * zeros; norm or NULL.
+ * Out: B_rot, C_rot (batch, seqlen, nheads, [rank,] dstate), one row per
+ * head, dtype of B (values rotated in fp32 and rounded to nearest-even on
+ * store); angle_final (batch, nheads, K) or NULL.  Every rank uses the same
+ * angle. */
 m3_status m3_rope_bc(const void *B, const void *C, m3_dtype dtype, const float *theta,
                      const float *dt, const float *angle0, const m3_bcnorm *norm,
                      m3_dims d, void *B_rot, void *C_rot, float *angle_final,
@@ -140,7 +149,7 @@ m3_status m3_siso_chunked_fwd(const void *x, const float *dt, const float *A,
  *   U_t        = sum_r Bbar_{t,r} X_{t,r}^T
  *   y_t[p]     = sum_r W_y[h,r,p] (Cbar_{t,r}^T h_t)[p] + D_h x_t[p]
  * Arguments as m3_siso_chunked_fwd plus W_x, W_y (nheads, rank, headdim)
- * fp32, each NULL for all ones; B, C are (batch, seqlen, nheads, rank,
+ * fp32, each NULL for all ones; B, C are (batch, seqlen, ngroups, rank,
  * dstate).  prevBx_final is U_{T-1} (summed over ranks). */
 m3_status m3_mimo_chunked_fwd(const void *x, const float *dt, const float *A,
                               const float *lam, const float *theta, const void *B,
@@ -154,11 +163,11 @@ m3_status m3_mimo_chunked_fwd(const void *x, const float *dt, const float *A,
 /* S5 -- one SISO decode step for every (batch, head) lane.  (dotLLM pull
  * request: persistent ssm_state / cum_angle and the single-token step;
  * TorchMamba README: forward == prefill + step, cache (angle, ssm, ...).)
- * In: x_t (batch, nheads, headdim) and B_t, C_t (batch, nheads, dstate) of
- * `dtype`; dt_t, lam_t (batch, nheads), theta_t (batch, nheads, dstate/2),
+ * In: x_t (batch, nheads, headdim) and B_t, C_t (batch, ngroups, dstate) of
+ * `dtype`; dt_t, lam_t (batch, nheads), theta_t (batch, nheads, K),
  * A, D (nheads) fp32.
  * In/out: h, prevBx (batch, nheads, dstate, headdim) fp32 and angle
- * (batch, nheads, dstate/2) fp32, updated in place.
+ * (batch, nheads, K) fp32, updated in place.
  * Out: y_t (batch, nheads, headdim) of `dtype`.  d.seqlen is ignored. */
 m3_status m3_step_decode(const void *x_t, const float *dt_t, const float *A,
                          const float *lam_t, const float *theta_t, const void *B_t,
@@ -174,7 +183,7 @@ m3_status m3_step_decode(const void *x_t, const float *dt_t, const float *A,
  *   h <- alpha h + beta prevBx + gamma U_t,  prevBx <- U_t
  *   y_t = sum_r W_y[r] (Cbar_r^T h) + D x_t
  * Arguments as m3_step_decode plus W_x, W_y (nheads, rank, headdim) fp32,
- * each NULL for all ones; B_t, C_t are (batch, nheads, rank, dstate);
+ * each NULL for all ones; B_t, C_t are (batch, ngroups, rank, dstate);
  * QkNorm/bias as in m3_bcnorm (bias (nheads, rank, dstate)).
  * 1 <= d.rank <= 8 and headdim a multiple of 4 (else M3_ERR_UNSUPPORTED). */
 m3_status m3_mimo_step_decode(const void *x_t, const float *dt_t, const float *A,

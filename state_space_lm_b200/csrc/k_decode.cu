@@ -6,7 +6,8 @@
 //   U = Bbar x^T;  h <- alpha h + beta prev_Bx + gamma U;  prev_Bx <- U
 //   y = Cbar^T h + D x
 // The state (h and prev_Bx, 2 x N x P fp32 per lane, read and written) is all
-// the traffic that matters; every thread streams VEC-wide rows of it.
+// the traffic that matters; every thread streams VEC-wide rows of it.  Head h
+// reads the B/C row of group h / (H / G); pairs j >= K do not rotate.
 #include "m3_internal.cuh"
 
 namespace m3 {
@@ -29,11 +30,12 @@ template <typename T, int VEC>
 __global__ void __launch_bounds__(256) k_decode(DecodeArgs a) {
     using V = typename vecf<VEC>::type;
     const int64_t lane = blockIdx.x, h = lane % a.H;
-    const int P = (int)a.P, N = (int)a.N, NP2 = N / 2;
+    const int P = (int)a.P, N = (int)a.N, NP2 = N / 2, K = (int)a.K;
     const int tid = threadIdx.x, nt = blockDim.x;
+    const int64_t row = (lane / a.H) * a.G + h / (a.H / a.G);   // the group's B/C row
     const T *x = static_cast<const T *>(a.x);
-    const T *Bg = static_cast<const T *>(a.B);
-    const T *Cg = static_cast<const T *>(a.C);
+    const T *Bg = static_cast<const T *>(a.B) + row * N;
+    const T *Cg = static_cast<const T *>(a.C) + row * N;
     T *y = static_cast<T *>(a.y);
 
     extern __shared__ float sm[];
@@ -51,7 +53,7 @@ __global__ void __launch_bounds__(256) k_decode(DecodeArgs a) {
     if (a.nrm.wB || a.nrm.wC) {
         float sb = 0.f, sc = 0.f;
         for (int n = tid; n < N; n += nt) {
-            const float vb = ldf(Bg, lane * N + n), vc = ldf(Cg, lane * N + n);
+            const float vb = ldf(Bg, n), vc = ldf(Cg, n);
             sb += vb * vb;
             sc += vc * vc;
         }
@@ -62,12 +64,14 @@ __global__ void __launch_bounds__(256) k_decode(DecodeArgs a) {
         invC = rsqrtf(sc / N + a.nrm.eps);
     }
     for (int j = tid; j < NP2; j += nt) {
-        const float phi = a.angle[lane * NP2 + j] + dl * a.theta[lane * NP2 + j];
-        a.angle[lane * NP2 + j] = phi;
-        float sn, cn;
-        sincosf(phi, &sn, &cn);
-        float b0 = ldf(Bg, lane * N + 2 * j), b1 = ldf(Bg, lane * N + 2 * j + 1);
-        float c0 = ldf(Cg, lane * N + 2 * j), c1 = ldf(Cg, lane * N + 2 * j + 1);
+        float sn = 0.f, cn = 1.f;
+        if (j < K) {
+            const float phi = a.angle[lane * K + j] + dl * a.theta[lane * K + j];
+            a.angle[lane * K + j] = phi;
+            sincosf(phi, &sn, &cn);
+        }
+        float b0 = ldf(Bg, 2 * j), b1 = ldf(Bg, 2 * j + 1);
+        float c0 = ldf(Cg, 2 * j), c1 = ldf(Cg, 2 * j + 1);
         if (a.nrm.wB) { b0 *= invB * a.nrm.wB[2 * j]; b1 *= invB * a.nrm.wB[2 * j + 1]; }
         if (a.nrm.wC) { c0 *= invC * a.nrm.wC[2 * j]; c1 *= invC * a.nrm.wC[2 * j + 1]; }
         if (a.nrm.biasB) { b0 += a.nrm.biasB[h * N + 2 * j]; b1 += a.nrm.biasB[h * N + 2 * j + 1]; }
@@ -159,11 +163,12 @@ template <typename T, int RT, bool FACT>
 __global__ void __launch_bounds__(256) k_decode_gen(DecodeArgs a) {
     constexpr int VEC = 4;
     const int64_t lane = blockIdx.x, h = lane % a.H;
-    const int P = (int)a.P, N = (int)a.N, NP2 = N / 2, R = (int)a.R;
+    const int P = (int)a.P, N = (int)a.N, NP2 = N / 2, R = (int)a.R, K = (int)a.K;
     const int tid = threadIdx.x, nt = blockDim.x;
+    const int64_t grow = (lane / a.H) * a.G + h / (a.H / a.G);  // the group's B/C rows
     const T *x = static_cast<const T *>(a.x);
-    const T *Bg = static_cast<const T *>(a.B);
-    const T *Cg = static_cast<const T *>(a.C);
+    const T *Bg = static_cast<const T *>(a.B) + grow * R * N;
+    const T *Cg = static_cast<const T *>(a.C) + grow * R * N;
     T *y = static_cast<T *>(a.y);
 
     extern __shared__ float sm[];
@@ -188,7 +193,7 @@ __global__ void __launch_bounds__(256) k_decode_gen(DecodeArgs a) {
             if (r >= R) break;
             float sb = 0.f, sc = 0.f;
             for (int n = tid; n < N; n += nt) {
-                const float vb = ldf(Bg, (lane * R + r) * N + n), vc = ldf(Cg, (lane * R + r) * N + n);
+                const float vb = ldf(Bg, r * N + n), vc = ldf(Cg, r * N + n);
                 sb += vb * vb;
                 sc += vc * vc;
             }
@@ -207,14 +212,16 @@ __global__ void __launch_bounds__(256) k_decode_gen(DecodeArgs a) {
     if (FACT)
         for (int k = tid; k < R * N; k += nt) Pb[k] = a.bprev[lane * R * N + k];
     for (int j = tid; j < NP2; j += nt) {
-        const float phi = a.angle[lane * NP2 + j] + dl * a.theta[lane * NP2 + j];
-        a.angle[lane * NP2 + j] = phi;
-        float sn, cn;
-        sincosf(phi, &sn, &cn);
+        float sn = 0.f, cn = 1.f;
+        if (j < K) {
+            const float phi = a.angle[lane * K + j] + dl * a.theta[lane * K + j];
+            a.angle[lane * K + j] = phi;
+            sincosf(phi, &sn, &cn);
+        }
 #pragma unroll
         for (int r = 0; r < RT; r++) {
             if (r >= R) break;
-            const int64_t o = (lane * R + r) * N + 2 * j;
+            const int64_t o = r * N + 2 * j;
             float b0 = ldf(Bg, o), b1 = ldf(Bg, o + 1), c0 = ldf(Cg, o), c1 = ldf(Cg, o + 1);
             if (a.nrm.wB) { b0 *= invB[r] * a.nrm.wB[2 * j]; b1 *= invB[r] * a.nrm.wB[2 * j + 1]; }
             if (a.nrm.wC) { c0 *= invC[r] * a.nrm.wC[2 * j]; c1 *= invC[r] * a.nrm.wC[2 * j + 1]; }

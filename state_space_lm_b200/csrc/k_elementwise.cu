@@ -75,13 +75,15 @@ __device__ __forceinline__ void st2(__nv_bfloat16 *p, int64_t i, float a, float 
 // One CTA per (b, h) lane walks the sequence in tiles of ny*SEG tokens.  The
 // thread grid is (ny rows) x (N/2 pairs): in pass 1 every row sums dt*theta
 // over its SEG tokens, the rows' partial sums give each row its starting
-// angle, and pass 2 walks the same tokens again rotating B and C.
+// angle, and pass 2 walks the same tokens again rotating B and C.  Only pairs
+// j < K turn (partial RoPE); the rest are copied with QkNorm/bias applied.
+// The lane reads the B/C rows of its group h / (H / G) and writes per head.
 template <typename T>
 __global__ void __launch_bounds__(256) k_rope(RopeArgs a) {
     constexpr int SEG = 16;
     const int64_t lane = blockIdx.x, b = lane / a.H, h = lane % a.H;
-    const int64_t Tn = a.T, H = a.H;
-    const int N = (int)a.N, R = (int)a.R, NP2 = N / 2;
+    const int64_t Tn = a.T, H = a.H, G = a.G, hg = h / (H / G);
+    const int N = (int)a.N, R = (int)a.R, NP2 = N / 2, K = (int)a.K;
     const int ny = min((int)blockDim.x / NP2, 64);
     const int ty = threadIdx.x / NP2, j = threadIdx.x % NP2;
     const bool active = ty < ny;
@@ -99,18 +101,18 @@ __global__ void __launch_bounds__(256) k_rope(RopeArgs a) {
     float *invC = invB + TT * R;      // TT * R
 
     for (int k = threadIdx.x; k < NP2; k += blockDim.x)
-        carry[k] = a.angle0 ? a.angle0[lane * NP2 + k] : 0.f;
+        carry[k] = (a.angle0 && k < K) ? a.angle0[lane * K + k] : 0.f;
     __syncthreads();
 
     const int warp = threadIdx.x >> 5, l32 = threadIdx.x & 31, nw = blockDim.x >> 5;
     for (int64_t t0 = 0; t0 < Tn; t0 += TT) {
         float s = 0.f;
         if (active) {
-            for (int k = 0; k < SEG; k++) {
+            for (int k = 0; k < SEG && j < K; k++) {
                 const int64_t t = t0 + ty * SEG + k;
                 if (t < Tn) {
                     const int64_t bt = (b * Tn + t) * H + h;
-                    s += a.dt[bt] * a.theta[bt * NP2 + j];
+                    s += a.dt[bt] * a.theta[bt * K + j];
                 }
             }
             part[ty * NP2 + j] = s;
@@ -119,7 +121,7 @@ __global__ void __launch_bounds__(256) k_rope(RopeArgs a) {
             for (int row = warp; row < TT * R; row += nw) {
                 const int64_t t = t0 + row / R;
                 if (t >= Tn) continue;
-                const int64_t base = (((b * Tn + t) * H + h) * R + row % R) * N;
+                const int64_t base = (((b * Tn + t) * G + hg) * R + row % R) * N;
                 float sb = 0.f, sc = 0.f;
                 for (int n = l32; n < N; n += 32) {
                     const float vb = ldf(B, base + n), vc = ldf(C, base + n);
@@ -155,12 +157,15 @@ __global__ void __launch_bounds__(256) k_rope(RopeArgs a) {
                 const int64_t t = t0 + tl;
                 if (t >= Tn) break;
                 const int64_t bt = (b * Tn + t) * H + h;
-                phi += a.dt[bt] * a.theta[bt * NP2 + j];
-                float sn, cs;
-                sincosf(phi, &sn, &cs);
+                float sn = 0.f, cs = 1.f;
+                if (j < K) {
+                    phi += a.dt[bt] * a.theta[bt * K + j];
+                    sincosf(phi, &sn, &cs);
+                }
                 for (int r = 0; r < R; r++) {
                     const int64_t idx = (bt * R + r) * N + 2 * j;
-                    float2 bv = ld2(B, idx), cv = ld2(C, idx);
+                    const int64_t src = (((b * Tn + t) * G + hg) * R + r) * N + 2 * j;
+                    float2 bv = ld2(B, src), cv = ld2(C, src);
                     if (a.nrm.wB) {
                         const float iv = invB[tl * R + r];
                         bv.x *= iv * a.nrm.wB[2 * j];
@@ -179,16 +184,21 @@ __global__ void __launch_bounds__(256) k_rope(RopeArgs a) {
                         cv.x += a.nrm.biasC[(h * R + r) * N + 2 * j];
                         cv.y += a.nrm.biasC[(h * R + r) * N + 2 * j + 1];
                     }
-                    st2(Bo, idx, cs * bv.x - sn * bv.y, sn * bv.x + cs * bv.y);
-                    st2(Co, idx, cs * cv.x - sn * cv.y, sn * cv.x + cs * cv.y);
+                    if (j < K) {
+                        st2(Bo, idx, cs * bv.x - sn * bv.y, sn * bv.x + cs * bv.y);
+                        st2(Co, idx, cs * cv.x - sn * cv.y, sn * cv.x + cs * cv.y);
+                    } else {
+                        st2(Bo, idx, bv.x, bv.y);
+                        st2(Co, idx, cv.x, cv.y);
+                    }
                 }
-                if (t == Tn - 1 && a.angle_out) a.angle_out[lane * NP2 + j] = phi;
+                if (t == Tn - 1 && a.angle_out && j < K) a.angle_out[lane * K + j] = phi;
             }
         }
         __syncthreads();
     }
     if (Tn == 0 && a.angle_out)
-        for (int k = threadIdx.x; k < NP2; k += blockDim.x) a.angle_out[lane * NP2 + k] = carry[k];
+        for (int k = threadIdx.x; k < K; k += blockDim.x) a.angle_out[lane * K + k] = carry[k];
 }
 
 cudaError_t launch_rope(const RopeArgs &a, m3_dtype dt, cudaStream_t s) {

@@ -17,6 +17,9 @@
 // For MIMO every token contributes R rows (t, r); the mask depends on the
 // tokens only, X_{s,r} = W_x[r] * x_s and y_t = sum_r W_y[r] * Y_{t,r} + D x_t.
 //
+// Head h reads the B/C rows of group h / (H / G); only the first K pairs
+// rotate (partial RoPE), and theta and the angle hold K values per head.
+//
 // One CTA owns one (b, h) lane and walks its chunks in order; the state g
 // (N x P fp32) and the running angle stay in shared memory for the whole
 // sequence, so no workspace is used.
@@ -54,8 +57,8 @@ int scan_simt_chunk(int64_t P, int64_t N, int64_t R, int64_t chunk) {
 template <typename T>
 __global__ void __launch_bounds__(256) k_scan_simt(ScanArgs a) {
     const int64_t lane = blockIdx.x, b = lane / a.H, h = lane % a.H;
-    const int64_t Tn = a.T, H = a.H;
-    const int P = (int)a.P, N = (int)a.N, R = (int)a.R, Q = a.Q;
+    const int64_t Tn = a.T, H = a.H, G = a.G, hg = h / (H / G);
+    const int P = (int)a.P, N = (int)a.N, R = (int)a.R, Q = a.Q, K = (int)a.K;
     const int NP2 = N / 2, ldn = N + 1, QR = Q * R;
     const int64_t NPs = (int64_t)N * P;
     const int tid = threadIdx.x, nt = blockDim.x;
@@ -72,7 +75,7 @@ __global__ void __launch_bounds__(256) k_scan_simt(ScanArgs a) {
     float *Cb = Bb + (size_t)QR * ldn;   // QR*ldn   rotated C rows
     float *X = Cb + (size_t)QR * ldn;    // QR*P     W_x * x rows
     float *S = X + (size_t)QR * P;       // QR*QR    masked scores
-    float *Ph = S + (size_t)QR * QR;     // Q*NP2    angles
+    float *Ph = S + (size_t)QR * QR;     // Q*K      angles (Q*NP2 reserved)
     float *cum = Ph + (size_t)Q * NP2;   // Q
     float *w = cum + Q;                  // Q
     float *gam = w + Q;                  // Q
@@ -81,9 +84,9 @@ __global__ void __launch_bounds__(256) k_scan_simt(ScanArgs a) {
     float *dts = ec + Q;                 // Q
     float *invB = dts + Q;               // QR
     float *invC = invB + QR;             // QR
-    float *phi = invC + QR;              // NP2      running angle
+    float *phi = invC + QR;              // K        running angle
 
-    for (int j = tid; j < NP2; j += nt) phi[j] = a.angle0 ? a.angle0[lane * NP2 + j] : 0.f;
+    for (int j = tid; j < K; j += nt) phi[j] = a.angle0 ? a.angle0[lane * K + j] : 0.f;
     float f0 = 0.f;
     if (Tn > 0) {
         const int64_t i0 = (b * Tn) * H + h;
@@ -114,7 +117,7 @@ __global__ void __launch_bounds__(256) k_scan_simt(ScanArgs a) {
         // QkNorm: inverse RMS of every B and C row of the chunk
         if (a.nrm.wB || a.nrm.wC) {
             for (int row = warp; row < LR; row += nw) {
-                const int64_t base = (((b * Tn + t0 + row / R) * H + h) * R + row % R) * N;
+                const int64_t base = (((b * Tn + t0 + row / R) * G + hg) * R + row % R) * N;
                 float sb = 0.f, sc = 0.f;
                 for (int n = l32; n < N; n += 32) {
                     const float vb = ldf(Bg, base + n), vc = ldf(Cg, base + n);
@@ -145,11 +148,11 @@ __global__ void __launch_bounds__(256) k_scan_simt(ScanArgs a) {
             ec[i] = expf(cum[i]);
         }
         // (b) running angle per pair over the chunk's tokens
-        for (int j = tid; j < NP2; j += nt) {
+        for (int j = tid; j < K; j += nt) {
             float c = phi[j];
             for (int i = 0; i < L; i++) {
-                c += dts[i] * a.theta[((b * Tn + t0 + i) * H + h) * NP2 + j];
-                Ph[i * NP2 + j] = c;
+                c += dts[i] * a.theta[((b * Tn + t0 + i) * H + h) * K + j];
+                Ph[i * K + j] = c;
             }
             phi[j] = c;
         }
@@ -157,7 +160,7 @@ __global__ void __launch_bounds__(256) k_scan_simt(ScanArgs a) {
         // (c) QkNorm gain, bias and rotation of every B and C row
         for (int it = tid; it < LR * NP2; it += nt) {
             const int j = it % NP2, row = it / NP2, i = row / R, r = row % R;
-            const int64_t base = (((b * Tn + t0 + i) * H + h) * R + r) * N + 2 * j;
+            const int64_t base = (((b * Tn + t0 + i) * G + hg) * R + r) * N + 2 * j;
             float2 bv = ldpair(Bg, base), cv = ldpair(Cg, base);
             if (a.nrm.wB) {
                 bv.x *= invB[row] * a.nrm.wB[2 * j];
@@ -175,8 +178,8 @@ __global__ void __launch_bounds__(256) k_scan_simt(ScanArgs a) {
                 cv.x += a.nrm.biasC[(h * R + r) * N + 2 * j];
                 cv.y += a.nrm.biasC[(h * R + r) * N + 2 * j + 1];
             }
-            float sn, cn;
-            sincosf(Ph[i * NP2 + j], &sn, &cn);
+            float sn = 0.f, cn = 1.f;
+            if (j < K) sincosf(Ph[i * K + j], &sn, &cn);
             Bb[row * ldn + 2 * j] = cn * bv.x - sn * bv.y;
             Bb[row * ldn + 2 * j + 1] = sn * bv.x + cn * bv.y;
             Cb[row * ldn + 2 * j] = cn * cv.x - sn * cv.y;
@@ -245,7 +248,7 @@ __global__ void __launch_bounds__(256) k_scan_simt(ScanArgs a) {
         for (int64_t k = tid; k < NPs; k += nt)
             a.prevBx_out[lane * NPs + k] = a.prevBx0 ? a.prevBx0[lane * NPs + k] : 0.f;
     if (a.angle_out)
-        for (int j = tid; j < NP2; j += nt) a.angle_out[lane * NP2 + j] = phi[j];
+        for (int j = tid; j < K; j += nt) a.angle_out[lane * K + j] = phi[j];
 }
 
 cudaError_t launch_scan_simt(const ScanArgs &a, m3_dtype dt, cudaStream_t s) {

@@ -132,13 +132,15 @@ constexpr uint32_t COL_D1 = 0, COL_D2 = 64, COL_D3 = 128, COL_D4 = 192, D3_STRID
 
 struct TcArgs {
     void *y;               // (Bt, T, H, P) bf16
-    const float *theta;    // (Bt, T, H, N/2) fp32
+    const float *theta;    // (Bt, T, H, K) fp32
     const float *dt, *A, *lam, *D;
     const float *Wx, *Wy;  // MIMO expand / contract vectors (H, R, P), NULL = ones
     const float *h0, *prevBx0, *angle0;
     NormArgs nrm;
     float *h_out, *prevBx_out, *angle_out;
     int64_t Bt, T, H;
+    int64_t G;         // B/C groups: head h reads group h / (H / G)
+    int K;             // rotated pairs (a multiple of 4, <= N/2); pairs >= K pass through
     int64_t seg_len;   // tokens per segment (a multiple of Q); one segment covers the whole sequence
     int nseg;          // segments per lane
     float *ws;         // segment slots (nseg > 1)
@@ -405,6 +407,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int tid = threadIdx.x, warp = tid >> 5, l32 = tid & 31;
     const int nsb = SO ? a.nseg - 1 : a.nseg;          // CTAs per lane in this pass
     const int64_t lane_id = blockIdx.x / nsb, b = lane_id / a.H, h = lane_id % a.H;
+    const int hg = (int)(h / (a.H / a.G));                // B/C group of this head
     const int seg = blockIdx.x % nsb;
     const int64_t Tn = a.T, H = a.H;
     const int64_t t_beg = (int64_t)seg * a.seg_len;
@@ -468,11 +471,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    if (tid < NP2) {
-        float p0 = 0.f;                                   // state-only: the segment's own frame
-        if (!SO) p0 = slot_in ? slot_in[SLOT_PHIN + tid] : (a.angle0 ? a.angle0[lane_id * NP2 + tid] : 0.f);
-        phic[tid] = p0;
-    }
     if (R > 1) {
         for (int k = tid; k < R * P; k += THREADS) {
             wxs[k] = a.Wx ? a.Wx[h * R * P + k] : 1.f;
@@ -488,15 +486,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         // ------------------------------------------------------------ producer
         // converged warp, warp-uniform coordinates, one elected lane issues
         {
-            // B and C of a chunk: rows (token, rank) -- a 4-D box (N, H, T, Bt)
-            // for SISO, a 5-D box (N, R, H, T, Bt) for MIMO
+            // B and C of a chunk: rows (token, rank) of this head's group -- a
+            // 4-D box (N, G, T, Bt) for SISO, a 5-D box (N, R, G, T, Bt) for MIMO
             auto load_bc = [&](uint32_t dst, const CUtensorMap *m, int t0, uint32_t fb) {
-                if (R == 1) tma_load4(dst, m, 0, (int)h, t0, (int)b, fb);
-                else tma_load5(dst, m, 0, 0, (int)h, t0, (int)b, fb);
+                if (R == 1) tma_load4(dst, m, 0, hg, t0, (int)b, fb);
+                else tma_load5(dst, m, 0, 0, hg, t0, (int)b, fb);
             };
             auto prefetch_bc = [&](const CUtensorMap *m, int t0) {
-                if (R == 1) tma_prefetch4(m, 0, (int)h, t0, (int)b);
-                else tma_prefetch5(m, 0, 0, (int)h, t0, (int)b);
+                if (R == 1) tma_prefetch4(m, 0, hg, t0, (int)b);
+                else tma_prefetch5(m, 0, 0, hg, t0, (int)b);
             };
             // L2 prefetch runs PFD chunks ahead of the shared-memory rings, so
             // a load issued when a stage frees up finds its data in L2
@@ -643,17 +641,29 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t atom = (uint32_t)(j4 >> 3) * (Q * 128);
         const int chk = j4 & 7;                    // 16-byte chunk within the 128-byte atom row
         const int i0 = tg * TPT;
+        if (pt < NP2) {
+            // the angle entering the first chunk (read after the first named barrier
+            // of the chunk loop); state-only: the segment's own frame, zero
+            float p0 = 0.f;
+            if (!SO)
+                p0 = slot_in ? slot_in[SLOT_PHIN + pt]
+                             : ((a.angle0 && pt < a.K) ? a.angle0[lane_id * a.K + pt] : 0.f);
+            phic[pt] = p0;
+        }
         // theta of my tokens comes straight from global memory into registers,
-        // one chunk ahead (the producer has already pulled it into L2)
+        // one chunk ahead (the producer has already pulled it into L2).  Pairs
+        // from K on take theta = 0: their angle stays 0 and they pass through.
         const float4 *thg = reinterpret_cast<const float4 *>(a.theta);
+        const int K4 = a.K / 4;
+        const bool turns = j4 < K4;
         float4 thv[TPT];
         auto load_theta = [&](int c) {
             const int64_t t0 = t_beg + (int64_t)c * QT;
 #pragma unroll
             for (int u = 0; u < TPT; u++) {
                 const int64_t t = t0 + i0 + u;
-                thv[u] = (c < nchunks && t < t_end) ? thg[((b * Tn + t) * H + h) * (NP2 / 4) + j4]
-                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                thv[u] = (c < nchunks && t < t_end && turns) ? thg[((b * Tn + t) * H + h) * K4 + j4]
+                                                             : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         };
         load_theta(0);
@@ -825,9 +835,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (tg == 15) {
                 // the last token group ends at the chunk's last token
                 *reinterpret_cast<float4 *>(phic + 4 * j4) = make_float4(phi[0], phi[1], phi[2], phi[3]);
-                if (last_chunk && a.angle_out)
-                    *reinterpret_cast<float4 *>(a.angle_out + lane_id * NP2 + 4 * j4) =
-                        make_float4(phi[0], phi[1], phi[2], phi[3]);
                 if (SO && c == nchunks - 1)
                     *reinterpret_cast<float4 *>(slot_out + SLOT_PHIL + 4 * j4) =
                         make_float4(phi[0], phi[1], phi[2], phi[3]);
@@ -837,6 +844,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                 mbar_arrive(bar(B_BEMPTY + sb));
                 mbar_arrive(bar(B_CEMPTY + scf));
             }
+        }
+        // the angle after the sequence's last token: phic after the last chunk
+        // (every prep thread leaves the loop at the same chunk)
+        if (last_seg && a.angle_out) {
+            named_bar(1, PREP_THREADS);
+            for (int k = pt; k < a.K; k += PREP_THREADS) a.angle_out[lane_id * a.K + k] = phic[k];
         }
     } else if (warp == W_XB) {
         // ------------------------------------------------------ X operands
@@ -1364,7 +1377,7 @@ __global__ void __launch_bounds__(256) k_seg_combine(TcArgs a) {
     const int64_t r0 = (lane * N + 2 * i) * P + p, r1 = r0 + P;
     float g0 = (a.h0 ? a.h0[r0] : 0.f) + f0 * (a.prevBx0 ? a.prevBx0[r0] : 0.f);
     float g1 = (a.h0 ? a.h0[r1] : 0.f) + f0 * (a.prevBx0 ? a.prevBx0[r1] : 0.f);
-    float phi = a.angle0 ? a.angle0[lane * NP2 + i] : 0.f;
+    float phi = (a.angle0 && i < a.K) ? a.angle0[lane * a.K + i] : 0.f;
     for (int j = 0; j < a.nseg - 1; j++) {
         float *sl = a.ws + ((size_t)lane * (a.nseg - 1) + j) * SLOT_FLOATS;
         const float l0 = sl[SLOT_G + 2 * i * P + p], l1 = sl[SLOT_G + (2 * i + 1) * P + p];
@@ -1394,6 +1407,7 @@ size_t scan_tc_workspace_bytes(int64_t Bt, int64_t H, int64_t T) {
 bool scan_tc_supported(const ScanArgs &a, m3_dtype dt) {
     const bool shape = a.mimo_layout ? (a.R == 2 || a.R == 4) : (a.R == 1);
     return dt == M3_BF16 && shape && a.P == tc::P && a.N == tc::N && a.Q > 0 && a.Q % (tc::Q / a.R) == 0 &&
+           a.K % 4 == 0 && a.K > 0 && a.G > 0 &&
            a.T > 0 && a.T <= ((int64_t)1 << 30) && a.Bt <= 65535 && a.H <= 65535;
 }
 
@@ -1404,11 +1418,11 @@ static cudaError_t launch_tc_r(const ScanArgs &a, cudaStream_t s) {
     CUtensorMap mx, mb, mc, mth;
     const int64_t rk = R > 1 ? R : 0;
     if (!make_map(&mx, a.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P, a.H, a.T, a.Bt, P, QT, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mb, a.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, a.H, a.T, a.Bt, N, QT, CU_TENSOR_MAP_SWIZZLE_NONE,
+        !make_map(&mb, a.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, a.G, a.T, a.Bt, N, QT, CU_TENSOR_MAP_SWIZZLE_NONE,
                   rk) ||
-        !make_map(&mc, a.C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, a.H, a.T, a.Bt, N, QT, CU_TENSOR_MAP_SWIZZLE_NONE,
+        !make_map(&mc, a.C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, a.G, a.T, a.Bt, N, QT, CU_TENSOR_MAP_SWIZZLE_NONE,
                   rk) ||
-        !make_map(&mth, a.theta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, NP2, a.H, a.T, a.Bt, NP2, QT,
+        !make_map(&mth, a.theta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.K, a.H, a.T, a.Bt, (uint32_t)a.K, QT,
                   CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     TcArgs t;
@@ -1419,7 +1433,7 @@ static cudaError_t launch_tc_r(const ScanArgs &a, cudaStream_t s) {
     t.h0 = a.h0; t.prevBx0 = a.prevBx0; t.angle0 = a.angle0;
     t.nrm = a.nrm;
     t.h_out = a.h_out; t.prevBx_out = a.prevBx_out; t.angle_out = a.angle_out;
-    t.Bt = a.Bt; t.T = a.T; t.H = a.H;
+    t.Bt = a.Bt; t.T = a.T; t.H = a.H; t.G = a.G; t.K = (int)a.K;
     const SegPlan pl = seg_plan(a.Bt * a.H, a.T);
     t.nseg = pl.nseg;
     t.seg_len = pl.seg_len;

@@ -46,6 +46,17 @@ m3_status check_core_dims(const m3_dims &d, bool need_seq) {
     return M3_OK;
 }
 
+// B/C groups and rotated pairs, with 0 meaning one group per head and every
+// pair (TorchMamba README, "Models": n_groups with H % G == 0; dotLLM pull
+// request, real-checkpoint run: num_rope_angles of dstate).
+m3_status resolve_groups(const m3_dims &d, int64_t &G, int64_t &K) {
+    if (d.ngroups < 0 || d.rope_pairs < 0) return M3_ERR_INVALID_ARG;
+    G = d.ngroups ? d.ngroups : d.nheads;
+    K = d.rope_pairs ? d.rope_pairs : d.dstate / 2;
+    if (d.nheads % G || K > d.dstate / 2) return M3_ERR_INVALID_ARG;
+    return M3_OK;
+}
+
 m3_status read_norm(const m3_bcnorm *n, NormArgs &o) {
     o = NormArgs{nullptr, nullptr, nullptr, nullptr, 0.f};
     if (!n) return M3_OK;
@@ -70,6 +81,8 @@ m3_status chunked_common(const void *x, const float *dt, const float *A, const f
     if ((st = check_dtype(dtype)) != M3_OK) return st;
     if ((st = check_core_dims(d, true)) != M3_OK) return st;
     if (d.chunk < 1) return M3_ERR_INVALID_ARG;
+    int64_t G, K;
+    if ((st = resolve_groups(d, G, K)) != M3_OK) return st;
     const int64_t R = mimo ? d.rank : 1;
     if (mimo && d.rank < 1) return M3_ERR_INVALID_ARG;
     if (R > kMaxRank) return M3_ERR_UNSUPPORTED;
@@ -99,6 +112,7 @@ m3_status chunked_common(const void *x, const float *dt, const float *A, const f
     a.nrm = nrm;
     a.y = y; a.h_out = h_final; a.prevBx_out = prevBx_final; a.angle_out = angle_final;
     a.Bt = d.batch; a.T = d.seqlen; a.H = d.nheads; a.P = d.headdim; a.N = d.dstate; a.R = R;
+    a.G = G; a.K = K;
     a.mimo_layout = mimo ? 1 : 0;
     a.ws = workspace;
     a.Q = (int)d.chunk;
@@ -139,6 +153,7 @@ size_t m3_workspace_bytes(int which, m3_dims d, m3_dtype dtype) {
     // only the tensor-core path uses scratch (long sequences over few lanes)
     if ((which != M3_WS_SISO && which != M3_WS_MIMO) || check_core_dims(d, true) != M3_OK || d.chunk < 1) return 0;
     ScanArgs a{};
+    if (resolve_groups(d, a.G, a.K) != M3_OK) return 0;
     a.Bt = d.batch; a.T = d.seqlen; a.H = d.nheads; a.P = d.headdim; a.N = d.dstate;
     a.R = which == M3_WS_MIMO ? d.rank : 1;
     a.Q = (int)d.chunk; a.mimo_layout = which == M3_WS_MIMO ? 1 : 0;
@@ -162,6 +177,8 @@ m3_status m3_rope_bc(const void *B, const void *C, m3_dtype dtype, const float *
     m3_status st;
     if ((st = check_dtype(dtype)) != M3_OK) return st;
     if ((st = check_core_dims(d, true)) != M3_OK) return st;
+    int64_t G, K;
+    if ((st = resolve_groups(d, G, K)) != M3_OK) return st;
     const int64_t R = d.rank > 1 ? d.rank : 1;
     if (d.rank < 0) return M3_ERR_INVALID_ARG;
     if (R > kMaxRank) return M3_ERR_UNSUPPORTED;
@@ -175,7 +192,7 @@ m3_status m3_rope_bc(const void *B, const void *C, m3_dtype dtype, const float *
     RopeArgs a;
     a.B = B; a.C = C; a.theta = theta; a.dt = dt; a.angle0 = angle0; a.nrm = nrm;
     a.Bo = B_rot; a.Co = C_rot; a.angle_out = angle_final;
-    a.Bt = d.batch; a.T = d.seqlen; a.H = d.nheads; a.R = R; a.N = d.dstate;
+    a.Bt = d.batch; a.T = d.seqlen; a.H = d.nheads; a.R = R; a.N = d.dstate; a.G = G; a.K = K;
     return launched(launch_rope(a, dtype, (cudaStream_t)stream));
 }
 
@@ -207,6 +224,8 @@ m3_status m3_step_decode(const void *x_t, const float *dt_t, const float *A, con
     m3_status st;
     if ((st = check_dtype(dtype)) != M3_OK) return st;
     if ((st = check_core_dims(d, false)) != M3_OK) return st;
+    int64_t G, K;
+    if ((st = resolve_groups(d, G, K)) != M3_OK) return st;
     M3_REQ(A); M3_REQ(D);
     if (d.batch > 0) {
         M3_REQ(x_t); M3_REQ(dt_t); M3_REQ(lam_t); M3_REQ(theta_t); M3_REQ(B_t); M3_REQ(C_t);
@@ -218,7 +237,7 @@ m3_status m3_step_decode(const void *x_t, const float *dt_t, const float *A, con
     DecodeArgs a;
     a.x = x_t; a.B = B_t; a.C = C_t; a.dt = dt_t; a.A = A; a.lam = lam_t; a.theta = theta_t; a.D = D;
     a.nrm = nrm; a.h = h; a.prevBx = prevBx; a.angle = angle; a.y = y_t;
-    a.Bt = d.batch; a.H = d.nheads; a.P = d.headdim; a.N = d.dstate;
+    a.Bt = d.batch; a.H = d.nheads; a.P = d.headdim; a.N = d.dstate; a.G = G; a.K = K;
     return launched(launch_decode(a, dtype, (cudaStream_t)stream));
 }
 
@@ -231,6 +250,8 @@ m3_status decode_gen(const void *x_t, const float *dt_t, const float *A, const f
     m3_status st;
     if ((st = check_dtype(dtype)) != M3_OK) return st;
     if ((st = check_core_dims(d, false)) != M3_OK) return st;
+    int64_t G, K;
+    if ((st = resolve_groups(d, G, K)) != M3_OK) return st;
     if (d.rank < 1) return M3_ERR_INVALID_ARG;
     if (d.rank > kMaxRank || d.headdim % 4) return M3_ERR_UNSUPPORTED;
     M3_REQ(A); M3_REQ(D);
@@ -247,7 +268,7 @@ m3_status decode_gen(const void *x_t, const float *dt_t, const float *A, const f
     DecodeArgs a;
     a.x = x_t; a.B = B_t; a.C = C_t; a.dt = dt_t; a.A = A; a.lam = lam_t; a.theta = theta_t; a.D = D;
     a.nrm = nrm; a.h = h; a.prevBx = prevBx; a.angle = angle; a.y = y_t;
-    a.Bt = d.batch; a.H = d.nheads; a.P = d.headdim; a.N = d.dstate;
+    a.Bt = d.batch; a.H = d.nheads; a.P = d.headdim; a.N = d.dstate; a.G = G; a.K = K;
     a.Wx = W_x; a.Wy = W_y; a.bprev = b_prev; a.xprev = x_prev; a.R = d.rank;
     return launched(launch_decode_gen(a, dtype, factored, (cudaStream_t)stream));
 }

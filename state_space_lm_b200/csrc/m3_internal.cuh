@@ -41,6 +41,7 @@ struct ScanArgs {
     void *y;
     float *h_out, *prevBx_out, *angle_out;
     int64_t Bt, T, H, P, N, R;
+    int64_t G = 0, K = 0;  // B/C groups (H % G == 0) and rotated pairs (K <= N/2), resolved
     int Q;             // chunk length actually used by the kernel
     int mimo_layout;   // B/C carry a rank axis
     void *ws;          // caller's workspace (may be null when none is needed)
@@ -53,6 +54,7 @@ struct DecodeArgs {
     float *h, *prevBx, *angle;
     void *y;
     int64_t Bt, H, P, N;
+    int64_t G = 0, K = 0;  // B/C groups and rotated pairs, resolved
     // rank-R and factored-state decode (k_decode_gen)
     const float *Wx = nullptr, *Wy = nullptr;   // (H, R, P), NULL = ones
     float *bprev = nullptr, *xprev = nullptr;   // factored previous-input state
@@ -66,6 +68,7 @@ struct RopeArgs {
     void *Bo, *Co;
     float *angle_out;
     int64_t Bt, T, H, R, N;
+    int64_t G = 0, K = 0;  // B/C groups and rotated pairs, resolved
 };
 
 // Host launchers (each returns cudaSuccess or the launch error).

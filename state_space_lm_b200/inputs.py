@@ -69,12 +69,14 @@ def _uniform(g, shape, lo, hi):
 
 def scan_inputs(batch, seqlen, nheads, headdim, dstate, rank=1, dtype="bf16",
                 dt_shift=-2.0, seed=SEED_BASE, mimo_weights=None, bcnorm=False,
-                generator=None):
+                generator=None, ngroups=0, rope_pairs=0):
     """Inputs of one chunked-scan call, as CPU tensors in their storage dtype.
 
     Returns a dict with x (Bt,T,H,P), dt (Bt,T,H), A (H), lam (Bt,T,H),
-    theta (Bt,T,H,N/2), B and C ((Bt,T,H,N) when rank == 1 and mimo_weights is
-    falsy, else (Bt,T,H,R,N)), D (H), and, for MIMO, Wx and Wy (H,R,P).
+    theta (Bt,T,H,K), B and C ((Bt,T,G,N) when rank == 1 and mimo_weights is
+    falsy, else (Bt,T,G,R,N)), D (H), and, for MIMO, Wx and Wy (H,R,P).
+    G = ngroups and K = rope_pairs, 0 meaning H and N/2 (the draws are the
+    same in number and order; only these shapes change).
     With bcnorm=True it adds normw_B, normw_C (N), bias_B, bias_C (H,R,N) and
     eps.  The generator is returned under "generator" so that later draws
     (decode steps) continue the same stream.
@@ -82,14 +84,15 @@ def scan_inputs(batch, seqlen, nheads, headdim, dstate, rank=1, dtype="bf16",
     g = generator if generator is not None else make_generator(seed)
     sdt = _DTYPES[dtype]
     Bt, T, H, P, N, R = batch, seqlen, nheads, headdim, dstate, rank
+    G, K = ngroups or H, rope_pairs or N // 2
     mimo = bool(mimo_weights) if mimo_weights is not None else R > 1
-    bc_shape = (Bt, T, H, R, N) if mimo else (Bt, T, H, N)
+    bc_shape = (Bt, T, G, R, N) if mimo else (Bt, T, G, N)
     out = {}
     out["x"] = _normal(g, (Bt, T, H, P)).to(sdt)
     out["dt"] = torch.nn.functional.softplus(_normal(g, (Bt, T, H)) + dt_shift).float()
     out["A"] = (-torch.exp(_uniform(g, (H,), 0.0, 1.0))).float()
     out["lam"] = torch.sigmoid(_normal(g, (Bt, T, H))).float()
-    out["theta"] = _uniform(g, (Bt, T, H, N // 2), -math.pi / 8, math.pi / 8).float()
+    out["theta"] = _uniform(g, (Bt, T, H, K), -math.pi / 8, math.pi / 8).float()
     out["B"] = (_normal(g, bc_shape) / math.sqrt(N)).to(sdt)
     out["C"] = (_normal(g, bc_shape) / math.sqrt(N)).to(sdt)
     out["D"] = _normal(g, (H,)).float()
@@ -107,19 +110,21 @@ def scan_inputs(batch, seqlen, nheads, headdim, dstate, rank=1, dtype="bf16",
 
 
 def decode_step_inputs(generator, batch, nheads, headdim, dstate, dtype="bf16",
-                       dt_shift=-2.0, rank=1, rank_axis=False):
+                       dt_shift=-2.0, rank=1, rank_axis=False, ngroups=0, rope_pairs=0):
     """Per-token inputs of one decode step, drawn from ``generator``:
-    x_t (Bt,H,P), dt_t (Bt,H), lam_t (Bt,H), theta_t (Bt,H,N/2), B_t and C_t
-    (Bt,H,N), or (Bt,H,R,N) when rank > 1 or rank_axis."""
+    x_t (Bt,H,P), dt_t (Bt,H), lam_t (Bt,H), theta_t (Bt,H,K), B_t and C_t
+    (Bt,G,N), or (Bt,G,R,N) when rank > 1 or rank_axis (G = ngroups or H,
+    K = rope_pairs or N/2)."""
     g = generator
     sdt = _DTYPES[dtype]
     Bt, H, P, N = batch, nheads, headdim, dstate
-    bc = (Bt, H, rank, N) if (rank > 1 or rank_axis) else (Bt, H, N)
+    G, K = ngroups or H, rope_pairs or N // 2
+    bc = (Bt, G, rank, N) if (rank > 1 or rank_axis) else (Bt, G, N)
     out = {}
     out["x"] = _normal(g, (Bt, H, P)).to(sdt)
     out["dt"] = torch.nn.functional.softplus(_normal(g, (Bt, H)) + dt_shift).float()
     out["lam"] = torch.sigmoid(_normal(g, (Bt, H))).float()
-    out["theta"] = _uniform(g, (Bt, H, N // 2), -math.pi / 8, math.pi / 8).float()
+    out["theta"] = _uniform(g, (Bt, H, K), -math.pi / 8, math.pi / 8).float()
     out["B"] = (_normal(g, bc) / math.sqrt(N)).to(sdt)
     out["C"] = (_normal(g, bc) / math.sqrt(N)).to(sdt)
     return out

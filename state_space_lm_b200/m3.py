@@ -37,7 +37,8 @@ class Dims(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64),
                 ("nheads", ctypes.c_int64), ("headdim", ctypes.c_int64),
                 ("dstate", ctypes.c_int64), ("rank", ctypes.c_int64),
-                ("chunk", ctypes.c_int64)]
+                ("chunk", ctypes.c_int64), ("ngroups", ctypes.c_int64),
+                ("rope_pairs", ctypes.c_int64)]
 
 
 class BcNorm(ctypes.Structure):
@@ -163,39 +164,43 @@ def discretize(dt, A, lam, out=None, stream=None):
     """S1: alpha, beta, gamma (Bt,T,H) fp32."""
     Bt, T, H = dt.shape
     al, be, ga = out if out is not None else tuple(torch.empty_like(dt) for _ in range(3))
-    d = Dims(Bt, T, H, 1, 2, 1, 1)
+    d = Dims(Bt, T, H, 1, 2, 1, 1, 0, 0)
     _check(lib().m3_discretize(_ptr(dt), _ptr(A), _ptr(lam), d, _ptr(al), _ptr(be), _ptr(ga),
                                _stream(stream)), "m3_discretize")
     return al, be, ga
 
 
 def rope_bc(B, C, theta, dt, angle0=None, norm=None, out=None, stream=None):
-    """S2: B_rot, C_rot (shape/dtype of B) and angle_final (Bt,H,N/2) fp32.
-    B, C are (Bt,T,H,N) or (Bt,T,H,R,N)."""
+    """S2: B_rot, C_rot (Bt,T,H,[R,]N), one row per head, dtype of B, and
+    angle_final (Bt,H,K) fp32.  B, C are (Bt,T,G,N) or (Bt,T,G,R,N) with G
+    dividing H; theta (Bt,T,H,K) gives H and the number K of rotated pairs."""
     if B.dim() == 4:
-        Bt, T, H, N = B.shape
+        Bt, T, G, N = B.shape
         R = 1
     else:
-        Bt, T, H, R, N = B.shape
+        Bt, T, G, R, N = B.shape
+    H, K = theta.shape[2], theta.shape[3]
     if out is None:
-        out = (torch.empty_like(B), torch.empty_like(C),
-               torch.empty(Bt, H, N // 2, device=B.device, dtype=torch.float32))
+        shape = (Bt, T, H, N) if B.dim() == 4 else (Bt, T, H, R, N)
+        out = (torch.empty(shape, device=B.device, dtype=B.dtype),
+               torch.empty(shape, device=B.device, dtype=B.dtype),
+               torch.empty(Bt, H, K, device=B.device, dtype=torch.float32))
     Br, Cr, ang = out
     nptr, keep = _norm(norm)
-    d = Dims(Bt, T, H, 1, N, R, 1)
+    d = Dims(Bt, T, H, 1, N, R, 1, G, K)
     _check(lib().m3_rope_bc(_ptr(B), _ptr(C), _DTYPE[B.dtype], _ptr(theta), _ptr(dt), _ptr(angle0),
                             nptr, d, _ptr(Br), _ptr(Cr), _ptr(ang), _stream(stream)), "m3_rope_bc")
     return Br, Cr, ang
 
 
-def _state_outs(x, N, P, out):
+def _state_outs(x, N, P, K, out):
     Bt, T, H = x.shape[0], x.shape[1], x.shape[2]
     if out is not None:
         return out
     dev = x.device
     return (torch.empty_like(x), torch.empty(Bt, H, N, P, device=dev, dtype=torch.float32),
             torch.empty(Bt, H, N, P, device=dev, dtype=torch.float32),
-            torch.empty(Bt, H, N // 2, device=dev, dtype=torch.float32))
+            torch.empty(Bt, H, K, device=dev, dtype=torch.float32))
 
 
 def _workspace(which, d, dtype, workspace, dev):
@@ -208,11 +213,12 @@ def _workspace(which, d, dtype, workspace, dev):
 
 def siso_chunked_fwd(x, dt, A, lam, theta, B, C, D, chunk, norm=None, h0=None, prevBx0=None,
                      angle0=None, workspace=None, out=None, stream=None):
-    """S1+S2+S3: returns y (Bt,T,H,P), h_final, prevBx_final (Bt,H,N,P), angle_final."""
+    """S1+S2+S3: returns y (Bt,T,H,P), h_final, prevBx_final (Bt,H,N,P), angle_final
+    (Bt,H,K).  B, C (Bt,T,G,N) with G dividing H; theta (Bt,T,H,K)."""
     Bt, T, H, P = x.shape
-    N = B.shape[-1]
-    y, hf, uf, af = _state_outs(x, N, P, out)
-    d = Dims(Bt, T, H, P, N, 1, int(chunk))
+    N, G, K = B.shape[-1], B.shape[2], theta.shape[-1]
+    y, hf, uf, af = _state_outs(x, N, P, K, out)
+    d = Dims(Bt, T, H, P, N, 1, int(chunk), G, K)
     dtype = _DTYPE[x.dtype]
     ws, nbytes = _workspace(M3_WS_SISO, d, dtype, workspace, x.device)
     nptr, keep = _norm(norm)
@@ -225,11 +231,11 @@ def siso_chunked_fwd(x, dt, A, lam, theta, B, C, D, chunk, norm=None, h0=None, p
 
 def mimo_chunked_fwd(x, dt, A, lam, theta, B, C, D, chunk, W_x=None, W_y=None, norm=None, h0=None,
                      prevBx0=None, angle0=None, workspace=None, out=None, stream=None):
-    """S4: B, C (Bt,T,H,R,N); W_x, W_y (H,R,P) or None for ones."""
+    """S4: B, C (Bt,T,G,R,N); W_x, W_y (H,R,P) or None for ones."""
     Bt, T, H, P = x.shape
-    R, N = B.shape[-2], B.shape[-1]
-    y, hf, uf, af = _state_outs(x, N, P, out)
-    d = Dims(Bt, T, H, P, N, R, int(chunk))
+    R, N, G, K = B.shape[-2], B.shape[-1], B.shape[2], theta.shape[-1]
+    y, hf, uf, af = _state_outs(x, N, P, K, out)
+    d = Dims(Bt, T, H, P, N, R, int(chunk), G, K)
     dtype = _DTYPE[x.dtype]
     ws, nbytes = _workspace(M3_WS_MIMO, d, dtype, workspace, x.device)
     nptr, keep = _norm(norm)
@@ -243,11 +249,12 @@ def mimo_chunked_fwd(x, dt, A, lam, theta, B, C, D, chunk, W_x=None, W_y=None, n
 
 def step_decode(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, prevBx, angle, norm=None, y_out=None,
                 stream=None):
-    """S5: one decode step; h, prevBx, angle are updated in place; returns y_t (Bt,H,P)."""
+    """S5: one decode step; B_t, C_t (Bt,G,N); theta_t (Bt,H,K); h, prevBx, angle
+    are updated in place; returns y_t (Bt,H,P)."""
     Bt, H, P = x_t.shape
-    N = B_t.shape[-1]
+    N, G, K = B_t.shape[-1], B_t.shape[1], theta_t.shape[-1]
     y = torch.empty_like(x_t) if y_out is None else y_out
-    d = Dims(Bt, 1, H, P, N, 1, 1)
+    d = Dims(Bt, 1, H, P, N, 1, 1, G, K)
     nptr, keep = _norm(norm)
     _check(lib().m3_step_decode(_ptr(x_t), _ptr(dt_t), _ptr(A), _ptr(lam_t), _ptr(theta_t),
                                 _ptr(B_t), _ptr(C_t), _ptr(D), _DTYPE[x_t.dtype], nptr, d, _ptr(h),
@@ -259,11 +266,11 @@ def step_decode(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, prevBx, angle, nor
 def mimo_step_decode(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, prevBx, angle, W_x=None, W_y=None,
                      norm=None, y_out=None, stream=None):
     """S5 for rank R: one decode step on the full previous-input state.  B_t, C_t
-    (Bt,H,R,N); h, prevBx, angle updated in place; returns y_t (Bt,H,P)."""
+    (Bt,G,R,N); h, prevBx, angle updated in place; returns y_t (Bt,H,P)."""
     Bt, H, P = x_t.shape
-    R, N = B_t.shape[-2], B_t.shape[-1]
+    R, N, G, K = B_t.shape[-2], B_t.shape[-1], B_t.shape[1], theta_t.shape[-1]
     y = torch.empty_like(x_t) if y_out is None else y_out
-    d = Dims(Bt, 1, H, P, N, R, 1)
+    d = Dims(Bt, 1, H, P, N, R, 1, G, K)
     nptr, keep = _norm(norm)
     _check(lib().m3_mimo_step_decode(_ptr(x_t), _ptr(dt_t), _ptr(A), _ptr(lam_t), _ptr(theta_t), _ptr(B_t),
                                      _ptr(C_t), _ptr(D), _ptr(W_x), _ptr(W_y), _DTYPE[x_t.dtype], nptr, d,
@@ -275,12 +282,12 @@ def mimo_step_decode(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, prevBx, angle
 def step_decode_factored(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, b_prev, x_prev, angle, W_x=None,
                          W_y=None, norm=None, y_out=None, stream=None):
     """One decode step on the factored previous-input state (any rank; B_t, C_t
-    (Bt,H,R,N)).  h, b_prev (Bt,H,R,N), x_prev (Bt,H,P) and angle are updated in
+    (Bt,G,R,N)).  h, b_prev (Bt,H,R,N), x_prev (Bt,H,P) and angle are updated in
     place; returns y_t (Bt,H,P)."""
     Bt, H, P = x_t.shape
-    R, N = B_t.shape[-2], B_t.shape[-1]
+    R, N, G, K = B_t.shape[-2], B_t.shape[-1], B_t.shape[1], theta_t.shape[-1]
     y = torch.empty_like(x_t) if y_out is None else y_out
-    d = Dims(Bt, 1, H, P, N, R, 1)
+    d = Dims(Bt, 1, H, P, N, R, 1, G, K)
     nptr, keep = _norm(norm)
     _check(lib().m3_step_decode_factored(_ptr(x_t), _ptr(dt_t), _ptr(A), _ptr(lam_t), _ptr(theta_t),
                                          _ptr(B_t), _ptr(C_t), _ptr(D), _ptr(W_x), _ptr(W_y),

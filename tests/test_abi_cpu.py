@@ -47,9 +47,10 @@ MIS = 0x10004       # misaligned
 
 
 def dims(**kw):
-    base = dict(batch=2, seqlen=8, nheads=2, headdim=4, dstate=4, rank=1, chunk=4)
+    base = dict(batch=2, seqlen=8, nheads=2, headdim=4, dstate=4, rank=1, chunk=4, ngroups=0, rope_pairs=0)
     base.update(kw)
-    return m3.Dims(*[base[k] for k in ("batch", "seqlen", "nheads", "headdim", "dstate", "rank", "chunk")])
+    return m3.Dims(*[base[k] for k in ("batch", "seqlen", "nheads", "headdim", "dstate", "rank", "chunk",
+                                       "ngroups", "rope_pairs")])
 
 
 def siso(L, d, x=FAKE, dt=FAKE, A=FAKE, lam=FAKE, theta=FAKE, B=FAKE, C=FAKE, D=FAKE, dtype=m3.M3_BF16,
@@ -137,6 +138,38 @@ def test_rank_decode_validation(L):
     assert fact(dims(rank=1), bp=None) == m3.M3_ERR_INVALID_ARG        # the factored state needs b_prev
     assert fact(dims(rank=3), xp=MIS) == m3.M3_ERR_INVALID_ARG
     assert fact(dims(rank=3), Wy=MIS) == m3.M3_ERR_INVALID_ARG
+
+
+def test_groups_and_rope_pairs_validation(L):
+    """B/C groups must divide the heads; rotated pairs are 1..dstate/2; 0 means
+    the default (one group per head, every pair)."""
+    def rope(d):
+        return L.m3_rope_bc(FAKE, FAKE, m3.M3_BF16, FAKE, FAKE, None, None, d, FAKE, FAKE, None, None)
+
+    def step(d):
+        return L.m3_step_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, m3.M3_BF16, None, d,
+                                FAKE, FAKE, FAKE, FAKE, None)
+
+    def fact(d):
+        return L.m3_step_decode_factored(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, m3.M3_BF16,
+                                         None, d, FAKE, FAKE, FAKE, FAKE, FAKE, None)
+
+    base = dict(nheads=6, dstate=8)
+    for bad in (dict(ngroups=4), dict(ngroups=-1), dict(rope_pairs=5), dict(rope_pairs=-2)):
+        d = dims(**base, **bad)
+        assert siso(L, d) == m3.M3_ERR_INVALID_ARG, bad
+        assert rope(d) == m3.M3_ERR_INVALID_ARG, bad
+        assert step(d) == m3.M3_ERR_INVALID_ARG, bad
+        assert fact(d) == m3.M3_ERR_INVALID_ARG, bad
+    # valid groups and pairs get past the size checks (a null x then fails)
+    for ok in (dict(ngroups=1), dict(ngroups=3), dict(ngroups=6, rope_pairs=1), dict(rope_pairs=4)):
+        assert siso(L, dims(**base, **ok), x=None) == m3.M3_ERR_INVALID_ARG
+        assert m3.workspace_bytes(m3.M3_WS_SISO, dims(**base, **ok), m3.M3_BF16) == 0
+    long3 = dict(batch=1, seqlen=32768, nheads=32, headdim=64, dstate=128, chunk=128)
+    assert m3.workspace_bytes(m3.M3_WS_SISO, dims(**long3, ngroups=1, rope_pairs=32), m3.M3_BF16) > 0
+    # a pair count that is not a multiple of 4 runs on the FFMA path: no scratch
+    assert m3.workspace_bytes(m3.M3_WS_SISO, dims(**long3, ngroups=1, rope_pairs=30), m3.M3_BF16) == 0
+    assert m3.workspace_bytes(m3.M3_WS_SISO, dims(**long3, ngroups=5), m3.M3_BF16) == 0
 
 
 def test_workspace_query(L):
