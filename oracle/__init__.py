@@ -6,6 +6,6 @@ imports this package.
 """
 from .oracle import (  # noqa: F401
     build_oracle, discretize, rope_bc, siso_loop, mimo_loop, siso_chunked,
-    step_decode, mimo_step_decode, step_decode_factored, oracle_lib_path, oracle_source_path,
-    compile_source, use_library,
+    step_decode, mimo_step_decode, step_decode_factored, loop_bwd, GRAD_NAMES, oracle_lib_path,
+    oracle_source_path, compile_source, use_library,
 )

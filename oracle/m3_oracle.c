@@ -664,3 +664,280 @@ int m3o_step_decode_factored(const double *x, const double *dt, const double *A,
     free(tmp); free(Bb); free(Cb); free(Xr); free(Xp);
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Backward: the gradient of the scan's outputs with respect to every input */
+/* (training needs it: TorchMamba README, "Models" and "Verification";      */
+/* dotLLM pull request, the note that training is out of its scope).         */
+/*                                                                            */
+/* The loss is L = <dy, y> + <dh_final, h_{T-1}> + <dprevBx, U_{T-1}> +      */
+/* <dangle, Phi_{T-1}> (each seed may be NULL for zero).  This is the       */
+/* reverse sweep of the rank-R loop above, one lane at a time, with the     */
+/* forward values of the lane kept in memory:                                */
+/*   Gh_t  = adjoint of h_t = alpha_{t+1} Gh_{t+1} + sum_r C_rot_{t,r}        */
+/*           (W_y[r] dy_t)^T       (Gh_{T-1} starts from dh_final)          */
+/*   GU_t  = adjoint of U_t = gamma_t Gh_t + beta_{t+1} Gh_{t+1}             */
+/*           (dprevBx at t = T-1)                                            */
+/*   dalpha_t = <Gh_t, h_{t-1}>, dbeta_t = <Gh_t, U_{t-1}>,                 */
+/*   dgamma_t = <Gh_t, U_t>;  dh0 = alpha_0 Gh_0, dprevBx0 = beta_0 Gh_0;    */
+/*   a rotation by Phi turns the pair adjoint back by -Phi and adds          */
+/*   -dv[2i] v_rot[2i+1] + dv[2i+1] v_rot[2i] to the adjoint of Phi_t[i],     */
+/*   which flows unchanged to Phi_{t-1} and gives dtheta_t = dt_t GPhi_t,    */
+/*   ddt_t += <theta_t, GPhi_t>;  dangle0 = GPhi_0.                          */
+/* Every gradient buffer may be NULL (not wanted); the others are            */
+/* overwritten.  Shared parameters (A, D, W_x, W_y, the norm gains and       */
+/* biases, and grouped B/C rows) sum over the lanes that use them.           */
+/* ------------------------------------------------------------------------ */
+typedef struct {
+    double *dx, *ddt, *dA, *dlam, *dtheta, *dB, *dC, *dD, *dWx, *dWy;
+    double *dnormw_B, *dnormw_C, *dbias_B, *dbias_C;
+    double *dh0, *dprevBx0, *dangle0;
+} m3o_grads;
+
+static void zero_if(double *p, long n)
+{
+    if (p) memset(p, 0, sizeof(double) * (size_t)n);
+}
+
+/* adjoint of bc_prepare: dst = src * inv * w + bias (inv, w only with w) */
+static void bc_prepare_bwd(const double *src, long N, const double *w, double eps,
+                           const double *ddst, double *dsrc, double *dw, double *dbias)
+{
+    if (dbias)
+        for (long n = 0; n < N; n++) dbias[n] += ddst[n];
+    if (!w) {
+        for (long n = 0; n < N; n++) dsrc[n] += ddst[n];
+        return;
+    }
+    double ss = 0.0;
+    for (long n = 0; n < N; n++) ss += src[n] * src[n];
+    double inv = 1.0 / sqrt(ss / (double)N + eps);
+    double s = 0.0;  /* sum_n ddst[n] w[n] src[n] */
+    for (long n = 0; n < N; n++) {
+        s += ddst[n] * w[n] * src[n];
+        if (dw) dw[n] += ddst[n] * src[n] * inv;
+    }
+    for (long n = 0; n < N; n++)
+        dsrc[n] += inv * ddst[n] * w[n] - src[n] * inv * inv * inv * s / (double)N;
+}
+
+int m3o_mimo_loop_bwd(const double *x, const double *dt, const double *A,
+                      const double *lam, const double *theta, const double *B,
+                      const double *C, const double *D, const double *Wx,
+                      const double *Wy, const m3o_bcnorm *nrm, const double *h0,
+                      const double *prevBx0, const double *angle0, m3o_dims d,
+                      const double *dy, const double *dh_final,
+                      const double *dprevBx_final, const double *dangle_final,
+                      m3o_grads *g)
+{
+    if (check_dims(d, 1)) return -1;
+    if (!x || !dt || !A || !lam || !theta || !B || !C || !D || !g) return -1;
+    long Bt = d.batch, T = d.seqlen, H = d.nheads, P = d.headdim, N = d.dstate, R = d.rank;
+    long K = n_pairs(d), G = n_groups(d), NP = N * P;
+    long RN = R * N, RP = R * P;
+    zero_if(g->dx, Bt * T * H * P);
+    zero_if(g->ddt, Bt * T * H);
+    zero_if(g->dA, H);
+    zero_if(g->dlam, Bt * T * H);
+    zero_if(g->dtheta, Bt * T * H * K);
+    zero_if(g->dB, Bt * T * G * RN);
+    zero_if(g->dC, Bt * T * G * RN);
+    zero_if(g->dD, H);
+    zero_if(g->dWx, H * RP);
+    zero_if(g->dWy, H * RP);
+    zero_if(g->dnormw_B, N);
+    zero_if(g->dnormw_C, N);
+    zero_if(g->dbias_B, H * RN);
+    zero_if(g->dbias_C, H * RN);
+    zero_if(g->dh0, Bt * H * NP);
+    zero_if(g->dprevBx0, Bt * H * NP);
+    zero_if(g->dangle0, Bt * H * K);
+    double eps = nrm ? nrm->eps : 0.0;
+    const double *wB = nrm ? nrm->normw_B : NULL, *wC = nrm ? nrm->normw_C : NULL;
+
+    double *phis = (double *)malloc(sizeof(double) * (T + 1) * K);   /* Phi_{t-1}, t = 0..T */
+    double *Bp = (double *)malloc(sizeof(double) * (T * RN + 1));    /* QkNorm'd + bias'd */
+    double *Cp = (double *)malloc(sizeof(double) * (T * RN + 1));
+    double *Bb = (double *)malloc(sizeof(double) * (T * RN + 1));    /* rotated */
+    double *Cb = (double *)malloc(sizeof(double) * (T * RN + 1));
+    double *X = (double *)malloc(sizeof(double) * (T * RP + 1));     /* W_x[r] x_t */
+    double *al = (double *)malloc(sizeof(double) * (T + 1));
+    double *be = (double *)malloc(sizeof(double) * (T + 1));
+    double *ga = (double *)malloc(sizeof(double) * (T + 1));
+    double *hs = (double *)malloc(sizeof(double) * (T + 1) * NP);    /* h_{t-1}, t = 0..T */
+    double *Ut = (double *)malloc(sizeof(double) * NP);
+    double *Um = (double *)malloc(sizeof(double) * NP);
+    double *Gh = (double *)malloc(sizeof(double) * NP);
+    double *GU = (double *)malloc(sizeof(double) * NP);
+    double *GUf = (double *)malloc(sizeof(double) * NP);
+    double *Gphi = (double *)malloc(sizeof(double) * K);
+    double *dBb = (double *)malloc(sizeof(double) * RN);
+    double *dCb = (double *)malloc(sizeof(double) * RN);
+    double *dBp = (double *)malloc(sizeof(double) * N);
+    double *dCp = (double *)malloc(sizeof(double) * N);
+    double *dX = (double *)malloc(sizeof(double) * RP);
+    double *tmp = (double *)malloc(sizeof(double) * N);
+
+    for (long b = 0; b < Bt; b++)
+        for (long h = 0; h < H; h++) {
+            long lane = b * H + h;
+            /* ---- forward, keeping what the reverse sweep needs ---- */
+            for (long i = 0; i < K; i++) phis[i] = angle0 ? angle0[lane * K + i] : 0.0;
+            for (long k = 0; k < NP; k++) hs[k] = h0 ? h0[lane * NP + k] : 0.0;
+            for (long k = 0; k < NP; k++) Um[k] = prevBx0 ? prevBx0[lane * NP + k] : 0.0;
+            for (long t = 0; t < T; t++) {
+                long bth = (b * T + t) * H + h;
+                double dl = dt[bth], lm = lam[bth];
+                al[t] = exp(dl * A[h]);
+                be[t] = (1.0 - lm) * dl * al[t];
+                ga[t] = lm * dl;
+                double *phi = phis + (t + 1) * K;
+                for (long i = 0; i < K; i++) phi[i] = phis[t * K + i] + dl * theta[bth * K + i];
+                for (long r = 0; r < R; r++) {
+                    long off = bc_off(d, b, t, h, r);
+                    bc_prepare(B + off, N, wB, nrm && nrm->bias_B ? nrm->bias_B + (h * R + r) * N : NULL, eps,
+                               Bp + (t * R + r) * N);
+                    bc_prepare(C + off, N, wC, nrm && nrm->bias_C ? nrm->bias_C + (h * R + r) * N : NULL, eps,
+                               Cp + (t * R + r) * N);
+                    rotate_pairs(Bp + (t * R + r) * N, phi, K, N, Bb + (t * R + r) * N);
+                    rotate_pairs(Cp + (t * R + r) * N, phi, K, N, Cb + (t * R + r) * N);
+                    for (long p = 0; p < P; p++)
+                        X[(t * R + r) * P + p] = (Wx ? Wx[(h * R + r) * P + p] : 1.0) * x[bth * P + p];
+                }
+                for (long n = 0; n < N; n++)
+                    for (long p = 0; p < P; p++) {
+                        double u = 0.0;
+                        for (long r = 0; r < R; r++) u += Bb[(t * R + r) * N + n] * X[(t * R + r) * P + p];
+                        hs[(t + 1) * NP + n * P + p] = al[t] * hs[t * NP + n * P + p] + be[t] * Um[n * P + p] +
+                                                       ga[t] * u;
+                        Ut[n * P + p] = u;
+                    }
+                memcpy(Um, Ut, sizeof(double) * NP);
+            }
+            /* ---- reverse sweep ---- */
+            for (long k = 0; k < NP; k++) {
+                Gh[k] = dh_final ? dh_final[lane * NP + k] : 0.0;
+                GUf[k] = dprevBx_final ? dprevBx_final[lane * NP + k] : 0.0;
+            }
+            for (long i = 0; i < K; i++) Gphi[i] = dangle_final ? dangle_final[lane * K + i] : 0.0;
+            for (long t = T - 1; t >= 0; t--) {
+                long bth = (b * T + t) * H + h;
+                double dl = dt[bth], lm = lam[bth];
+                const double *ht = hs + (t + 1) * NP, *hm = hs + t * NP;
+                const double *dyt = dy ? dy + bth * P : NULL;
+                const double *xt = x + bth * P;
+                /* y_t = sum_r W_y[r] (C_rot_{t,r}^T h_t) + D x_t */
+                for (long r = 0; r < R; r++)
+                    for (long n = 0; n < N; n++) dCb[r * N + n] = 0.0;
+                if (dyt) {
+                    for (long r = 0; r < R; r++) {
+                        const double *cb = Cb + (t * R + r) * N;
+                        for (long p = 0; p < P; p++) {
+                            double wy = Wy ? Wy[(h * R + r) * P + p] : 1.0;
+                            double yr = 0.0;
+                            for (long n = 0; n < N; n++) {
+                                yr += cb[n] * ht[n * P + p];
+                                Gh[n * P + p] += cb[n] * wy * dyt[p];
+                                dCb[r * N + n] += wy * dyt[p] * ht[n * P + p];
+                            }
+                            if (g->dWy) g->dWy[(h * R + r) * P + p] += dyt[p] * yr;
+                        }
+                    }
+                    for (long p = 0; p < P; p++) {
+                        if (g->dD) g->dD[h] += dyt[p] * xt[p];
+                        if (g->dx) g->dx[bth * P + p] += D[h] * dyt[p];
+                    }
+                }
+                /* h_t = alpha h_{t-1} + beta U_{t-1} + gamma U_t */
+                double dal = 0.0, dbe = 0.0, dga = 0.0;
+                for (long n = 0; n < N; n++)
+                    for (long p = 0; p < P; p++) {
+                        double u = 0.0, um = 0.0;
+                        for (long r = 0; r < R; r++) {
+                            u += Bb[(t * R + r) * N + n] * X[(t * R + r) * P + p];
+                            if (t > 0) um += Bb[((t - 1) * R + r) * N + n] * X[((t - 1) * R + r) * P + p];
+                        }
+                        if (t == 0) um = prevBx0 ? prevBx0[lane * NP + n * P + p] : 0.0;
+                        double gh = Gh[n * P + p];
+                        dal += gh * hm[n * P + p];
+                        dbe += gh * um;
+                        dga += gh * u;
+                        GU[n * P + p] = ga[t] * gh + GUf[n * P + p];
+                    }
+                /* U_t = sum_r B_rot_{t,r} X_{t,r}^T */
+                for (long r = 0; r < R; r++) {
+                    const double *bb = Bb + (t * R + r) * N, *xr = X + (t * R + r) * P;
+                    for (long n = 0; n < N; n++) {
+                        double s = 0.0;
+                        for (long p = 0; p < P; p++) s += GU[n * P + p] * xr[p];
+                        dBb[r * N + n] = s;
+                    }
+                    for (long p = 0; p < P; p++) {
+                        double s = 0.0;
+                        for (long n = 0; n < N; n++) s += GU[n * P + p] * bb[n];
+                        dX[r * P + p] = s;
+                        double wx = Wx ? Wx[(h * R + r) * P + p] : 1.0;
+                        if (g->dx) g->dx[bth * P + p] += wx * s;
+                        if (g->dWx) g->dWx[(h * R + r) * P + p] += xt[p] * s;
+                    }
+                }
+                /* hand the state adjoints to step t-1 */
+                for (long k = 0; k < NP; k++) {
+                    GUf[k] = be[t] * Gh[k];
+                    Gh[k] = al[t] * Gh[k];
+                }
+                /* discretization: alpha = e^{dt A}, beta = (1-lam) dt alpha, gamma = lam dt */
+                double a = al[t];
+                if (g->ddt) g->ddt[bth] += dal * A[h] * a + dbe * (1.0 - lm) * (a + dl * A[h] * a) + dga * lm;
+                if (g->dA) g->dA[h] += dal * dl * a + dbe * (1.0 - lm) * dl * dl * a;
+                if (g->dlam) g->dlam[bth] += -dbe * dl * a + dga * dl;
+                /* rotation by Phi_t: angle adjoint and the un-rotated pair adjoints */
+                const double *phi = phis + (t + 1) * K;
+                for (long i = 0; i < K; i++) {
+                    double gp = 0.0;
+                    for (long r = 0; r < R; r++) {
+                        const double *bb = Bb + (t * R + r) * N, *cb = Cb + (t * R + r) * N;
+                        const double *db = dBb + r * N, *dc = dCb + r * N;
+                        gp += -db[2 * i] * bb[2 * i + 1] + db[2 * i + 1] * bb[2 * i];
+                        gp += -dc[2 * i] * cb[2 * i + 1] + dc[2 * i + 1] * cb[2 * i];
+                    }
+                    Gphi[i] += gp;
+                    if (g->dtheta) g->dtheta[bth * K + i] += dl * Gphi[i];
+                    if (g->ddt) g->ddt[bth] += theta[bth * K + i] * Gphi[i];
+                }
+                for (long r = 0; r < R; r++) {
+                    const double *db = dBb + r * N, *dc = dCb + r * N;
+                    for (long i = 0; i < K; i++) {
+                        double c = cos(phi[i]), s = sin(phi[i]);
+                        dBp[2 * i] = c * db[2 * i] + s * db[2 * i + 1];
+                        dBp[2 * i + 1] = -s * db[2 * i] + c * db[2 * i + 1];
+                        dCp[2 * i] = c * dc[2 * i] + s * dc[2 * i + 1];
+                        dCp[2 * i + 1] = -s * dc[2 * i] + c * dc[2 * i + 1];
+                    }
+                    for (long n = 2 * K; n < N; n++) {
+                        dBp[n] = db[n];
+                        dCp[n] = dc[n];
+                    }
+                    long off = bc_off(d, b, t, h, r);
+                    for (long n = 0; n < N; n++) tmp[n] = 0.0;
+                    bc_prepare_bwd(B + off, N, wB, eps, dBp, tmp, g->dnormw_B,
+                                   g->dbias_B && nrm && nrm->bias_B ? g->dbias_B + (h * R + r) * N : NULL);
+                    if (g->dB)
+                        for (long n = 0; n < N; n++) g->dB[off + n] += tmp[n];
+                    for (long n = 0; n < N; n++) tmp[n] = 0.0;
+                    bc_prepare_bwd(C + off, N, wC, eps, dCp, tmp, g->dnormw_C,
+                                   g->dbias_C && nrm && nrm->bias_C ? g->dbias_C + (h * R + r) * N : NULL);
+                    if (g->dC)
+                        for (long n = 0; n < N; n++) g->dC[off + n] += tmp[n];
+                }
+            }
+            /* the adjoints of the initial state: h_{-1} = h0, U_{-1} = prev_Bx0 */
+            if (g->dh0) memcpy(g->dh0 + lane * NP, Gh, sizeof(double) * NP);
+            if (g->dprevBx0) memcpy(g->dprevBx0 + lane * NP, GUf, sizeof(double) * NP);
+            if (g->dangle0) memcpy(g->dangle0 + lane * K, Gphi, sizeof(double) * K);
+        }
+    free(phis); free(Bp); free(Cp); free(Bb); free(Cb); free(X); free(al); free(be); free(ga);
+    free(hs); free(Ut); free(Um); free(Gh); free(GU); free(GUf); free(Gphi); free(dBb); free(dCb);
+    free(dBp); free(dCp); free(dX); free(tmp);
+    return 0;
+}

@@ -56,6 +56,14 @@ class _Dims(ctypes.Structure):
                 ("ngroups", ctypes.c_long), ("rope_pairs", ctypes.c_long)]
 
 
+GRAD_NAMES = ("dx", "ddt", "dA", "dlam", "dtheta", "dB", "dC", "dD", "dWx", "dWy",
+              "dnormw_B", "dnormw_C", "dbias_B", "dbias_C", "dh0", "dprevBx0", "dangle0")
+
+
+class _Grads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in GRAD_NAMES]
+
+
 class _Norm(ctypes.Structure):
     _fields_ = [("normw_B", ctypes.c_void_p), ("normw_C", ctypes.c_void_p),
                 ("bias_B", ctypes.c_void_p), ("bias_C", ctypes.c_void_p),
@@ -65,7 +73,8 @@ class _Norm(ctypes.Structure):
 def _open(path):
     lib = ctypes.CDLL(path)
     for name in ("m3o_discretize", "m3o_rope_bc", "m3o_siso_loop", "m3o_mimo_loop",
-                 "m3o_siso_chunked", "m3o_step_decode", "m3o_mimo_step_decode", "m3o_step_decode_factored"):
+                 "m3o_siso_chunked", "m3o_step_decode", "m3o_mimo_step_decode", "m3o_step_decode_factored",
+                 "m3o_mimo_loop_bwd"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -270,3 +279,37 @@ def step_decode_factored(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, bprev, xp
     if rc < 0:
         raise ValueError("oracle rejected the arguments")
     return y, h, bprev, xprev, angle
+
+
+def loop_bwd(x, dt, A, lam, theta, B, C, D, dy=None, Wx=None, Wy=None, h0=None, prevBx0=None,
+             angle0=None, norm=None, dh=None, dprevBx=None, dangle=None):
+    """Gradients of L = <dy, y> + <dh, h_final> + <dprevBx, prevBx_final> +
+    <dangle, angle_final> with respect to every input of the scan (SISO when B
+    is (Bt,T,G,N), rank R when it is (Bt,T,G,R,N)).  Returns a dict keyed by
+    GRAD_NAMES (dWx, dWy are the gradients for all-ones vectors when Wx, Wy
+    are None; the norm entries are None when that part of the norm is off)."""
+    x, dt, A, lam, theta, B, C, D = (_f64(a) for a in (x, dt, A, lam, theta, B, C, D))
+    Wx, Wy, h0, prevBx0, angle0 = (_f64(a) for a in (Wx, Wy, h0, prevBx0, angle0))
+    dy, dh, dprevBx, dangle = (_f64(a) for a in (dy, dh, dprevBx, dangle))
+    Bt, T, H, P = x.shape
+    R = B.shape[3] if B.ndim == 5 else 1
+    N, G, K = B.shape[-1], B.shape[2], theta.shape[-1]
+    shapes = dict(dx=x.shape, ddt=dt.shape, dA=(H,), dlam=lam.shape, dtheta=theta.shape, dB=B.shape,
+                  dC=C.shape, dD=(H,), dWx=(H, R, P), dWy=(H, R, P), dnormw_B=(N,), dnormw_C=(N,),
+                  dbias_B=(H, R, N), dbias_C=(H, R, N), dh0=(Bt, H, N, P), dprevBx0=(Bt, H, N, P),
+                  dangle0=(Bt, H, K))
+    out = {k: np.zeros(v) for k, v in shapes.items()}
+    nm = norm or {}
+    for k, key in (("dnormw_B", "normw_B"), ("dnormw_C", "normw_C"), ("dbias_B", "bias_B"),
+                   ("dbias_C", "bias_C")):
+        if nm.get(key) is None:
+            out[k] = None
+    g = _Grads(*[_p(out[k]) for k in GRAD_NAMES])
+    nptr, keep = _norm(norm)
+    rc = _load().m3o_mimo_loop_bwd(_p(x), _p(dt), _p(A), _p(lam), _p(theta), _p(B), _p(C), _p(D), _p(Wx),
+                                   _p(Wy), nptr, _p(h0), _p(prevBx0), _p(angle0),
+                                   _dims(Bt, T, H, P, N, R, G, K), _p(dy), _p(dh), _p(dprevBx), _p(dangle),
+                                   ctypes.byref(g))
+    if rc < 0:
+        raise ValueError("oracle rejected the arguments")
+    return out

@@ -10,6 +10,7 @@ import os
 import numpy as np
 import pytest
 
+import test_oracle_grad_pins as gpins
 import test_oracle_pins as pins
 
 MUTATIONS = [
@@ -35,6 +36,17 @@ MUTATIONS = [
      "for (long n = 2 * K; n < N; n++) out[n] = 0.0;"),
     ("partial RoPE rotates the last pairs", "double v0 = v[2 * i], v1 = v[2 * i + 1];\n        out[2 * i] = c * v0 - s * v1;\n        out[2 * i + 1] = s * v0 + c * v1;\n    }\n    for (long n = 2 * K; n < N; n++) out[n] = v[n];",
      "long j = i + N / 2 - K;\n        double v0 = v[2 * j], v1 = v[2 * j + 1];\n        out[2 * j] = c * v0 - s * v1;\n        out[2 * j + 1] = s * v0 + c * v1;\n    }\n    for (long n = 0; n < N - 2 * K; n++) out[n] = v[n];"),
+    ("backward: beta adjoint from U_t", "dbe += gh * um;", "dbe += gh * u;"),
+    ("backward: state adjoint not decayed", "Gh[k] = al[t] * Gh[k];", "Gh[k] = Gh[k];"),
+    ("backward: angle adjoint sign", "gp += -db[2 * i] * bb[2 * i + 1] + db[2 * i + 1] * bb[2 * i];",
+     "gp += db[2 * i] * bb[2 * i + 1] - db[2 * i + 1] * bb[2 * i];"),
+    ("backward: pair adjoint rotated forward", "dBp[2 * i] = c * db[2 * i] + s * db[2 * i + 1];",
+     "dBp[2 * i] = c * db[2 * i] - s * db[2 * i + 1];"),
+    ("backward: QkNorm adjoint without the RMS term",
+     "dsrc[n] += inv * ddst[n] * w[n] - src[n] * inv * inv * inv * s / (double)N;",
+     "dsrc[n] += inv * ddst[n] * w[n];"),
+    ("backward: lookahead adjoint dropped", "GU[n * P + p] = ga[t] * gh + GUf[n * P + p];",
+     "GU[n * P + p] = ga[t] * gh;"),
 ]
 
 PIN_CASES = [
@@ -50,6 +62,8 @@ PIN_CASES = [
     lambda o: pins.test_mimo_decode_steps_equal_mimo_loop(o),
     lambda o: pins.test_grouped_partial_siso(o, 2, 1),
     lambda o: pins.test_partial_rope_turns_only_first_pairs(o),
+    lambda o: gpins.test_siso_grad_matches_finite_differences(2),
+    lambda o: gpins.test_siso_grad_norm_bias_groups_partial(),
 ]
 
 
