@@ -173,13 +173,16 @@ def traffic_record(key, src_paths):
 # ---------------------------------------------------------------------------
 def scan_bytes(c):
     """Algorithmic bytes of one chunked-scan call: every input once, every
-    output once, plus the final states (h, prev_Bx, angle)."""
+    output once, plus the final states (h, prev_Bx, angle).  B and C are read
+    once per group (G groups, K rotated pairs)."""
     Bt, T, H, P, N, R = c["batch"], c["seqlen"], c["nheads"], c["headdim"], c["dstate"], c["rank"]
+    G, K = c.get("ngroups", 0) or H, c.get("rope_pairs", 0) or N // 2
     es = 2 if c["dtype"] == "bf16" else 4
-    per_token_head = es * P + 2 * es * R * N + 4 + 4 + 4 * (N // 2) + es * P
-    states = Bt * H * (2 * N * P * 4 + (N // 2) * 4)
+    per_token_head = es * P + 4 + 4 + 4 * K + es * P
+    per_token_group = 2 * es * R * N
+    states = Bt * H * (2 * N * P * 4 + K * 4)
     params = H * 8 + (2 * H * R * P * 4 if R > 1 else 0)
-    return Bt * T * H * per_token_head + states + params
+    return Bt * T * (H * per_token_head + G * per_token_group) + states + params
 
 
 def scan_flops(c):
@@ -220,11 +223,12 @@ class ScanWorkload:
         self.host.pop("generator")
         self.dev = {k: v.to(device) for k, v in self.host.items() if isinstance(v, torch.Tensor)}
         Bt, T, H, P, N = c["batch"], c["seqlen"], c["nheads"], c["headdim"], c["dstate"]
+        self.G, self.K = c.get("ngroups", 0) or H, c.get("rope_pairs", 0) or N // 2
         self.out = (torch.empty(Bt, T, H, P, device=device, dtype=self.dev["x"].dtype),
                     torch.empty(Bt, H, N, P, device=device), torch.empty(Bt, H, N, P, device=device),
-                    torch.empty(Bt, H, N // 2, device=device))
+                    torch.empty(Bt, H, self.K, device=device))
         self.mimo = c["rank"] > 1
-        d = self.m3.Dims(Bt, T, H, P, N, c["rank"], c["chunk"])
+        d = self.m3.Dims(Bt, T, H, P, N, c["rank"], c["chunk"], self.G, self.K)
         which = self.m3.M3_WS_MIMO if self.mimo else self.m3.M3_WS_SISO
         nws = self.m3.workspace_bytes(which, d, self.m3.M3_BF16 if c["dtype"] == "bf16" else self.m3.M3_F32)
         self.ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=device)
@@ -232,7 +236,7 @@ class ScanWorkload:
         self.bytes = scan_bytes(c)
         self.flops = scan_flops(c)
         tc = (c["dtype"] == "bf16" and c["rank"] in (1, 2, 4) and c["headdim"] == 64 and c["dstate"] == 128
-              and c["chunk"] % (64 // c["rank"]) == 0)
+              and c["chunk"] % (64 // c["rank"]) == 0 and self.K % 4 == 0)
         self.kernel = "k_scan_tc" if tc else "k_scan_simt"
         self.srcs = [os.path.join(ROOT, "state_space_lm_b200", "csrc", self.kernel + ".cu")]
         # long sequences over few lanes run as three launches (state-only pass,
@@ -255,6 +259,7 @@ class ScanWorkload:
         c = self.c
         return {"workload": c["name"], "batch": c["batch"], "seqlen": c["seqlen"], "nheads": c["nheads"],
                 "headdim": c["headdim"], "dstate": c["dstate"], "rank": c["rank"], "chunk": c["chunk"],
+                "ngroups": self.G, "rope_pairs": self.K,
                 "inputs": "x/B/C %s, dt/lam/theta/A/D fp32, seeded synthetic" % c["dtype"],
                 "l2": "inputs larger than L2 (%.0f MB vs 126 MB), no flush" % (self.input_bytes / 1e6)}
 
@@ -272,6 +277,11 @@ class ScanWorkload:
         for k in keys:
             v = self.host[k]
             arr[k] = gen.to_f64(v[hs[0]:hs[-1] + 1] if k in ("A", "D") else sl(v))
+        if self.G != H:   # the sampled heads' B/C rows, one per head
+            hpg = H // self.G
+            for k in ("B", "C"):
+                v = self.host[k][bs[0]:bs[-1] + 1]
+                arr[k] = gen.to_f64(torch.stack([v[:, :, h // hpg] for h in range(hs[0], hs[-1] + 1)], 2))
         nl = len(bs) * len(hs)
         t0 = time.perf_counter()
         if self.mimo:
@@ -391,7 +401,7 @@ def run_ours(args, world, rank, local):
     from state_space_lm_b200 import build, m3
     if not os.path.exists(build.LIB):
         raise SystemExit("CUDA library not built: run python -m state_space_lm_b200.build")
-    if args.config >= 4:
+    if "steps" in gen.CONFIGS[args.config]:      # the decode workloads
         w = DecodeWorkload(args.config, device, args.steps + args.warmup)
     else:
         w = ScanWorkload(args.config, device)
@@ -512,6 +522,8 @@ def run_reference(args, world, rank):
     w.host = gen.config_inputs(args.config)
     w.host.pop("generator")
     w.mimo = w.c["rank"] > 1
+    w.G = w.c.get("ngroups", 0) or w.c["nheads"]
+    w.K = w.c.get("rope_pairs", 0) or w.c["dstate"] // 2
     cores = os.cpu_count() or 1
     H = w.c["nheads"]
     total_lanes = w.c["batch"] * H
@@ -546,7 +558,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=1, choices=[0, 1, 2, 3, 4, 5, 6])
+    ap.add_argument("--config", type=int, default=1, choices=[0, 1, 2, 3, 4, 5, 6, 7])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -44,6 +44,10 @@ CONFIGS = {
     6: dict(name="decode_factored_mimo_r4_512xh16_p64_n128", batch=512, seqlen=256, nheads=16,
             headdim=64, dstate=128, rank=4, chunk=64, dtype="bf16", dt_shift=-2.0, steps=1024,
             state="factored"),
+    # one B/C group shared by all heads and 32 rotated pairs of 64 (the 370M
+    # checkpoint's n_groups 1 and rope fraction 0.5), default workload's shape
+    7: dict(name="siso_g1_rope32_8x2048_h16_p64_n128", batch=8, seqlen=2048, nheads=16, headdim=64,
+            dstate=128, rank=1, chunk=64, dtype="bf16", dt_shift=-2.0, ngroups=1, rope_pairs=32),
 }
 
 _DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}
@@ -131,15 +135,16 @@ def decode_step_inputs(generator, batch, nheads, headdim, dstate, dtype="bf16",
 
 
 def config_inputs(idx, seed=None, **overrides):
-    """Inputs of workload ``idx`` (0-3: one chunked-scan call; 4-6: the prefill
-    of a decode workload -- its steps come from ``decode_step_inputs`` with the
-    returned generator)."""
+    """Inputs of workload ``idx`` (0-3 and 7: one chunked-scan call; 4-6: the
+    prefill of a decode workload -- its steps come from ``decode_step_inputs``
+    with the returned generator)."""
     c = dict(CONFIGS[idx])
     c.update(overrides)
     s = SEED_BASE + idx if seed is None else seed
     return scan_inputs(c["batch"], c["seqlen"], c["nheads"], c["headdim"], c["dstate"],
                        rank=c["rank"], dtype=c["dtype"], dt_shift=c["dt_shift"], seed=s,
-                       mimo_weights=c["rank"] > 1)
+                       mimo_weights=c["rank"] > 1, ngroups=c.get("ngroups", 0),
+                       rope_pairs=c.get("rope_pairs", 0))
 
 
 def to_f64(t):
