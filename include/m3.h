@@ -213,6 +213,40 @@ m3_status m3_step_decode_factored(const void *x_t, const float *dt_t, const floa
                                   m3_dims d, float *h, float *b_prev, float *x_prev,
                                   float *angle, void *y_t, void *stream);
 
+/* Gradients of the chunked scan, each fp32 with the shape of its input
+ * (dx like x; dB, dC like B, C: (batch, seqlen, ngroups, [rank,] dstate);
+ * dnormw_* (dstate); dbias_* (nheads, rank, dstate); dh0, dprevBx0 like
+ * h0; dangle0 (batch, nheads, K)).  Any pointer may be NULL (not wanted);
+ * the others are overwritten. */
+typedef struct {
+    float *dx, *ddt, *dA, *dlam, *dtheta, *dB, *dC, *dD, *dW_x, *dW_y;
+    float *dnormw_B, *dnormw_C, *dbias_B, *dbias_C;
+    float *dh0, *dprevBx0, *dangle0;
+} m3_grads;
+
+/* Backward of the chunked forward (SISO when d.rank <= 1 and W_x, W_y are
+ * NULL; rank-R MIMO otherwise, with B, C carrying the rank axis).  Training
+ * needs it (TorchMamba README, "Models" and "Verification"); the forward is
+ * m3_siso_chunked_fwd / m3_mimo_chunked_fwd on the same arguments.
+ * For the loss L = <dy, y> + <dh_final, h_final> + <dprevBx_final,
+ * prevBx_final> + <dangle_final, angle_final> it writes dL/d(input) for every
+ * input into `grads`.  dy (batch, seqlen, nheads, headdim) has the dtype of
+ * x and is required when seqlen > 0; the three state adjoints are fp32 in
+ * the shapes of the forward's final states, each NULL for zero.
+ * The gradients are computed in fp32 on the FFMA pipes, recomputing the
+ * forward chunk by chunk from entering states kept in the workspace; every
+ * sum runs in a fixed order, so repeated calls give identical bits.
+ * workspace: at least m3_workspace_bytes(M3_WS_BWD_SISO or M3_WS_BWD_MIMO,
+ * d, dtype) bytes. */
+m3_status m3_chunked_bwd(const void *x, const float *dt, const float *A, const float *lam,
+                         const float *theta, const void *B, const void *C, const float *D,
+                         const float *W_x, const float *W_y, m3_dtype dtype,
+                         const m3_bcnorm *norm, const float *h0, const float *prevBx0,
+                         const float *angle0, m3_dims d, const void *dy,
+                         const float *dh_final, const float *dprevBx_final,
+                         const float *dangle_final, const m3_grads *grads, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
 /* Size in bytes of the scratch buffer built into the library for
  * m3_siso_chunked_fwd_noalloc (32 MiB). */
 #define M3_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
@@ -249,7 +283,7 @@ m3_status m3_siso_chunked_fwd_noalloc(const void *x, const float *dt, const floa
                                       float *angle_final, void *stream);
 
 /* Workspace query for the chunked forwards. */
-enum { M3_WS_SISO = 0, M3_WS_MIMO = 1 };
+enum { M3_WS_SISO = 0, M3_WS_MIMO = 1, M3_WS_BWD_SISO = 2, M3_WS_BWD_MIMO = 3 };
 size_t m3_workspace_bytes(int which, m3_dims d, m3_dtype dtype);
 
 /* Static description of a status code (never NULL). */

@@ -150,6 +150,14 @@ m3_status m3_device_error(void *stream, int *site) {
 }
 
 size_t m3_workspace_bytes(int which, m3_dims d, m3_dtype dtype) {
+    if (which == M3_WS_BWD_SISO || which == M3_WS_BWD_MIMO) {
+        BwdArgs b{};
+        if (check_core_dims(d, true) != M3_OK || d.chunk < 1 || resolve_groups(d, b.G, b.K) != M3_OK) return 0;
+        b.Bt = d.batch; b.T = d.seqlen; b.H = d.nheads; b.P = d.headdim; b.N = d.dstate;
+        b.R = which == M3_WS_BWD_MIMO ? (d.rank > 1 ? d.rank : 1) : 1;
+        b.Q = (int)(d.chunk < 64 ? d.chunk : 64);
+        return scan_bwd_workspace_bytes(b);
+    }
     // only the tensor-core path uses scratch (long sequences over few lanes)
     if ((which != M3_WS_SISO && which != M3_WS_MIMO) || check_core_dims(d, true) != M3_OK || d.chunk < 1) return 0;
     ScanArgs a{};
@@ -289,6 +297,56 @@ m3_status m3_step_decode_factored(const void *x_t, const float *dt_t, const floa
                                   void *stream) {
     return decode_gen(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, W_x, W_y, dtype, norm, d, h, nullptr, b_prev,
                       x_prev, angle, y_t, stream, true);
+}
+
+m3_status m3_chunked_bwd(const void *x, const float *dt, const float *A, const float *lam, const float *theta,
+                         const void *B, const void *C, const float *D, const float *W_x, const float *W_y,
+                         m3_dtype dtype, const m3_bcnorm *norm, const float *h0, const float *prevBx0,
+                         const float *angle0, m3_dims d, const void *dy, const float *dh_final,
+                         const float *dprevBx_final, const float *dangle_final, const m3_grads *grads,
+                         void *workspace, size_t workspace_bytes, void *stream) {
+    m3_status st;
+    if ((st = check_dtype(dtype)) != M3_OK) return st;
+    if ((st = check_core_dims(d, true)) != M3_OK) return st;
+    if (d.chunk < 1 || d.rank < 0 || !grads) return M3_ERR_INVALID_ARG;
+    int64_t G, K;
+    if ((st = resolve_groups(d, G, K)) != M3_OK) return st;
+    const bool mimo = d.rank > 1 || W_x || W_y;
+    const int64_t R = d.rank > 1 ? d.rank : 1;
+    if (R > kMaxRank) return M3_ERR_UNSUPPORTED;
+    M3_REQ(A); M3_REQ(D);
+    const bool have_tokens = d.batch > 0 && d.seqlen > 0;
+    if (have_tokens) {
+        M3_REQ(x); M3_REQ(dt); M3_REQ(lam); M3_REQ(theta); M3_REQ(B); M3_REQ(C); M3_REQ(dy);
+    } else {
+        M3_OPT(x); M3_OPT(dt); M3_OPT(lam); M3_OPT(theta); M3_OPT(B); M3_OPT(C); M3_OPT(dy);
+    }
+    M3_OPT(W_x); M3_OPT(W_y); M3_OPT(h0); M3_OPT(prevBx0); M3_OPT(angle0);
+    M3_OPT(dh_final); M3_OPT(dprevBx_final); M3_OPT(dangle_final); M3_OPT(workspace);
+    const m3_grads &g = *grads;
+    M3_OPT(g.dx); M3_OPT(g.ddt); M3_OPT(g.dA); M3_OPT(g.dlam); M3_OPT(g.dtheta); M3_OPT(g.dB); M3_OPT(g.dC);
+    M3_OPT(g.dD); M3_OPT(g.dW_x); M3_OPT(g.dW_y); M3_OPT(g.dnormw_B); M3_OPT(g.dnormw_C); M3_OPT(g.dbias_B);
+    M3_OPT(g.dbias_C); M3_OPT(g.dh0); M3_OPT(g.dprevBx0); M3_OPT(g.dangle0);
+    NormArgs nrm;
+    if ((st = read_norm(norm, nrm)) != M3_OK) return st;
+    BwdArgs a{};
+    a.x = x; a.B = B; a.C = C; a.dy = dy;
+    a.dt = dt; a.A = A; a.lam = lam; a.theta = theta; a.D = D; a.Wx = W_x; a.Wy = W_y;
+    a.h0 = h0; a.prevBx0 = prevBx0; a.angle0 = angle0;
+    a.dh = dh_final; a.du = dprevBx_final; a.da = dangle_final;
+    a.nrm = nrm;
+    a.dx = g.dx; a.ddt = g.ddt; a.dA = g.dA; a.dlam = g.dlam; a.dtheta = g.dtheta; a.dB = g.dB; a.dC = g.dC;
+    a.dD = g.dD; a.dWx = g.dW_x; a.dWy = g.dW_y; a.dwB = g.dnormw_B; a.dwC = g.dnormw_C; a.dbB = g.dbias_B;
+    a.dbC = g.dbias_C; a.dh0 = g.dh0; a.du0 = g.dprevBx0; a.da0 = g.dangle0;
+    a.Bt = d.batch; a.T = d.seqlen; a.H = d.nheads; a.P = d.headdim; a.N = d.dstate; a.R = R; a.G = G; a.K = K;
+    const int q = bwd_chunk(a.P, a.N, R, K, d.chunk);
+    if (q < 1) return M3_ERR_UNSUPPORTED;
+    const size_t need = m3_workspace_bytes(mimo ? M3_WS_BWD_MIMO : M3_WS_BWD_SISO, d, dtype);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return M3_ERR_WORKSPACE;
+    a.Q = q;
+    a.ws = static_cast<float *>(workspace);
+    if (d.batch == 0) return M3_OK;
+    return launched(launch_scan_bwd(a, dtype, (cudaStream_t)stream));
 }
 
 }  // extern "C"

@@ -71,6 +71,20 @@ struct RopeArgs {
     int64_t G = 0, K = 0;  // B/C groups and rotated pairs, resolved
 };
 
+struct BwdArgs {
+    const void *x, *B, *C, *dy;
+    const float *dt, *A, *lam, *theta, *D, *Wx, *Wy;
+    const float *h0, *prevBx0, *angle0;
+    const float *dh, *du, *da;     // adjoints of h_final, prevBx_final, angle_final (NULL = 0)
+    NormArgs nrm;
+    // gradients (each NULL = not wanted), fp32
+    float *dx, *ddt, *dA, *dlam, *dtheta, *dB, *dC, *dD, *dWx, *dWy, *dwB, *dwC, *dbB, *dbC, *dh0, *du0, *da0;
+    int64_t Bt, T, H, P, N, R, G, K;
+    int Q;                          // chunk length used by the backward kernels
+    float *ws;                      // caller's workspace
+    size_t ws_slots = 0, ws_partial = 0, ws_dBh = 0, ws_dCh = 0;   // offsets (floats), set by the launcher
+};
+
 // Host launchers (each returns cudaSuccess or the launch error).
 cudaError_t launch_discretize(const float *dt, const float *A, const float *lam, int64_t Bt,
                               int64_t T, int64_t H, float *al, float *be, float *ga,
@@ -87,6 +101,11 @@ bool scan_tc_supported(const ScanArgs &a, m3_dtype dt);
 cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s);
 int scan_tc_error_and_clear(cudaStream_t s);
 size_t scan_tc_workspace_bytes(int64_t Bt, int64_t H, int64_t T);
+
+// backward of the chunked scan (FFMA): chunk length that fits, workspace, launch
+int bwd_chunk(int64_t P, int64_t N, int64_t R, int64_t K, int64_t chunk);
+size_t scan_bwd_workspace_bytes(const BwdArgs &a);
+cudaError_t launch_scan_bwd(const BwdArgs &a, m3_dtype dt, cudaStream_t s);
 
 // Launch counter shared by all launchers.
 void count_launch(int n = 1);

@@ -15,7 +15,7 @@ from .build import LIB
 
 M3_OK, M3_ERR_INVALID_ARG, M3_ERR_UNSUPPORTED, M3_ERR_WORKSPACE, M3_ERR_CUDA, M3_ERR_TIMEOUT = range(6)
 M3_F32, M3_BF16 = 0, 1
-M3_WS_SISO, M3_WS_MIMO = 0, 1
+M3_WS_SISO, M3_WS_MIMO, M3_WS_BWD_SISO, M3_WS_BWD_MIMO = 0, 1, 2, 3
 
 _DTYPE = {torch.float32: M3_F32, torch.bfloat16: M3_BF16}
 
@@ -23,8 +23,11 @@ ABI_FUNCTIONS = (
     "m3_get_limits", "m3_discretize", "m3_rope_bc", "m3_siso_chunked_fwd",
     "m3_mimo_chunked_fwd", "m3_step_decode", "m3_workspace_bytes", "m3_status_string",
     "m3_launch_count", "m3_device_error", "m3_siso_chunked_fwd_noalloc", "m3_mimo_step_decode",
-    "m3_step_decode_factored",
+    "m3_step_decode_factored", "m3_chunked_bwd",
 )
+
+GRAD_FIELDS = ("dx", "ddt", "dA", "dlam", "dtheta", "dB", "dC", "dD", "dW_x", "dW_y",
+               "dnormw_B", "dnormw_C", "dbias_B", "dbias_C", "dh0", "dprevBx0", "dangle0")
 
 
 class M3Error(RuntimeError):
@@ -45,6 +48,10 @@ class BcNorm(ctypes.Structure):
     _fields_ = [("normw_B", ctypes.c_void_p), ("normw_C", ctypes.c_void_p),
                 ("bias_B", ctypes.c_void_p), ("bias_C", ctypes.c_void_p),
                 ("eps", ctypes.c_float)]
+
+
+class Grads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in GRAD_FIELDS]
 
 
 class Limits(ctypes.Structure):
@@ -101,6 +108,10 @@ def lib():
                                       ctypes.POINTER(BcNorm), Dims, _VP, _VP, _VP, _VP, _VP]
     L.m3_step_decode_factored.argtypes = [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int,
                                           ctypes.POINTER(BcNorm), Dims, _VP, _VP, _VP, _VP, _VP, _VP]
+    L.m3_chunked_bwd.restype = ctypes.c_int
+    L.m3_chunked_bwd.argtypes = [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int,
+                                 ctypes.POINTER(BcNorm), _VP, _VP, _VP, Dims, _VP, _VP, _VP, _VP,
+                                 ctypes.POINTER(Grads), _VP, ctypes.c_size_t, _VP]
     _lib = L
     return L
 
@@ -295,3 +306,38 @@ def step_decode_factored(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, b_prev, x
                                          _ptr(angle), _ptr(y), _stream(stream)),
            "m3_step_decode_factored")
     return y
+
+
+def chunked_bwd(x, dt, A, lam, theta, B, C, D, dy, chunk, W_x=None, W_y=None, norm=None, h0=None,
+                prevBx0=None, angle0=None, dh_final=None, dprevBx_final=None, dangle_final=None,
+                want=None, workspace=None, stream=None):
+    """Backward of the chunked forward: returns a dict of fp32 gradients (the
+    names in ``want``, by default all of them, without dW_x and dW_y for SISO;
+    the gain and bias entries only when that part of the norm is on).  B, C
+    (Bt,T,G,N) for SISO or (Bt,T,G,R,N) for rank R; dy has x's shape and dtype;
+    the state adjoints default to zero."""
+    Bt, T, H, P = x.shape
+    R = B.shape[3] if B.dim() == 5 else 1
+    N, G, K = B.shape[-1], B.shape[2], theta.shape[-1]
+    mimo = B.dim() == 5
+    if want is None:
+        want = tuple(k for k in GRAD_FIELDS if mimo or k not in ("dW_x", "dW_y"))
+    dev = x.device
+    shapes = dict(dx=x.shape, ddt=dt.shape, dA=A.shape, dlam=lam.shape, dtheta=theta.shape, dB=B.shape,
+                  dC=C.shape, dD=D.shape, dW_x=(H, R, P), dW_y=(H, R, P), dnormw_B=(N,), dnormw_C=(N,),
+                  dbias_B=(H, R, N), dbias_C=(H, R, N), dh0=(Bt, H, N, P), dprevBx0=(Bt, H, N, P),
+                  dangle0=(Bt, H, K))
+    nm = norm or {}
+    off = {"dnormw_B": "normw_B", "dnormw_C": "normw_C", "dbias_B": "bias_B", "dbias_C": "bias_C"}
+    out = {k: torch.empty(shapes[k], device=dev, dtype=torch.float32) for k in want
+           if k not in off or nm.get(off[k]) is not None}
+    g = Grads(*[_ptr(out.get(k)) for k in GRAD_FIELDS])
+    d = Dims(Bt, T, H, P, N, R if mimo else 1, int(chunk), G, K)
+    dtype = _DTYPE[x.dtype]
+    ws, nbytes = _workspace(M3_WS_BWD_MIMO if mimo else M3_WS_BWD_SISO, d, dtype, workspace, dev)
+    nptr, keep = _norm(norm)
+    _check(lib().m3_chunked_bwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(lam), _ptr(theta), _ptr(B), _ptr(C), _ptr(D),
+                                _ptr(W_x), _ptr(W_y), dtype, nptr, _ptr(h0), _ptr(prevBx0), _ptr(angle0), d,
+                                _ptr(dy), _ptr(dh_final), _ptr(dprevBx_final), _ptr(dangle_final),
+                                ctypes.byref(g), _ptr(ws), nbytes, _stream(stream)), "m3_chunked_bwd")
+    return out
