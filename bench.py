@@ -294,6 +294,90 @@ class ScanWorkload:
         return nl, dt, used
 
 
+def bwd_bytes(c):
+    """Algorithmic bytes of one backward call: the forward's inputs and dy read
+    once, every gradient written once (fp32), the initial-state gradients and
+    the shared parameters' gradients."""
+    Bt, T, H, P, N, R = c["batch"], c["seqlen"], c["nheads"], c["headdim"], c["dstate"], c["rank"]
+    G, K = c.get("ngroups", 0) or H, c.get("rope_pairs", 0) or N // 2
+    es = 2 if c["dtype"] == "bf16" else 4
+    per_token_head = 2 * es * P + 8 + 4 * K + (4 * P + 8 + 4 * K)
+    per_token_group = 2 * es * R * N + 2 * 4 * R * N
+    states = Bt * H * (2 * N * P * 4 + K * 4)
+    params = H * 8 * 2 + (4 * H * R * P * 4 if R > 1 else 0)
+    return Bt * T * (H * per_token_head + G * per_token_group) + states + params
+
+
+def bwd_flops(c):
+    """Causal flops of the chunked backward at the workload's chunk Q: per chunk
+    12 Q R N P (the entering-state pass and the five chunk-by-state products)
+    plus 2 pairs R^2 (3N + 2P) for the masked score products (+ 2 pairs R^2 P
+    for the MIMO output when W_y's gradient is wanted)."""
+    Bt, T, H, P, N, R, Q = (c["batch"], c["seqlen"], c["nheads"], c["headdim"], c["dstate"], c["rank"],
+                            c["chunk"])
+    total = 0
+    for t0 in range(0, T, Q):
+        L = min(Q, T - t0)
+        pairs = L * (L + 1) // 2
+        total += 12 * L * R * N * P + 2 * pairs * R * R * (3 * N + 2 * P + (P if R > 1 else 0))
+    return Bt * H * total
+
+
+FFMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # SMs x FP32 lanes x 2 flops x max SM clock
+
+
+class BwdWorkload(ScanWorkload):
+    """One backward call of a chunked-scan workload: every input gradient
+    from dy (the final-state adjoints zero), outputs preallocated."""
+
+    def __init__(self, idx, device):
+        super().__init__(idx, device)
+        c = self.c
+        self.host["dy"] = gen.grad_seed(self.host["x"], gen.SEED_BASE + 1000 + idx)
+        self.dev["dy"] = self.host["dy"].to(device)
+        Bt, T, H, P, N, R = c["batch"], c["seqlen"], c["nheads"], c["headdim"], c["dstate"], c["rank"]
+        d = self.m3.Dims(Bt, T, H, P, N, R if self.mimo else 1, c["chunk"], self.G, self.K)
+        nws = self.m3.workspace_bytes(self.m3.M3_WS_BWD_MIMO if self.mimo else self.m3.M3_WS_BWD_SISO, d,
+                                      self.m3.M3_BF16 if c["dtype"] == "bf16" else self.m3.M3_F32)
+        self.ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=device)
+        self.grads = self.m3.chunked_bwd(*[self.dev[k] for k in ("x", "dt", "A", "lam", "theta", "B", "C", "D")],
+                                         self.dev["dy"], c["chunk"], W_x=self.dev.get("Wx"),
+                                         W_y=self.dev.get("Wy"), workspace=self.ws)
+        self.out = tuple(self.grads.values())
+        self.bytes = bwd_bytes(c)
+        self.flops = bwd_flops(c)
+        self.kernel = "k_bwd_chunks"
+        self.kernel_label = "k_bwd_state + k_bwd_chunks + k_bwd_params (3 launches)"
+        self.srcs = [os.path.join(ROOT, "state_space_lm_b200", "csrc", "k_scan_bwd.cu")]
+        self.input_bytes += self.host["dy"].numel() * self.host["dy"].element_size()
+
+    def step(self, dev=None, out=None, stream=None):
+        d = self.dev if dev is None else dev
+        self.m3.chunked_bwd(*[d[k] for k in ("x", "dt", "A", "lam", "theta", "B", "C", "D")], d["dy"],
+                            self.c["chunk"], W_x=d.get("Wx"), W_y=d.get("Wy"), out=self.grads, workspace=self.ws,
+                            stream=stream)
+
+    def config(self):
+        cfg = super().config()
+        cfg["pass"] = "backward: all input gradients from dy (final-state adjoints zero), fp32 gradients"
+        return cfg
+
+    def oracle_sample(self, n_lanes, threads):
+        """The oracle's reverse sweep (one thread) on the first n lanes."""
+        import oracle
+        c = self.c
+        H = c["nheads"]
+        n = min(n_lanes, c["batch"] * H)
+        t0 = time.perf_counter()
+        for i in range(n):
+            b, h = i // H, i % H
+            lane = {k: gen.to_f64(self.host[k][b:b + 1, :, h:h + 1])
+                    for k in ("x", "dt", "lam", "theta", "B", "C")}
+            lane["A"], lane["D"] = gen.to_f64(self.host["A"][h:h + 1]), gen.to_f64(self.host["D"][h:h + 1])
+            oracle.loop_bwd(**lane, dy=gen.to_f64(self.host["dy"][b:b + 1, :, h:h + 1]))
+        return n, time.perf_counter() - t0, 1
+
+
 class DecodeWorkload:
     """Decode steps: every step advances all (batch, head) lanes by one token.
     The carried state comes from a seeded prefill (a chunked forward over the
@@ -391,6 +475,20 @@ def run_cpu_baseline(w, target_s=10.0, wall_s=1.5):
                       % (reps, nl, total_lanes, w.c["seqlen"], dt, used)}
 
 
+def run_cpu_baseline_bwd(w, target_s=8.0):
+    """The oracle's backward (single-threaded C loop) on as many lanes as fit
+    about target_s seconds; tokens/s scaled to whole (b, t) tokens."""
+    H = w.c["nheads"]
+    nl, dt, _ = w.oracle_sample(1, 1)
+    n = int(min(w.c["batch"] * H, max(1, target_s / max(dt, 1e-3))))
+    if n > 1:
+        nl, dt, _ = w.oracle_sample(n, 1)
+    tokens = nl * w.c["seqlen"] / H
+    return {"value": tokens / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "%d of %d (b,h) lanes x %d tokens, fp64 reverse sweep, %.1f s on 1 thread"
+                      % (nl, w.c["batch"] * H, w.c["seqlen"], dt)}
+
+
 # ---------------------------------------------------------------------------
 # the two arms
 # ---------------------------------------------------------------------------
@@ -403,6 +501,8 @@ def run_ours(args, world, rank, local):
         raise SystemExit("CUDA library not built: run python -m state_space_lm_b200.build")
     if "steps" in gen.CONFIGS[args.config]:      # the decode workloads
         w = DecodeWorkload(args.config, device, args.steps + args.warmup)
+    elif gen.CONFIGS[args.config].get("grad"):
+        w = BwdWorkload(args.config, device)
     else:
         w = ScanWorkload(args.config, device)
     stream = torch.cuda.current_stream(device)
@@ -482,14 +582,23 @@ def run_ours(args, world, rank, local):
     peaks, peak_kind = load_peaks()
     achieved = w.bytes / kernel_s / 1e9
     tr = traffic_record(w.kernel + ":" + w.c["name"], w.srcs)
-    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "traffic": (tr["dram_bytes_per_launch"] if tr else None),
-            "kernel": w.kernel_label, "algorithmic_bytes": w.bytes,
-            "kernel_ms": round(kernel_s * 1e3, 4),
-            "tensor_tflops": round(w.flops / kernel_s / 1e12, 2),
-            "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
-            else "fallback 6.65 TB/s"}
+    if isinstance(w, BwdWorkload):
+        # FFMA-bound: flops against the FP32 pipes' peak (148 SMs x 128 lanes x 2 x 1.965 GHz)
+        ach = w.flops / kernel_s / 1e12
+        roof = {"bound": "alu", "achieved": round(ach, 2), "peak": round(FFMA_PEAK_TFLOPS, 1), "unit": "TFLOP/s",
+                "frac": round(ach / FFMA_PEAK_TFLOPS, 4), "traffic": (tr["dram_bytes_per_launch"] if tr else None),
+                "kernel": w.kernel_label, "algorithmic_flops": w.flops, "algorithmic_bytes": w.bytes,
+                "hbm_gbs": round(achieved, 1), "kernel_ms": round(kernel_s * 1e3, 4),
+                "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 flops x 1965 MHz (no measured FP32 peak)"}
+    else:
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": (tr["dram_bytes_per_launch"] if tr else None),
+                "kernel": w.kernel_label, "algorithmic_bytes": w.bytes,
+                "kernel_ms": round(kernel_s * 1e3, 4),
+                "tensor_tflops": round(w.flops / kernel_s / 1e12, 2),
+                "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
+                else "fallback 6.65 TB/s"}
 
     line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tmax / args.steps * 1e3, 4),
@@ -501,7 +610,7 @@ def run_ours(args, world, rank, local):
                     "d2h_bytes_per_step": d2h},
             "clocks": clk.report(), "gpu_launches": int(launches)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline and isinstance(w, ScanWorkload):
-        line["cpu_baseline"] = run_cpu_baseline(w)
+        line["cpu_baseline"] = (run_cpu_baseline_bwd(w) if isinstance(w, BwdWorkload) else run_cpu_baseline(w))
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:
@@ -516,11 +625,14 @@ def run_reference(args, world, rank):
         return
     import oracle
     oracle.build_oracle()
-    w = ScanWorkload.__new__(ScanWorkload)
+    bwd = bool(gen.CONFIGS[args.config].get("grad"))
+    w = (BwdWorkload if bwd else ScanWorkload).__new__(BwdWorkload if bwd else ScanWorkload)
     w.c = dict(gen.CONFIGS[args.config])
     w.idx = args.config
     w.host = gen.config_inputs(args.config)
     w.host.pop("generator")
+    if bwd:
+        w.host["dy"] = gen.grad_seed(w.host["x"], gen.SEED_BASE + 1000 + args.config)
     w.mimo = w.c["rank"] > 1
     w.G = w.c.get("ngroups", 0) or w.c["nheads"]
     w.K = w.c.get("rope_pairs", 0) or w.c["dstate"] // 2
@@ -528,6 +640,8 @@ def run_reference(args, world, rank):
     H = w.c["nheads"]
     total_lanes = w.c["batch"] * H
     n = min(total_lanes, max(H, (cores // H) * H if cores >= H else H))
+    if bwd:
+        n = 2    # the reverse sweep is single-threaded: two lanes per step
     for _ in range(args.warmup):
         w.oracle_sample(n, cores)
     times = []
@@ -538,7 +652,8 @@ def run_reference(args, world, rank):
     tokens = nl * w.c["seqlen"] / H
     el = sum(times)
     value = tokens * args.steps / el
-    sample = "%d of %d (b,h) lanes x %d tokens per step, fp64 C loop" % (nl, total_lanes, w.c["seqlen"])
+    sample = "%d of %d (b,h) lanes x %d tokens per step, fp64 C %s" % (
+        nl, total_lanes, w.c["seqlen"], "reverse sweep, 1 thread" if bwd else "loop")
     c = w.c
     line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
@@ -558,7 +673,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=1, choices=[0, 1, 2, 3, 4, 5, 6, 7])
+    ap.add_argument("--config", type=int, default=1, choices=[0, 1, 2, 3, 4, 5, 6, 7, 8])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

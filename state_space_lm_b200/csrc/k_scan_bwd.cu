@@ -44,7 +44,7 @@ namespace m3 {
 // and of X, Dy (stride Pp + 4); the states are kept transposed, (P, Np + 4),
 // so that every small product below reads conflict-free 16-byte vectors.
 struct BwdLayout {
-    int Q, QR, Np, Pp, ldn, ldp;
+    int Q, QR, Np, Pp, ldn, ldp, ldq;
     size_t Bb, Cb, dBb, dCb, X, Dy, BG, CG, S, V, DM, MK, gs, Gs, Ph, GP, tok, inv, rsc, par, misc, total;
 };
 
@@ -65,9 +65,11 @@ __host__ __device__ inline BwdLayout bwd_layout(int64_t P, int64_t N, int64_t R,
     L.Pp = (int)((P + 3) & ~3);
     L.ldn = L.Np + 4;
     L.ldp = L.Pp + 4;
+    L.ldq = ((L.QR + 3) & ~3) + 4;   // row stride of the (rows x rows) score matrices
     auto al4 = [](size_t v) { return (v + 3) & ~(size_t)3; };
     size_t o = 0;
-    const size_t rowsN = (size_t)L.QR * L.ldn, rowsP = (size_t)L.QR * L.ldp, st = (size_t)L.Pp * L.ldn;
+    const size_t QRp = (size_t)((L.QR + 3) & ~3);   // rows rounded up: 4-row products read whole groups
+    const size_t rowsN = QRp * L.ldn, rowsP = QRp * L.ldp, st = (size_t)L.Pp * L.ldn;
     L.Bb = o; o += rowsN;
     L.Cb = o; o += rowsN;
     L.dBb = o; o += rowsN;
@@ -78,8 +80,8 @@ __host__ __device__ inline BwdLayout bwd_layout(int64_t P, int64_t N, int64_t R,
     L.CG = o; o += rowsP;
     L.gs = o; o += st;
     L.Gs = o; o += st;
-    L.S = o; o += al4((size_t)L.QR * L.QR);
-    L.V = o; o += al4((size_t)L.QR * L.QR);
+    L.S = o; o += (size_t)L.QR * L.ldq;
+    L.V = o; o += (size_t)L.QR * L.ldq;
     L.DM = o; o += al4((size_t)Q * Q);
     L.MK = o; o += al4((size_t)Q * Q);
     L.Ph = o; o += al4((size_t)Q * K);
@@ -253,6 +255,117 @@ __device__ void mm_state_update(float *St, int lds, int Np, int P, float e, cons
     }
 }
 
+// out[c][j..j+1] = rs[c/R] out[c][j..j+1] + sum_{k < nk} W[k][c] Rm[k][j..j+1]
+// (W read by columns: a warp shares 4 output rows c, its lanes own column pairs j)
+__device__ void mm_wT_rows(float *out, int ldo, int nrows, const float *W, int ldw, int nk, const float *Rm, int ldr,
+                           int ncols, const float *rs, int R) {
+    const int ngt = ncols / 2, njb = (ngt + 31) / 32, nrb = (nrows + 3) / 4;
+    for (int it = threadIdx.x; it < nrb * njb * 32; it += blockDim.x) {
+        const int l = it & 31, q = it >> 5, jb = q % njb, c0 = (q / njb) * 4;
+        const int jg = jb * 32 + l, j = 2 * (jg < ngt ? jg : 0);
+        float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
+        for (int k = 0; k < nk; k++) {
+            const float2 r = *reinterpret_cast<const float2 *>(Rm + (size_t)k * ldr + j);
+            const float4 wv = ld4(W + (size_t)k * ldw + c0);
+            a0.x = fmaf(wv.x, r.x, a0.x); a0.y = fmaf(wv.x, r.y, a0.y);
+            a1.x = fmaf(wv.y, r.x, a1.x); a1.y = fmaf(wv.y, r.y, a1.y);
+            a2.x = fmaf(wv.z, r.x, a2.x); a2.y = fmaf(wv.z, r.y, a2.y);
+            a3.x = fmaf(wv.w, r.x, a3.x); a3.y = fmaf(wv.w, r.y, a3.y);
+        }
+        if (jg < ngt) {
+            const float2 av[4] = {a0, a1, a2, a3};
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                if (c0 + i < nrows) {
+                    float2 *o = reinterpret_cast<float2 *>(out + (size_t)(c0 + i) * ldo + j);
+                    const float sc = rs[(c0 + i) / R];
+                    *o = make_float2(fmaf(sc, o->x, av[i].x), fmaf(sc, o->y, av[i].y));
+                }
+        }
+    }
+}
+
+// out[r][j..j+1] = rs[r/R] out[r][j..j+1] + sum_{k < nk} W[r][k] Rm[k][j..j+1]
+// (nk rounded up to 4: W's columns from nk on must be zero; a warp shares 4 rows r)
+__device__ void mm_w_rows(float *out, int ldo, int nrows, const float *W, int ldw, int nk, const float *Rm, int ldr,
+                          int ncols, const float *rs, int R) {
+    const int ngt = ncols / 2, njb = (ngt + 31) / 32, nrb = (nrows + 3) / 4, nk4 = (nk + 3) & ~3;
+    for (int it = threadIdx.x; it < nrb * njb * 32; it += blockDim.x) {
+        const int l = it & 31, q = it >> 5, jb = q % njb, r0 = (q / njb) * 4;
+        const int jg = jb * 32 + l, j = 2 * (jg < ngt ? jg : 0);
+        float2 acc[4];
+#pragma unroll
+        for (int i = 0; i < 4; i++) acc[i] = make_float2(0.f, 0.f);
+        for (int k = 0; k < nk4; k += 4) {
+            float2 rk[4];
+#pragma unroll
+            for (int u = 0; u < 4; u++) rk[u] = *reinterpret_cast<const float2 *>(Rm + (size_t)(k + u) * ldr + j);
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const float4 wv = ld4(W + (size_t)min(r0 + i, nrows - 1) * ldw + k);
+                acc[i].x = fmaf(wv.x, rk[0].x, fmaf(wv.y, rk[1].x, fmaf(wv.z, rk[2].x, fmaf(wv.w, rk[3].x, acc[i].x))));
+                acc[i].y = fmaf(wv.x, rk[0].y, fmaf(wv.y, rk[1].y, fmaf(wv.z, rk[2].y, fmaf(wv.w, rk[3].y, acc[i].y))));
+            }
+        }
+        if (jg < ngt) {
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                if (r0 + i < nrows) {
+                    float2 *o = reinterpret_cast<float2 *>(out + (size_t)(r0 + i) * ldo + j);
+                    const float sc = rs[(r0 + i) / R];
+                    *o = make_float2(fmaf(sc, o->x, acc[i].x), fmaf(sc, o->y, acc[i].y));
+                }
+        }
+    }
+}
+
+// S[rr][cr] = Cbar_rr . Bbar_cr and V[rr][cr] = Dy_rr . X_cr for token(cr) <= token(rr), else 0
+// (lanes own consecutive rows rr -- conflict-free 16-byte loads -- and a warp shares 4 columns cr)
+__device__ void scores(float *S, float *V, int ldq, const float *Cb, const float *Bb, int ldn, int Np, const float *Dy,
+                       const float *X, int ldp, int Pp, int nrows, int R) {
+    const int nrb = (nrows + 31) / 32, ncg = (nrows + 3) / 4;
+    for (int it = threadIdx.x; it < ncg * nrb * 32; it += blockDim.x) {
+        const int l = it & 31, q = it >> 5, rb = q % nrb, c0 = (q / nrb) * 4;
+        const int rr = rb * 32 + l;
+        const int rc = min(rr, nrows - 1);
+        if (c0 / R > rc / R) {   // the whole tile lies above the diagonal
+            if (rr < nrows) {
+                st4(S + (size_t)rr * ldq + c0, make_float4(0.f, 0.f, 0.f, 0.f));
+                st4(V + (size_t)rr * ldq + c0, make_float4(0.f, 0.f, 0.f, 0.f));
+            }
+            continue;
+        }
+        const float *cp = Cb + (size_t)rc * ldn, *dp = Dy + (size_t)rc * ldp;
+        const float *b0 = Bb + (size_t)min(c0, nrows - 1) * ldn, *b1 = Bb + (size_t)min(c0 + 1, nrows - 1) * ldn;
+        const float *b2 = Bb + (size_t)min(c0 + 2, nrows - 1) * ldn, *b3 = Bb + (size_t)min(c0 + 3, nrows - 1) * ldn;
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+        for (int n = 0; n < Np; n += 4) {
+            const float4 cv = ld4(cp + n);
+            s0 = dot4(cv, ld4(b0 + n), s0);
+            s1 = dot4(cv, ld4(b1 + n), s1);
+            s2 = dot4(cv, ld4(b2 + n), s2);
+            s3 = dot4(cv, ld4(b3 + n), s3);
+        }
+        const float *x0 = X + (size_t)min(c0, nrows - 1) * ldp, *x1 = X + (size_t)min(c0 + 1, nrows - 1) * ldp;
+        const float *x2 = X + (size_t)min(c0 + 2, nrows - 1) * ldp, *x3 = X + (size_t)min(c0 + 3, nrows - 1) * ldp;
+        float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
+        for (int p = 0; p < Pp; p += 4) {
+            const float4 dv = ld4(dp + p);
+            v0 = dot4(dv, ld4(x0 + p), v0);
+            v1 = dot4(dv, ld4(x1 + p), v1);
+            v2 = dot4(dv, ld4(x2 + p), v2);
+            v3 = dot4(dv, ld4(x3 + p), v3);
+        }
+        if (rr < nrows) {
+            const int tr = rr / R;
+            const bool k0 = c0 < nrows && c0 / R <= tr, k1 = c0 + 1 < nrows && (c0 + 1) / R <= tr;
+            const bool k2 = c0 + 2 < nrows && (c0 + 2) / R <= tr, k3 = c0 + 3 < nrows && (c0 + 3) / R <= tr;
+            st4(S + (size_t)rr * ldq + c0, make_float4(k0 ? s0 : 0.f, k1 ? s1 : 0.f, k2 ? s2 : 0.f, k3 ? s3 : 0.f));
+            st4(V + (size_t)rr * ldq + c0, make_float4(k0 ? v0 : 0.f, k1 ? v1 : 0.f, k2 ? v2 : 0.f, k3 ? v3 : 0.f));
+        }
+    }
+}
+
 // global (N, P) row-major  <->  shared transposed (P, ldn)
 __device__ void load_state_T(float *St, int lds, const float *g, int N, int P, float scale = 1.f,
                              const float *g2 = nullptr, float s2 = 0.f) {
@@ -264,9 +377,31 @@ __device__ void load_state_T(float *St, int lds, const float *g, int N, int P, f
     }
 }
 
+// 4-byte asynchronous global -> shared copies (all of a chunk's raw inputs in
+// flight at once, instead of one dependent load per loop iteration)
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+// rows of `words` 4-byte words: dst row k <- src + off(k)
+template <typename F>
+__device__ __forceinline__ void stage_rows(void *dst, int nrows, int words, F src_row) {
+    for (int it = threadIdx.x; it < nrows * words; it += blockDim.x) {
+        const int k = it / words, w = it % words;
+        cp_async4(static_cast<char *>(dst) + ((size_t)k * words + w) * 4,
+                  reinterpret_cast<const char *>(src_row(k)) + (size_t)w * 4);
+    }
+}
+
 // Chunk preparation shared by the state and the reverse pass: per-token
 // coefficients, angles from phi_in, QkNorm inverse RMS, rotated B (and C),
-// X = W_x x (and Dy = W_y dy).  Ends with a __syncthreads.
+// X = W_x x (and Dy = W_y dy).  The chunk's raw B, C, x, dy and theta are
+// first staged in arrays that are free until the prep ends (dBbar, dCbar,
+// BG, CG, GP).  Ends with a __syncthreads.
 template <typename T>
 __device__ void bwd_prep(const BwdArgs &a, const BwdSmem &s, const BwdLayout &Lo, int64_t b, int64_t h,
                          int64_t hg, int64_t t0, int L, const float *phi_in, bool full) {
@@ -282,6 +417,29 @@ __device__ void bwd_prep(const BwdArgs &a, const BwdSmem &s, const BwdLayout &Lo
     float *dts = s.tk(TK_DT, Q), *lam = s.tk(TK_LAM, Q), *la = s.tk(TK_LA, Q), *cum = s.tk(TK_CUM, Q);
     float *gam = s.tk(TK_GAM, Q), *w = s.tk(TK_W, Q), *ec = s.tk(TK_EC, Q), *cs = s.tk(TK_CS, Q);
     float *cw = s.tk(TK_CW, Q);
+    T *sB = reinterpret_cast<T *>(s.dBb), *sC = reinterpret_cast<T *>(s.dCb);
+    T *sx = reinterpret_cast<T *>(s.BG), *sdy = reinterpret_cast<T *>(s.CG);
+    float *sth = s.GP;
+    {
+        const int wbc = N * (int)sizeof(T) / 4;   // N is even: whole 4-byte words
+        auto brow = [&](int k) { return Bg + (((b * Tn + t0 + k / R) * G + hg) * R + k % R) * N; };
+        auto crow = [&](int k) { return Cg + (((b * Tn + t0 + k / R) * G + hg) * R + k % R) * N; };
+        stage_rows(sB, LR, wbc, brow);
+        if (full) stage_rows(sC, LR, wbc, crow);
+        stage_rows(sth, L, K, [&](int k) { return a.theta + ((b * Tn + t0 + k) * H + h) * K; });
+        if ((P * (int)sizeof(T)) % 4 == 0) {
+            const int wx = P * (int)sizeof(T) / 4;
+            stage_rows(sx, L, wx, [&](int k) { return x + ((b * Tn + t0 + k) * H + h) * P; });
+            if (full) stage_rows(sdy, L, wx, [&](int k) { return dy + ((b * Tn + t0 + k) * H + h) * P; });
+        } else {   // rows not a whole number of words: plain copies
+            for (int it = tid; it < L * P; it += nt) {
+                const int64_t xi = ((b * Tn + t0 + it / P) * H + h) * P + it % P;
+                sx[it] = x[xi];
+                if (full) sdy[it] = dy[xi];
+            }
+        }
+        cp_async_wait_all();
+    }
     for (int i = tid; i < L; i += nt) {
         const int64_t bt = (b * Tn + t0 + i) * H + h;
         const float dl = a.dt[bt], lm = a.lam[bt];
@@ -293,13 +451,13 @@ __device__ void bwd_prep(const BwdArgs &a, const BwdSmem &s, const BwdLayout &Lo
         gam[i] = lm * dl;
         w[i] = lm * dl + sg;
     }
+    __syncthreads();   // the staged rows are visible to every thread
     const bool has_norm = a.nrm.wB || a.nrm.wC;
     if (has_norm) {
         for (int row = warp; row < LR; row += nw) {
-            const int64_t base = (((b * Tn + t0 + row / R) * G + hg) * R + row % R) * N;
             float sb = 0.f, sc = 0.f;
             for (int n = l32; n < N; n += 32) {
-                const float vb = ldf(Bg, base + n), vc = ldf(Cg, base + n);
+                const float vb = ldf(sB, row * N + n), vc = full ? ldf(sC, row * N + n) : 0.f;
                 sb += vb * vb;
                 sc += vc * vc;
             }
@@ -321,12 +479,11 @@ __device__ void bwd_prep(const BwdArgs &a, const BwdSmem &s, const BwdLayout &Lo
             cum[i] = run;
         }
     }
-    // angles: theta loads of all tokens first (independent), then the running sum
+    // angles: the running sum of dt theta from the chunk's entering angle
     for (int j = tid; j < K; j += nt) {
-        for (int i = 0; i < L; i++) s.Ph[i * K + j] = a.theta[((b * Tn + t0 + i) * H + h) * K + j];
         float c = phi_in[j];
         for (int i = 0; i < L; i++) {
-            c += dts[i] * s.Ph[i * K + j];
+            c += dts[i] * sth[i * K + j];
             s.Ph[i * K + j] = c;
         }
     }
@@ -338,9 +495,9 @@ __device__ void bwd_prep(const BwdArgs &a, const BwdSmem &s, const BwdLayout &Lo
     }
     for (int it = tid; it < LR * (N / 2); it += nt) {
         const int j = it % (N / 2), row = it / (N / 2), i = row / R, r = row % R;
-        const int64_t base = (((b * Tn + t0 + i) * G + hg) * R + r) * N + 2 * j;
-        float b0 = ldf(Bg, base), b1 = ldf(Bg, base + 1);
-        float c0 = full ? ldf(Cg, base) : 0.f, c1 = full ? ldf(Cg, base + 1) : 0.f;
+        const int base = row * N + 2 * j;
+        float b0 = ldf(sB, base), b1 = ldf(sB, base + 1);
+        float c0 = full ? ldf(sC, base) : 0.f, c1 = full ? ldf(sC, base + 1) : 0.f;
         if (a.nrm.wB) { b0 *= s.inv[row] * a.nrm.wB[2 * j]; b1 *= s.inv[row] * a.nrm.wB[2 * j + 1]; }
         if (a.nrm.wC) { c0 *= s.inv[Q * R + row] * a.nrm.wC[2 * j]; c1 *= s.inv[Q * R + row] * a.nrm.wC[2 * j + 1]; }
         const int64_t bo = (h * R + r) * N + 2 * j;
@@ -357,9 +514,8 @@ __device__ void bwd_prep(const BwdArgs &a, const BwdSmem &s, const BwdLayout &Lo
     }
     for (int it = tid; it < LR * P; it += nt) {
         const int p = it % P, row = it / P, i = row / R, r = row % R;
-        const int64_t xi = ((b * Tn + t0 + i) * H + h) * P + p;
-        s.X[row * ldp + p] = (a.Wx ? a.Wx[(h * R + r) * P + p] : 1.f) * ldf(x, xi);
-        if (full) s.Dy[row * ldp + p] = (a.Wy ? a.Wy[(h * R + r) * P + p] : 1.f) * ldf(dy, xi);
+        s.X[row * ldp + p] = (a.Wx ? a.Wx[(h * R + r) * P + p] : 1.f) * ldf(sx, i * P + p);
+        if (full) s.Dy[row * ldp + p] = (a.Wy ? a.Wy[(h * R + r) * P + p] : 1.f) * ldf(sdy, i * P + p);
     }
     __syncthreads();
 }
@@ -420,7 +576,7 @@ __global__ void __launch_bounds__(256, 1) k_bwd_chunks(BwdArgs a) {
     const int64_t NP = (int64_t)N * P, nch = (Tn + Q - 1) / Q;
     const int RP = R * P, RN = R * N;
     const BwdLayout Lo = bwd_layout(P, N, R, K, Q);
-    const int ldn = Lo.ldn, ldp = Lo.ldp, Np = Lo.Np;
+    const int ldn = Lo.ldn, ldp = Lo.ldp, Np = Lo.Np, ldq = Lo.ldq;
     extern __shared__ float sm[];
     const BwdSmem s(sm, Lo);
     const int tid = threadIdx.x, nt = blockDim.x, warp = tid >> 5, l32 = tid & 31, nw = nt >> 5;
@@ -469,18 +625,7 @@ __global__ void __launch_bounds__(256, 1) k_bwd_chunks(BwdArgs a) {
         // V = Dy X^T (causal pairs only)
         mm_rows_by_state(s.Bb, ldn, LR, s.Gs, ldn, Np, P, s.BG, ldp);
         mm_rows_by_state(s.Cb, ldn, LR, s.gs, ldn, Np, P, s.CG, ldp);
-        for (int it = tid; it < LR * LR; it += nt) {
-            const int cr = it % LR, rr = it / LR;
-            float sv = 0.f, vv = 0.f;
-            if (cr / R <= rr / R) {
-                const float *cp = s.Cb + rr * ldn, *bp = s.Bb + cr * ldn;
-                for (int n = 0; n < Np; n += 4) sv = dot4(ld4(cp + n), ld4(bp + n), sv);
-                const float *dp = s.Dy + rr * ldp, *xp = s.X + cr * ldp;
-                for (int p = 0; p < Lo.Pp; p += 4) vv = dot4(ld4(dp + p), ld4(xp + p), vv);
-            }
-            s.S[rr * LR + cr] = sv;
-            s.V[rr * LR + cr] = vv;
-        }
+        scores(s.S, s.V, ldq, s.Cb, s.Bb, ldn, Np, s.Dy, s.X, ldp, Lo.Pp, LR, R);
         __syncthreads();
         // (f) token scalars: q_t = <Gin, U_t>, yi_s = sum_r Dy_s . CG_s, dM, dy . x
         for (int i = warp; i < L; i += nw) {
@@ -508,7 +653,7 @@ __global__ void __launch_bounds__(256, 1) k_bwd_chunks(BwdArgs a) {
                 for (int r2 = 0; r2 < R; r2++)
                     for (int r1 = 0; r1 < R; r1++) {
                         const int rr = ss * R + r2, cr = tt * R + r1;
-                        v += s.S[rr * LR + cr] * s.V[rr * LR + cr];
+                        v += s.S[rr * ldq + cr] * s.V[rr * ldq + cr];
                     }
             s.DM[ss * Q + tt] = v;
         }
@@ -540,87 +685,46 @@ __global__ void __launch_bounds__(256, 1) k_bwd_chunks(BwdArgs a) {
             dw[i] = dwi;
             dgam[i] = s.DM[i * Q + i] + dwi;
         }
-        // (h2) dX -> dx (dX kept in BG for dW_x); dBbar, dCbar intra parts; MIMO: Y -> dW_y
+        // the masked scores S <- M o S, V <- M o V (the token mask expanded over ranks)
+        for (int it = tid; it < LR * LR; it += nt) {
+            const int cr = it % LR, rr = it / LR;
+            const float m = s.MK[(rr / R) * Q + cr / R];
+            s.S[rr * ldq + cr] *= m;
+            s.V[rr * ldq + cr] *= m;
+        }
+        __syncthreads();
+        // (h2) dX = w cs BG + S'^T Dy (into BG); dBbar = w cs GX + V'^T Cbar (into dBb);
+        // dCbar = e^{cum} GD + V' Bbar (into dCb); MIMO: Y = e^{cum} CG + S' X (into CG)
+        const float *cw = s.tk(TK_CW, Q);
+        mm_wT_rows(s.BG, ldp, LR, s.S, ldq, LR, s.Dy, ldp, Lo.Pp, cw, R);
+        mm_wT_rows(s.dBb, ldn, LR, s.V, ldq, LR, s.Cb, ldn, Np, cw, R);
+        mm_w_rows(s.dCb, ldn, LR, s.V, ldq, LR, s.Bb, ldn, Np, ec, R);
+        if (a.dWy) mm_w_rows(s.CG, ldp, LR, s.S, ldq, LR, s.X, ldp, Lo.Pp, ec, R);
+        __syncthreads();
+        if (last && a.du) {   // prev_Bx_final = U_{T-1}: its adjoint reaches the last token's rows
+            const float *du = a.du + lane * NP;
+            for (int it = tid; it < R * P; it += nt) {
+                const int p = it % P, cr = (L - 1) * R + it / P;
+                float e = 0.f;
+                for (int n = 0; n < N; n++) e += du[n * P + p] * s.Bb[cr * ldn + n];
+                s.BG[cr * ldp + p] += e;
+            }
+            for (int it = tid; it < R * N; it += nt) {
+                const int n = it % N, cr = (L - 1) * R + it / N;
+                float e = 0.f;
+                for (int p = 0; p < P; p++) e += du[n * P + p] * s.X[cr * ldp + p];
+                s.dBb[cr * ldn + n] += e;
+            }
+            __syncthreads();
+        }
+        // dx = D dy + sum_r W_x[r] dX_r
         for (int it = tid; it < L * P; it += nt) {
             const int p = it % P, i = it / P;
             const int64_t xi = ((b * Tn + t0 + i) * H + h) * P + p;
-            const float dyv = ldf(dy, xi);
-            float dxs = Dh * dyv;
-            for (int r = 0; r < R; r++) {
-                const int cr = i * R + r;
-                float v = w[i] * cs[i] * s.BG[cr * ldp + p];
-                for (int ss = i; ss < L; ss++) {
-                    const float m = s.MK[ss * Q + i];
-                    float acc = 0.f;
-                    for (int r2 = 0; r2 < R; r2++) {
-                        const int rr = ss * R + r2;
-                        acc += s.S[rr * LR + cr] * s.Dy[rr * ldp + p];
-                    }
-                    v += m * acc;
-                }
-                if (last && i == L - 1 && a.du) {
-                    const float *du = a.du + lane * NP;
-                    const float *bp = s.Bb + cr * ldn;
-                    float e = 0.f;
-                    for (int n = 0; n < N; n++) e += du[n * P + p] * bp[n];
-                    v += e;
-                }
-                const float wx = a.Wx ? a.Wx[(h * R + r) * P + p] : 1.f;
-                dxs += wx * v;
-                s.BG[cr * ldp + p] = v;   // dX_{t,r}[p] (this thread's own element)
-            }
+            float dxs = Dh * ldf(dy, xi);
+            for (int r = 0; r < R; r++) dxs += (a.Wx ? a.Wx[(h * R + r) * P + p] : 1.f) * s.BG[(i * R + r) * ldp + p];
             if (a.dx) a.dx[xi] = dxs;
         }
-        for (int it = tid; it < LR * N; it += nt) {
-            const int n = it % N, cr = it / N, i = cr / R;
-            float v = w[i] * cs[i] * s.dBb[cr * ldn + n];
-            if (last && i == L - 1 && a.du) {   // dprevBx_final X_{T-1}
-                const float *du = a.du + lane * NP + (int64_t)n * P, *xp = s.X + cr * ldp;
-                for (int p = 0; p < P; p++) v += du[p] * xp[p];
-            }
-            for (int ss = i; ss < L; ss++) {
-                const float m = s.MK[ss * Q + i];
-                float acc = 0.f;
-                for (int r2 = 0; r2 < R; r2++) {
-                    const int rr = ss * R + r2;
-                    acc += s.V[rr * LR + cr] * s.Cb[rr * ldn + n];
-                }
-                v += m * acc;
-            }
-            s.dBb[cr * ldn + n] = v;
-        }
-        for (int it = tid; it < LR * N; it += nt) {
-            const int n = it % N, rr = it / N, i = rr / R;
-            float v = ec[i] * s.dCb[rr * ldn + n];
-            for (int tt = 0; tt <= i; tt++) {
-                const float m = s.MK[i * Q + tt];
-                float acc = 0.f;
-                for (int r1 = 0; r1 < R; r1++) {
-                    const int cr = tt * R + r1;
-                    acc += s.V[rr * LR + cr] * s.Bb[cr * ldn + n];
-                }
-                v += m * acc;
-            }
-            s.dCb[rr * ldn + n] = v;
-        }
-        if (a.dWy) {
-            // the forward's per-rank output, in place of CG (each thread its own element):
-            // Y_{s,r}[p] = sum_{t<=s} M[s,t] sum_r1 S[(s,r),(t,r1)] X_{t,r1}[p] + e^{cum_s} CG_{s,r}[p]
-            for (int it = tid; it < LR * P; it += nt) {
-                const int p = it % P, rr = it / P, i = rr / R;
-                float yv = ec[i] * s.CG[rr * ldp + p];
-                for (int tt = 0; tt <= i; tt++) {
-                    float acc = 0.f;
-                    for (int r1 = 0; r1 < R; r1++) {
-                        const int cr = tt * R + r1;
-                        acc += s.S[rr * LR + cr] * s.X[cr * ldp + p];
-                    }
-                    yv += s.MK[i * Q + tt] * acc;
-                }
-                s.CG[rr * ldp + p] = yv;
-            }
-        }
-        __syncthreads();
         if (tid == 0) {
             float run = 0.f;
             for (int i = L - 1; i >= 0; i--) {

@@ -48,6 +48,9 @@ CONFIGS = {
     # checkpoint's n_groups 1 and rope fraction 0.5), default workload's shape
     7: dict(name="siso_g1_rope32_8x2048_h16_p64_n128", batch=8, seqlen=2048, nheads=16, headdim=64,
             dstate=128, rank=1, chunk=64, dtype="bf16", dt_shift=-2.0, ngroups=1, rope_pairs=32),
+    # the backward (all input gradients) of the default workload
+    8: dict(name="bwd_siso_8x2048_h16_p64_n128", batch=8, seqlen=2048, nheads=16, headdim=64,
+            dstate=128, rank=1, chunk=64, dtype="bf16", dt_shift=-2.0, grad=True),
 }
 
 _DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}
@@ -135,9 +138,10 @@ def decode_step_inputs(generator, batch, nheads, headdim, dstate, dtype="bf16",
 
 
 def config_inputs(idx, seed=None, **overrides):
-    """Inputs of workload ``idx`` (0-3 and 7: one chunked-scan call; 4-6: the
-    prefill of a decode workload -- its steps come from ``decode_step_inputs``
-    with the returned generator)."""
+    """Inputs of workload ``idx`` (0-3, 7 and 8: one chunked-scan call, forward
+    or backward; 4-6: the prefill of a decode workload -- its steps come from
+    ``decode_step_inputs`` with the returned generator).  The backward's dy is
+    drawn by ``grad_seed``."""
     c = dict(CONFIGS[idx])
     c.update(overrides)
     s = SEED_BASE + idx if seed is None else seed
@@ -145,6 +149,12 @@ def config_inputs(idx, seed=None, **overrides):
                        rank=c["rank"], dtype=c["dtype"], dt_shift=c["dt_shift"], seed=s,
                        mimo_weights=c["rank"] > 1, ngroups=c.get("ngroups", 0),
                        rope_pairs=c.get("rope_pairs", 0))
+
+
+def grad_seed(x, seed):
+    """dy ~ N(0, 1) in x's shape and dtype (the backward's output adjoint)."""
+    g = make_generator(seed)
+    return _normal(g, tuple(x.shape)).to(x.dtype)
 
 
 def to_f64(t):

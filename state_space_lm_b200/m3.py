@@ -310,12 +310,13 @@ def step_decode_factored(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, b_prev, x
 
 def chunked_bwd(x, dt, A, lam, theta, B, C, D, dy, chunk, W_x=None, W_y=None, norm=None, h0=None,
                 prevBx0=None, angle0=None, dh_final=None, dprevBx_final=None, dangle_final=None,
-                want=None, workspace=None, stream=None):
+                want=None, out=None, workspace=None, stream=None):
     """Backward of the chunked forward: returns a dict of fp32 gradients (the
     names in ``want``, by default all of them, without dW_x and dW_y for SISO;
     the gain and bias entries only when that part of the norm is on).  B, C
     (Bt,T,G,N) for SISO or (Bt,T,G,R,N) for rank R; dy has x's shape and dtype;
-    the state adjoints default to zero."""
+    the state adjoints default to zero.  ``out`` may hold preallocated fp32
+    tensors by name (they are written and returned)."""
     Bt, T, H, P = x.shape
     R = B.shape[3] if B.dim() == 5 else 1
     N, G, K = B.shape[-1], B.shape[2], theta.shape[-1]
@@ -329,7 +330,8 @@ def chunked_bwd(x, dt, A, lam, theta, B, C, D, dy, chunk, W_x=None, W_y=None, no
                   dangle0=(Bt, H, K))
     nm = norm or {}
     off = {"dnormw_B": "normw_B", "dnormw_C": "normw_C", "dbias_B": "bias_B", "dbias_C": "bias_C"}
-    out = {k: torch.empty(shapes[k], device=dev, dtype=torch.float32) for k in want
+    pre = out or {}
+    out = {k: (pre[k] if k in pre else torch.empty(shapes[k], device=dev, dtype=torch.float32)) for k in want
            if k not in off or nm.get(off[k]) is not None}
     g = Grads(*[_ptr(out.get(k)) for k in GRAD_FIELDS])
     d = Dims(Bt, T, H, P, N, R if mimo else 1, int(chunk), G, K)
