@@ -299,6 +299,15 @@ const char *m3_status_string(m3_status s);
  * none).  It is the one entry point that synchronises. */
 m3_status m3_device_error(void *stream, int *site);
 
+/* Self-test of the timeout path.  Enqueues one kernel that waits, with the
+ * library's bounded wait, on a barrier that nothing ever completes: after
+ * about one second the wait gives up and records M3_SELFTEST_SITE in the
+ * device error word, and the kernel returns normally (no fault, no trap; the
+ * context stays usable).  m3_device_error then reports M3_ERR_TIMEOUT with
+ * that site.  Returns M3_OK once enqueued. */
+#define M3_SELFTEST_SITE 99
+m3_status m3_selftest_bounded_wait(void *stream);
+
 /* Number of kernels the library has enqueued since it was loaded (host-side
  * counter, incremented once per launch; used to count launches in a timed
  * region). */

@@ -1393,7 +1393,34 @@ __global__ void __launch_bounds__(256) k_seg_combine(TcArgs a) {
     }
 }
 
+// Exercises the timeout path of the bounded waits without any fault: one
+// thread waits, with the kernels' own bounded wait, on an mbarrier that
+// nothing ever arrives on.  The wait gives up after WAIT_LIMIT_CYCLES, sets
+// the abort flag, records `site` in the device error word and the kernel
+// returns normally.
+__global__ void k_wait_selftest(int *err, int site) {
+    __shared__ alignas(8) uint64_t never;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&never), 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)wait_bar(smem_u32(&never), 0, &abort_flag, err, site);
+    __syncthreads();
+}
+
 }  // namespace tc
+
+cudaError_t launch_wait_selftest(int site, cudaStream_t s) {
+    int *err = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void **>(&err), tc::g_tc_error);
+    if (e != cudaSuccess) return e;
+    tc::k_wait_selftest<<<1, 32, 0, s>>>(err, site);
+    count_launch();
+    return cudaGetLastError();
+}
 
 size_t scan_tc_workspace_bytes(int64_t Bt, int64_t H, int64_t T) {
     const tc::SegPlan pl = tc::seg_plan(Bt * H, T);

@@ -149,6 +149,10 @@ m3_status m3_device_error(void *stream, int *site) {
     return e ? M3_ERR_TIMEOUT : M3_OK;
 }
 
+m3_status m3_selftest_bounded_wait(void *stream) {
+    return launched(launch_wait_selftest(M3_SELFTEST_SITE, (cudaStream_t)stream));
+}
+
 size_t m3_workspace_bytes(int which, m3_dims d, m3_dtype dtype) {
     if (which == M3_WS_BWD_SISO || which == M3_WS_BWD_MIMO) {
         BwdArgs b{};

@@ -100,6 +100,8 @@ cudaError_t launch_decode_gen(const DecodeArgs &a, m3_dtype dt, bool factored, c
 bool scan_tc_supported(const ScanArgs &a, m3_dtype dt);
 cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t s);
 int scan_tc_error_and_clear(cudaStream_t s);
+// one bounded wait on a barrier nothing completes (tests the timeout path)
+cudaError_t launch_wait_selftest(int site, cudaStream_t s);
 size_t scan_tc_workspace_bytes(int64_t Bt, int64_t H, int64_t T);
 
 // backward of the chunked scan (FFMA): chunk length that fits, workspace, launch

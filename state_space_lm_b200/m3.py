@@ -23,8 +23,9 @@ ABI_FUNCTIONS = (
     "m3_get_limits", "m3_discretize", "m3_rope_bc", "m3_siso_chunked_fwd",
     "m3_mimo_chunked_fwd", "m3_step_decode", "m3_workspace_bytes", "m3_status_string",
     "m3_launch_count", "m3_device_error", "m3_siso_chunked_fwd_noalloc", "m3_mimo_step_decode",
-    "m3_step_decode_factored", "m3_chunked_bwd",
+    "m3_step_decode_factored", "m3_chunked_bwd", "m3_selftest_bounded_wait",
 )
+M3_SELFTEST_SITE = 99
 
 GRAD_FIELDS = ("dx", "ddt", "dA", "dlam", "dtheta", "dB", "dC", "dD", "dW_x", "dW_y",
                "dnormw_B", "dnormw_C", "dbias_B", "dbias_C", "dh0", "dprevBx0", "dangle0")
@@ -108,6 +109,8 @@ def lib():
                                       ctypes.POINTER(BcNorm), Dims, _VP, _VP, _VP, _VP, _VP]
     L.m3_step_decode_factored.argtypes = [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int,
                                           ctypes.POINTER(BcNorm), Dims, _VP, _VP, _VP, _VP, _VP, _VP]
+    L.m3_selftest_bounded_wait.restype = ctypes.c_int
+    L.m3_selftest_bounded_wait.argtypes = [_VP]
     L.m3_chunked_bwd.restype = ctypes.c_int
     L.m3_chunked_bwd.argtypes = [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int,
                                  ctypes.POINTER(BcNorm), _VP, _VP, _VP, Dims, _VP, _VP, _VP, _VP,
@@ -131,6 +134,12 @@ def device_error(stream=None, with_site=False):
     site = ctypes.c_int(0)
     st = int(lib().m3_device_error(_stream(stream), ctypes.byref(site)))
     return (st, site.value) if with_site else st
+
+
+def selftest_bounded_wait(stream=None):
+    """Enqueue the timeout-path self-test (one bounded wait that runs out after
+    about a second); read the outcome with device_error()."""
+    _check(lib().m3_selftest_bounded_wait(_stream(stream)), "m3_selftest_bounded_wait")
 
 
 def limits():
