@@ -1351,14 +1351,28 @@ struct SegPlan {
 static SegPlan seg_plan(int64_t lanes, int64_t T) {
     SegPlan p{1, T};
     if (lanes >= 96 || T <= 8 * Q) return p;
-    const int64_t target = (4 * 148 + lanes - 1) / lanes;   // about four CTAs per SM in all
-    int64_t len = (T + target - 1) / target;
-    len = ((len + Q - 1) / Q) * Q;
-    if (len < 4 * Q) len = 4 * Q;
-    const int64_t ns = (T + len - 1) / len;
-    if (ns < 2) return p;
-    p.nseg = (int)ns;
-    p.seg_len = len;
+    // A CTA holds a whole SM (shared memory), so a pass over k CTAs takes
+    // ceil(k / 148) waves of (chunks per segment) chunk times; the state-only
+    // pass over the nseg - 1 leading segments costs about 0.6 of a full chunk
+    // per chunk.  Pick the segment count with the least time in those units,
+    // with at least 4 chunks per segment and the workspace ((nseg - 1) * lanes
+    // slots) within 24 MB.
+    const int64_t nq = (T + Q - 1) / Q;
+    const int64_t max_slots = ((int64_t)24 << 20) / ((int64_t)SLOT_FLOATS * 4);
+    auto waves = [](int64_t ctas) { return (ctas + 147) / 148; };
+    double best = (double)waves(lanes) * (double)nq;
+    for (int64_t ns = 2; ns <= 64; ns++) {
+        const int64_t len_q = (nq + ns - 1) / ns;
+        if (len_q < 4) break;
+        const int64_t nsr = (nq + len_q - 1) / len_q;   // segments at that length
+        if (nsr < 2 || (nsr - 1) * lanes > max_slots) continue;
+        const double cost = ((double)waves(lanes * nsr) + 0.6 * (double)waves(lanes * (nsr - 1))) * (double)len_q;
+        if (cost < best - 1e-9) {
+            best = cost;
+            p.nseg = (int)nsr;
+            p.seg_len = len_q * Q;
+        }
+    }
     return p;
 }
 
