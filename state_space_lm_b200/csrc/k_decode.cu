@@ -176,7 +176,18 @@ __global__ void __launch_bounds__(256) k_decode_gen(DecodeArgs a) {
     float *Cb = Bb + RT * N;        // RT x N  rotated C
     float *Pb = Cb + RT * N;        // RT x N  b_prev (factored form)
     float *red = Pb + RT * N;       // 32
-    float *ypart = red + 32;        // ngroups x RT x P
+    float *phs = red + 32;          // N/2 angles of this token
+    float *ypart = phs + N / 2;     // ngroups x RT x P
+
+    const int PV = P / VEC;              // vectors per state row
+    const int ngroups = nt / PV;         // rows streamed concurrently
+    const int pv = tid % PV, ng = tid / PV;
+    float4 *hp = reinterpret_cast<float4 *>(a.h + lane * (int64_t)N * P);
+    // start pulling my rows of h into L2 now: the state stream below then
+    // finds them there instead of waiting on HBM after the prologue
+    if (ng < ngroups)
+        for (int n = ng; n < N; n += ngroups)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(hp + n * PV + pv));
 
     const float dl = a.dt[lane], lm = a.lam[lane];
     const float al = expf(dl * a.A[h]);
@@ -205,26 +216,28 @@ __global__ void __launch_bounds__(256) k_decode_gen(DecodeArgs a) {
             invC[r] = rsqrtf(sc / N + a.nrm.eps);
         }
     }
-    const int PV = P / VEC;              // vectors per state row
-    const int ngroups = nt / PV;         // rows streamed concurrently
-    const int pv = tid % PV, ng = tid / PV;
-    float4 *hp = reinterpret_cast<float4 *>(a.h + lane * (int64_t)N * P);
     if (FACT)
         for (int k = tid; k < R * N; k += nt) Pb[k] = a.bprev[lane * R * N + k];
-    for (int j = tid; j < NP2; j += nt) {
+    for (int j = tid; j < K; j += nt) {
+        const float phi = a.angle[lane * K + j] + dl * a.theta[lane * K + j];
+        a.angle[lane * K + j] = phi;
+        phs[j] = phi;
+    }
+    __syncthreads();
+    // one (pair, rank) per thread: every rank's loads in flight at once
+    for (int it = tid; it < R * NP2; it += nt) {
+        const int j = it % NP2, r = it / NP2;
         float sn = 0.f, cn = 1.f;
-        if (j < K) {
-            const float phi = a.angle[lane * K + j] + dl * a.theta[lane * K + j];
-            a.angle[lane * K + j] = phi;
-            sincosf(phi, &sn, &cn);
-        }
-#pragma unroll
-        for (int r = 0; r < RT; r++) {
-            if (r >= R) break;
+        if (j < K) sincosf(phs[j], &sn, &cn);
+        {
             const int64_t o = r * N + 2 * j;
             float b0 = ldf(Bg, o), b1 = ldf(Bg, o + 1), c0 = ldf(Cg, o), c1 = ldf(Cg, o + 1);
-            if (a.nrm.wB) { b0 *= invB[r] * a.nrm.wB[2 * j]; b1 *= invB[r] * a.nrm.wB[2 * j + 1]; }
-            if (a.nrm.wC) { c0 *= invC[r] * a.nrm.wC[2 * j]; c1 *= invC[r] * a.nrm.wC[2 * j + 1]; }
+            float ib = 1.f, ic = 1.f;   // this rank's inverse RMS (selected, not indexed)
+#pragma unroll
+            for (int rr = 0; rr < RT; rr++)
+                if (rr == r) { ib = invB[rr]; ic = invC[rr]; }
+            if (a.nrm.wB) { b0 *= ib * a.nrm.wB[2 * j]; b1 *= ib * a.nrm.wB[2 * j + 1]; }
+            if (a.nrm.wC) { c0 *= ic * a.nrm.wC[2 * j]; c1 *= ic * a.nrm.wC[2 * j + 1]; }
             const int64_t bo = (h * R + r) * N + 2 * j;
             if (a.nrm.biasB) { b0 += a.nrm.biasB[bo]; b1 += a.nrm.biasB[bo + 1]; }
             if (a.nrm.biasC) { c0 += a.nrm.biasC[bo]; c1 += a.nrm.biasC[bo + 1]; }
@@ -327,7 +340,7 @@ template <typename T, int RT>
 static cudaError_t launch_decode_gen_rt(const DecodeArgs &a, bool factored, cudaStream_t s) {
     const int threads = 256;
     const int ngroups = threads / (int)(a.P / 4);
-    const size_t smem = sizeof(float) * (3 * RT * a.N + 32 + (size_t)ngroups * RT * a.P);
+    const size_t smem = sizeof(float) * (3 * RT * a.N + 32 + a.N / 2 + (size_t)ngroups * RT * a.P);
     if (factored) k_decode_gen<T, RT, true><<<(unsigned)(a.Bt * a.H), threads, smem, s>>>(a);
     else k_decode_gen<T, RT, false><<<(unsigned)(a.Bt * a.H), threads, smem, s>>>(a);
     count_launch();
