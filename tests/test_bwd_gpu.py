@@ -92,6 +92,13 @@ def test_bwd_siso_small(dtype, T, chunk):
     _assert(_case(inp, chunk, False, True, True, seed=T))
 
 
+@pytest.mark.parametrize("dtype,R", [("bf16", 1), ("f32", 1), ("bf16", 2)])
+def test_bwd_odd_headdim(dtype, R):
+    # P = 5: rows that are not whole 4-byte words in bf16 (copied without cp.async)
+    inp = gen.scan_inputs(2, 23, 2, 5, 6, rank=R, dtype=dtype, seed=605 + R, mimo_weights=R > 1)
+    _assert(_case(inp, 8, R > 1, True, True, seed=11))
+
+
 def test_bwd_siso_no_state_no_seeds():
     inp = gen.scan_inputs(2, 40, 2, 8, 8, dtype="f32", seed=610)
     _assert(_case(inp, 16, False, False, False, seed=3))
