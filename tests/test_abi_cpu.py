@@ -172,6 +172,33 @@ def test_groups_and_rope_pairs_validation(L):
     assert m3.workspace_bytes(m3.M3_WS_SISO, dims(**long3, ngroups=5), m3.M3_BF16) == 0
 
 
+def test_backward_validation(L):
+    """m3_chunked_bwd rejects bad arguments before any launch."""
+    g = m3.Grads(*([None] * len(m3.GRAD_FIELDS)))
+
+    def bwd(d, dy=FAKE, grads=True, ws=None, nbytes=0, dtype=m3.M3_BF16, gx=None):
+        gg = m3.Grads(*([gx] + [None] * (len(m3.GRAD_FIELDS) - 1))) if gx is not None else g
+        return L.m3_chunked_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, dtype, None, None,
+                                None, None, d, dy, None, None, None, ctypes.byref(gg) if grads else None, ws,
+                                nbytes, None)
+
+    assert bwd(dims(), grads=False) == m3.M3_ERR_INVALID_ARG           # no gradient struct
+    assert bwd(dims(), dy=None) == m3.M3_ERR_INVALID_ARG               # dy is required
+    assert bwd(dims(dstate=5)) == m3.M3_ERR_INVALID_ARG
+    assert bwd(dims(chunk=0)) == m3.M3_ERR_INVALID_ARG
+    assert bwd(dims(rank=9)) == m3.M3_ERR_UNSUPPORTED
+    assert bwd(dims(), dtype=7) == m3.M3_ERR_INVALID_ARG
+    assert bwd(dims(nheads=6, ngroups=4)) == m3.M3_ERR_INVALID_ARG      # groups must divide the heads
+    assert bwd(dims(), gx=MIS) == m3.M3_ERR_INVALID_ARG                 # misaligned gradient buffer
+    # the workspace is required and checked before any launch
+    need = m3.workspace_bytes(m3.M3_WS_BWD_SISO, dims(), m3.M3_BF16)
+    assert need > 0
+    assert bwd(dims()) == m3.M3_ERR_WORKSPACE
+    assert bwd(dims(), ws=FAKE, nbytes=need - 16) == m3.M3_ERR_WORKSPACE
+    # workspace grows with the sequence (one entering state per chunk)
+    assert m3.workspace_bytes(m3.M3_WS_BWD_SISO, dims(seqlen=64), m3.M3_BF16) > need
+
+
 def test_workspace_query(L):
     for which in (m3.M3_WS_SISO, m3.M3_WS_MIMO):
         n = m3.workspace_bytes(which, dims(), m3.M3_BF16)
