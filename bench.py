@@ -475,6 +475,51 @@ def run_cpu_baseline(w, target_s=10.0, wall_s=1.5):
                       % (reps, nl, total_lanes, w.c["seqlen"], dt, used)}
 
 
+def decode_oracle_sample(c, nb, steps, threads):
+    """The oracle's decode step (the one the workload's kernel computes: full
+    state, rank R, or factored) over `steps` steps of the first nb sequences,
+    all heads, from a zero state (the time does not depend on the values).
+    Returns (sequences x steps, seconds, threads used)."""
+    import oracle
+    H, P, N, R = c["nheads"], c["headdim"], c["dstate"], c["rank"]
+    factored = c.get("state") == "factored"
+    # the parameters and per-step inputs of the workload's shape, drawn small
+    # (the full prefill is not needed: the time does not depend on the values)
+    inp = gen.scan_inputs(1, 1, H, P, N, rank=R, dtype=c["dtype"], seed=gen.SEED_BASE + 77,
+                          mimo_weights=R > 1)
+    g = inp.pop("generator")
+    A, D = gen.to_f64(inp["A"]), gen.to_f64(inp["D"])
+    Wx = gen.to_f64(inp["Wx"]) if R > 1 else None
+    Wy = gen.to_f64(inp["Wy"]) if R > 1 else None
+    st = [gen.decode_step_inputs(g, nb, H, P, N, rank=R, rank_axis=factored) for _ in range(steps)]
+    st = [{k: gen.to_f64(v) for k, v in s.items()} for s in st]
+    h, u = np.zeros((nb, H, N, P)), np.zeros((nb, H, N, P))
+    a = np.zeros((nb, H, N // 2))
+    bp, xp = np.zeros((nb, H, R, N)), np.zeros((nb, H, P))
+    t0 = time.perf_counter()
+    for s in st:
+        args = (s["x"], s["dt"], A, s["lam"], s["theta"], s["B"], s["C"], D)
+        if factored:
+            _, h, bp, xp, a = oracle.step_decode_factored(*args, h, bp, xp, a, Wx=Wx, Wy=Wy)
+        elif R > 1:
+            _, h, u, a = oracle.mimo_step_decode(*args, h, u, a, Wx=Wx, Wy=Wy, nthreads=threads)
+        else:
+            _, h, u, a = oracle.step_decode(*args, h, u, a, nthreads=threads)
+    used = 1 if factored else min(threads, nb * H)
+    return nb * steps, time.perf_counter() - t0, used
+
+
+def run_cpu_baseline_decode(c, target_s=6.0):
+    cores = os.cpu_count() or 1
+    nb = min(c["batch"], 16)
+    n, dt, used = decode_oracle_sample(c, nb, 2, cores)
+    steps = int(max(2, min(200, 2 * target_s / max(dt, 1e-3))))
+    n, dt, used = decode_oracle_sample(c, nb, steps, cores)
+    return {"value": n / dt, "unit": UNIT, "cores": int(used), "kind": "oracle",
+            "sample": "%d decode steps of %d of %d sequences (all heads), fp64 C step, %.1f s on %d threads"
+                      % (steps, nb, c["batch"], dt, used)}
+
+
 def run_cpu_baseline_bwd(w, target_s=8.0):
     """The oracle's backward (single-threaded C loop) on as many lanes as fit
     about target_s seconds; tokens/s scaled to whole (b, t) tokens."""
@@ -609,8 +654,11 @@ def run_ours(args, world, rank, local):
             "e2e": {"value": round(e2e_val, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "clocks": clk.report(), "gpu_launches": int(launches)}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and isinstance(w, ScanWorkload):
-        line["cpu_baseline"] = (run_cpu_baseline_bwd(w) if isinstance(w, BwdWorkload) else run_cpu_baseline(w))
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        if isinstance(w, DecodeWorkload):
+            line["cpu_baseline"] = run_cpu_baseline_decode(w.c)
+        else:
+            line["cpu_baseline"] = (run_cpu_baseline_bwd(w) if isinstance(w, BwdWorkload) else run_cpu_baseline(w))
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:
@@ -625,6 +673,9 @@ def run_reference(args, world, rank):
         return
     import oracle
     oracle.build_oracle()
+    if "steps" in gen.CONFIGS[args.config]:      # decode workloads: the oracle's decode step
+        run_reference_decode(args, world)
+        return
     bwd = bool(gen.CONFIGS[args.config].get("grad"))
     w = (BwdWorkload if bwd else ScanWorkload).__new__(BwdWorkload if bwd else ScanWorkload)
     w.c = dict(gen.CONFIGS[args.config])
@@ -664,6 +715,27 @@ def run_reference(args, world, rank):
             "impl": "reference",
             "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": int(used), "kind": "oracle",
                              "sample": sample},
+            "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_reference_decode(args, world):
+    c = dict(gen.CONFIGS[args.config])
+    cores = os.cpu_count() or 1
+    nb = min(c["batch"], 16)
+    for _ in range(args.warmup):
+        decode_oracle_sample(c, nb, 1, cores)
+    n, el, used = decode_oracle_sample(c, nb, args.steps, cores)
+    value = n / el
+    line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": c["name"], "batch": c["batch"], "nheads": c["nheads"], "headdim": c["headdim"],
+                       "dstate": c["dstate"], "rank": c["rank"], "state": c.get("state", "full")},
+            "impl": "reference",
+            "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": int(used), "kind": "oracle",
+                             "sample": "%d of %d sequences (all heads) per decode step, fp64 C step"
+                                       % (nb, c["batch"])},
             "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
