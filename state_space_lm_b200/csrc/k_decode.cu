@@ -27,7 +27,7 @@ template <> struct vecf<1> {
 };
 
 template <typename T, int VEC>
-__global__ void __launch_bounds__(256) k_decode(DecodeArgs a) {
+__global__ void __launch_bounds__(256, 5) k_decode(DecodeArgs a) {
     using V = typename vecf<VEC>::type;
     const int64_t lane = blockIdx.x, h = lane % a.H;
     const int P = (int)a.P, N = (int)a.N, NP2 = N / 2, K = (int)a.K;
@@ -43,6 +43,20 @@ __global__ void __launch_bounds__(256) k_decode(DecodeArgs a) {
     float *Cb = Bb + N;        // N
     float *red = Cb + N;       // 32
     float *ypart = red + 32;   // ngroups * P
+
+    const int PV = P / VEC;              // vectors per state row
+    const int ngroups = nt / PV;         // rows streamed concurrently
+    const int pv = tid % PV, ng = tid / PV;
+    {   // start pulling my rows of h and prev_Bx into L2 now, so the state
+        // stream below finds them there instead of waiting on HBM after the prologue
+        const V *hq = reinterpret_cast<const V *>(a.h + lane * (int64_t)N * P) + pv;
+        const V *uq = reinterpret_cast<const V *>(a.prevBx + lane * (int64_t)N * P) + pv;
+        if (ng < ngroups)
+            for (int n = ng; n < N; n += ngroups) {
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(hq + n * PV));
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(uq + n * PV));
+            }
+    }
 
     const float dl = a.dt[lane], lm = a.lam[lane];
     const float al = expf(dl * a.A[h]);
@@ -83,9 +97,6 @@ __global__ void __launch_bounds__(256) k_decode(DecodeArgs a) {
     }
     __syncthreads();
 
-    const int PV = P / VEC;              // vectors per state row
-    const int ngroups = nt / PV;         // rows streamed concurrently
-    const int pv = tid % PV, ng = tid / PV;
     float xv[VEC], yacc[VEC];
 #pragma unroll
     for (int k = 0; k < VEC; k++) {
