@@ -448,6 +448,18 @@ class DecodeWorkload:
                 "l2": "state larger than L2 (%.0f MB vs 126 MB), no flush" % (self.input_bytes / 1e6)}
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def run_cpu_baseline(w, target_s=10.0, wall_s=1.5):
     """Time the oracle as it stands on the host cores on a bounded sample of
     lanes; tokens/s are scaled to whole (b, t) tokens of all heads."""
@@ -470,9 +482,12 @@ def run_cpu_baseline(w, target_s=10.0, wall_s=1.5):
             dt += d1
         used = used2
     tokens = reps * nl * w.c["seqlen"] / H
+    # one thread on one lane, scaled to whole tokens of all heads
+    _, d1, _ = w.oracle_sample(1, 1)
     return {"value": tokens / dt, "unit": UNIT, "cores": int(used), "kind": "oracle",
             "sample": "%d x %d of %d (b,h) lanes x %d tokens, fp64 C loop, %.1f s wall on %d threads"
-                      % (reps, nl, total_lanes, w.c["seqlen"], dt, used)}
+                      % (reps, nl, total_lanes, w.c["seqlen"], dt, used),
+            "one_thread_value": w.c["seqlen"] / H / d1, "cpu_model": cpu_model()}
 
 
 def decode_oracle_sample(c, nb, steps, threads):
