@@ -47,6 +47,10 @@ MUTATIONS = [
      "dsrc[n] += inv * ddst[n] * w[n];"),
     ("backward: lookahead adjoint dropped", "GU[n * P + p] = ga[t] * gh + GUf[n * P + p];",
      "GU[n * P + p] = ga[t] * gh;"),
+    ("backward: dtheta without dt", "g->dtheta[bth * K + i] += dl * Gphi[i];", "g->dtheta[bth * K + i] += Gphi[i];"),
+    ("backward: dt misses the angle term", "if (g->ddt) g->ddt[bth] += theta[bth * K + i] * Gphi[i];", ""),
+    ("backward: a group's B rows overwritten, not summed over its heads",
+     "for (long n = 0; n < N; n++) g->dB[off + n] += tmp[n];", "for (long n = 0; n < N; n++) g->dB[off + n] = tmp[n];"),
 ]
 
 PIN_CASES = [
