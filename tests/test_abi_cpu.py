@@ -213,3 +213,17 @@ def test_workspace_query(L):
     # a missing or short workspace is rejected before any launch
     assert siso(L, long3) == m3.M3_ERR_WORKSPACE
     assert siso(L, long3, ws=FAKE, nbytes=need - 16) == m3.M3_ERR_WORKSPACE
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    """Without the built CUDA library every call raises: there is no other
+    implementation behind the binding's names."""
+    import importlib
+    mod = importlib.reload(m3)
+    monkeypatch.setattr(mod, "LIB", str(tmp_path / "nonexistent_libm3.so"))
+    monkeypatch.setattr(mod, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        mod.lib()
+    with pytest.raises(RuntimeError):
+        mod.limits()
+    importlib.reload(m3)
