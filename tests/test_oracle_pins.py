@@ -367,6 +367,31 @@ def test_factored_decode_from_zero_equals_mimo_loop(oracle_mod, R):
     close(a, a1)
 
 
+def test_factored_and_mimo_decode_with_norm_bias_equal_the_loop(oracle_mod):
+    """QkNorm gains and per-head biases in the decode steps: factored and full
+    state, grouped B/C, partial RoPE, against the one-shot loop."""
+    rng = np.random.default_rng(47)
+    Bt, T, H, G, P, N, R, K = 2, 5, 4, 2, 3, 8, 2, 3
+    inp = _grouped(rng, Bt, T, H, G, P, N, R, K)
+    Wx = 1 + 0.3 * rng.standard_normal((H, R, P))
+    Wy = 1 + 0.3 * rng.standard_normal((H, R, P))
+    nrm = dict(normw_B=1 + 0.2 * rng.standard_normal(N), normw_C=1 + 0.2 * rng.standard_normal(N),
+               bias_B=rng.standard_normal((H, R, N)), bias_C=rng.standard_normal((H, R, N)), eps=1e-5)
+    y1, h1, u1, a1 = oracle_mod.mimo_loop(**inp, Wx=Wx, Wy=Wy, norm=nrm)
+    h, u, a = np.zeros((Bt, H, N, P)), np.zeros((Bt, H, N, P)), np.zeros((Bt, H, K))
+    hf, bp, xp, af = h.copy(), np.zeros((Bt, H, R, N)), np.zeros((Bt, H, P)), a.copy()
+    for t in range(T):
+        yt, h, u, a = oracle_mod.mimo_step_decode(*_tok(inp, t), h, u, a, Wx=Wx, Wy=Wy, norm=nrm)
+        close(yt, y1[:, t])
+        yf, hf, bp, xp, af = oracle_mod.step_decode_factored(*_tok(inp, t), hf, bp, xp, af, Wx=Wx, Wy=Wy,
+                                                             norm=nrm)
+        close(yf, y1[:, t])
+    close(h, h1)
+    close(u, u1)
+    close(hf, h1)
+    close(af, a1)
+
+
 def test_factored_decode_after_prefill(oracle_mod):
     """Schedule 4 + 3: a prefill by the loop, then decode steps on the factored
     state taken from the prefill's last token (its rotated B and its x)."""
