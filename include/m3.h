@@ -65,10 +65,11 @@ typedef enum {
 typedef enum { M3_F32 = 0, M3_BF16 = 1 } m3_dtype;
 
 /* Problem sizes.  rank is ignored by the SISO entry points (taken as 1);
- * chunk is the chunk length of the chunked algorithm (>= 1); seqlen is
- * ignored by the decode steps.  ngroups: B/C groups G (0 = nheads; else
- * nheads % ngroups == 0).  rope_pairs: rotated pairs K (0 = dstate/2; else
- * 1 <= K <= dstate/2).  Anything else is M3_ERR_INVALID_ARG. */
+ * chunk is the chunk length of the chunked algorithm (>= 1; a request of
+ * 2^30 or more behaves as 2^30); seqlen is ignored by the decode steps.
+ * ngroups: B/C groups G (0 = nheads; else nheads % ngroups == 0).
+ * rope_pairs: rotated pairs K (0 = dstate/2; else 1 <= K <= dstate/2).
+ * Anything else is M3_ERR_INVALID_ARG. */
 typedef struct {
     int64_t batch, seqlen, nheads, headdim, dstate, rank, chunk;
     int64_t ngroups, rope_pairs;
@@ -87,7 +88,9 @@ typedef struct {
 } m3_bcnorm;
 
 /* Limits of this build: dstate <= 256 and even, headdim <= 256,
- * dstate * headdim <= 16384, rank <= 8 (MIMO). */
+ * dstate * headdim <= 16384, rank <= 8 (MIMO); batch <= 2^24, nheads <= 4096,
+ * batch * nheads <= 2^31 - 1 lanes, and batch * seqlen * nheads *
+ * max(headdim, dstate) <= 2^46.  Sizes past them are M3_ERR_UNSUPPORTED. */
 typedef struct {
     int64_t max_dstate, max_headdim, max_state_elems, max_rank;
 } m3_limits;

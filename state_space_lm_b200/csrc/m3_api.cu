@@ -3,6 +3,7 @@
 // allocates, frees or synchronises.
 #include <atomic>
 #include <cmath>
+#include <initializer_list>
 
 #include "m3_internal.cuh"
 
@@ -16,6 +17,26 @@ using namespace m3;
 namespace {
 
 constexpr int64_t kMaxDstate = 256, kMaxHeaddim = 256, kMaxStateElems = 16384, kMaxRank = 8;
+// Every kernel runs one CTA per (batch, head) lane in a 1-D grid, and no
+// tensor may hold more than 2^46 elements (far beyond device memory), so
+// that every index product below stays well inside int64.
+constexpr int64_t kMaxLanes = 0x7fffffff, kMaxElems = (int64_t)1 << 46;
+
+// Product of non-negative sizes, saturated at kMaxElems + 1.
+int64_t sat_product(std::initializer_list<int64_t> f) {
+    for (int64_t v : f)
+        if (v == 0) return 0;
+    int64_t p = 1;
+    for (int64_t v : f) {
+        if (v > kMaxElems || p > kMaxElems / v) return kMaxElems + 1;
+        p *= v;
+    }
+    return p;
+}
+
+// The requested chunk as an int: any request of 2^30 tokens or more behaves
+// as 2^30 (longer than any supported sequence).
+inline int chunk_request(int64_t c) { return (int)(c < ((int64_t)1 << 30) ? c : ((int64_t)1 << 30)); }
 
 inline bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
@@ -43,6 +64,9 @@ m3_status check_core_dims(const m3_dims &d, bool need_seq) {
         return M3_ERR_UNSUPPORTED;
     if (d.batch > (int64_t)1 << 24 || d.nheads > 4096 || (need_seq && d.seqlen > ((int64_t)1 << 31)))
         return M3_ERR_UNSUPPORTED;
+    if (d.batch * d.nheads > kMaxLanes) return M3_ERR_UNSUPPORTED;
+    const int64_t width = d.headdim > d.dstate ? d.headdim : d.dstate;
+    if (need_seq && sat_product({d.batch, d.seqlen, d.nheads, width}) > kMaxElems) return M3_ERR_UNSUPPORTED;
     return M3_OK;
 }
 
@@ -115,7 +139,7 @@ m3_status chunked_common(const void *x, const float *dt, const float *A, const f
     a.G = G; a.K = K;
     a.mimo_layout = mimo ? 1 : 0;
     a.ws = workspace;
-    a.Q = (int)d.chunk;
+    a.Q = chunk_request(d.chunk);
     if (scan_tc_supported(a, dtype)) return launched(launch_scan_tc(a, (cudaStream_t)stream));
     a.Q = q;
     return launched(launch_scan_simt(a, dtype, (cudaStream_t)stream));
@@ -168,7 +192,7 @@ size_t m3_workspace_bytes(int which, m3_dims d, m3_dtype dtype) {
     if (resolve_groups(d, a.G, a.K) != M3_OK) return 0;
     a.Bt = d.batch; a.T = d.seqlen; a.H = d.nheads; a.P = d.headdim; a.N = d.dstate;
     a.R = which == M3_WS_MIMO ? d.rank : 1;
-    a.Q = (int)d.chunk; a.mimo_layout = which == M3_WS_MIMO ? 1 : 0;
+    a.Q = chunk_request(d.chunk); a.mimo_layout = which == M3_WS_MIMO ? 1 : 0;
     if (!scan_tc_supported(a, dtype)) return 0;
     return scan_tc_workspace_bytes(d.batch, d.nheads, d.seqlen);
 }
@@ -176,6 +200,7 @@ size_t m3_workspace_bytes(int which, m3_dims d, m3_dtype dtype) {
 m3_status m3_discretize(const float *dt, const float *A, const float *lam, m3_dims d, float *alpha,
                         float *beta, float *gamma, void *stream) {
     if (d.batch < 0 || d.seqlen < 0 || d.nheads < 1) return M3_ERR_INVALID_ARG;
+    if (sat_product({d.batch, d.seqlen, d.nheads}) > kMaxElems) return M3_ERR_UNSUPPORTED;
     M3_REQ(A);
     if (d.batch * d.seqlen == 0) return M3_OK;
     M3_REQ(dt); M3_REQ(lam); M3_REQ(alpha); M3_REQ(beta); M3_REQ(gamma);

@@ -213,6 +213,36 @@ def test_workspace_query(L):
     # a missing or short workspace is rejected before any launch
     assert siso(L, long3) == m3.M3_ERR_WORKSPACE
     assert siso(L, long3, ws=FAKE, nbytes=need - 16) == m3.M3_ERR_WORKSPACE
+    # a chunk request past 2^30 behaves as 2^30: the same path and scratch as
+    # any other multiple of the kernel's 64-row chunk
+    for huge in (1 << 30, (1 << 31) + 128, (1 << 32) + 128, (1 << 62)):
+        big = dims(batch=1, seqlen=32768, nheads=32, headdim=64, dstate=128, chunk=huge)
+        assert m3.workspace_bytes(m3.M3_WS_SISO, big, m3.M3_BF16) == need, huge
+        assert siso(L, big) == m3.M3_ERR_WORKSPACE, huge
+
+
+def test_sizes_past_the_index_limits(L):
+    """Lane counts past a 1-D grid and tensors past 2^46 elements are
+    M3_ERR_UNSUPPORTED at every entry point, before any launch, with no
+    integer overflow in the checks themselves."""
+    g = m3.Grads(*([None] * len(m3.GRAD_FIELDS)))
+    lanes = dict(batch=1 << 24, nheads=256)                             # 2^32 lanes
+    elems = dict(batch=1 << 20, seqlen=1 << 30, nheads=16, headdim=64, dstate=128)   # 2^61 elements
+    wrap = dict(batch=1 << 24, seqlen=1 << 31, nheads=4096, headdim=256, dstate=256)  # 2^75: wraps int64
+    for kw in (lanes, elems, wrap):
+        d = dims(**kw)
+        assert siso(L, d) == m3.M3_ERR_UNSUPPORTED, kw
+        assert L.m3_rope_bc(FAKE, FAKE, m3.M3_BF16, FAKE, FAKE, None, None, d, FAKE, FAKE, None,
+                            None) == m3.M3_ERR_UNSUPPORTED, kw
+        assert L.m3_chunked_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, m3.M3_BF16, None,
+                                None, None, None, d, FAKE, None, None, None, ctypes.byref(g), None, 0,
+                                None) == m3.M3_ERR_UNSUPPORTED, kw
+        assert m3.workspace_bytes(m3.M3_WS_BWD_SISO, d, m3.M3_BF16) == 0, kw
+    d = dims(**lanes)
+    assert L.m3_step_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, m3.M3_BF16, None, d,
+                            FAKE, FAKE, FAKE, FAKE, None) == m3.M3_ERR_UNSUPPORTED
+    for big in (dims(batch=1 << 40, seqlen=1 << 40), dims(batch=1 << 30, seqlen=1 << 17, nheads=1 << 20)):
+        assert L.m3_discretize(FAKE, FAKE, FAKE, big, FAKE, FAKE, FAKE, None) == m3.M3_ERR_UNSUPPORTED
 
 
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):
