@@ -158,6 +158,39 @@ def _ptr(t):
     return t.data_ptr()
 
 
+def _expect(where, dev, name, t, numel, dtype, required=True):
+    """The library sees only pointers and the sizes in m3_dims, so the binding
+    checks each tensor against those sizes (element count, dtype, device)
+    before the call: a tensor shorter than the sizes say would otherwise be
+    read or written past its end."""
+    if t is None:
+        if required:
+            raise ValueError("%s: %s is required" % (where, name))
+        return
+    if t.numel() != numel:
+        raise ValueError("%s: %s has %d elements (shape %s), the sizes need %d"
+                         % (where, name, t.numel(), tuple(t.shape), numel))
+    if t.dtype != dtype:
+        raise ValueError("%s: %s is %s, expected %s" % (where, name, t.dtype, dtype))
+    if t.device != dev:
+        raise ValueError("%s: %s is on %s, expected %s" % (where, name, t.device, dev))
+
+
+def _io_dtype(where, t):
+    if t.dtype not in _DTYPE:
+        raise ValueError("%s: x, B, C must be float32 or bfloat16, got %s" % (where, t.dtype))
+    return t.dtype
+
+
+def _expect_norm(where, dev, norm, H, R, N):
+    if norm is None:
+        return
+    for k in ("normw_B", "normw_C"):
+        _expect(where, dev, k, norm.get(k), N, torch.float32, required=False)
+    for k in ("bias_B", "bias_C"):
+        _expect(where, dev, k, norm.get(k), H * R * N, torch.float32, required=False)
+
+
 def _stream(stream):
     s = torch.cuda.current_stream() if stream is None else stream
     return s.cuda_stream
@@ -184,6 +217,10 @@ def discretize(dt, A, lam, out=None, stream=None):
     """S1: alpha, beta, gamma (Bt,T,H) fp32."""
     Bt, T, H = dt.shape
     al, be, ga = out if out is not None else tuple(torch.empty_like(dt) for _ in range(3))
+    w, f, n, dev = "m3_discretize", torch.float32, Bt * T * H, dt.device
+    for name, t in (("dt", dt), ("lam", lam), ("alpha", al), ("beta", be), ("gamma", ga)):
+        _expect(w, dev, name, t, n, f)
+    _expect(w, dev, "A", A, H, f)
     d = Dims(Bt, T, H, 1, 2, 1, 1, 0, 0)
     _check(lib().m3_discretize(_ptr(dt), _ptr(A), _ptr(lam), d, _ptr(al), _ptr(be), _ptr(ga),
                                _stream(stream)), "m3_discretize")
@@ -206,6 +243,15 @@ def rope_bc(B, C, theta, dt, angle0=None, norm=None, out=None, stream=None):
                torch.empty(shape, device=B.device, dtype=B.dtype),
                torch.empty(Bt, H, K, device=B.device, dtype=torch.float32))
     Br, Cr, ang = out
+    w, f, dev, io = "m3_rope_bc", torch.float32, B.device, _io_dtype("m3_rope_bc", B)
+    _expect(w, dev, "C", C, B.numel(), io)
+    _expect(w, dev, "theta", theta, Bt * T * H * K, f)
+    _expect(w, dev, "dt", dt, Bt * T * H, f)
+    _expect(w, dev, "angle0", angle0, Bt * H * K, f, required=False)
+    _expect(w, dev, "B_rot", Br, Bt * T * H * R * N, io)
+    _expect(w, dev, "C_rot", Cr, Bt * T * H * R * N, io)
+    _expect(w, dev, "angle_final", ang, Bt * H * K, f, required=False)
+    _expect_norm(w, dev, norm, H, R, N)
     nptr, keep = _norm(norm)
     d = Dims(Bt, T, H, 1, N, R, 1, G, K)
     _check(lib().m3_rope_bc(_ptr(B), _ptr(C), _DTYPE[B.dtype], _ptr(theta), _ptr(dt), _ptr(angle0),
@@ -223,10 +269,46 @@ def _state_outs(x, N, P, K, out):
             torch.empty(Bt, H, K, device=dev, dtype=torch.float32))
 
 
+def _expect_scan(w, x, dt, A, lam, theta, B, C, D, R, W_x=None, W_y=None, norm=None, h0=None, prevBx0=None,
+                 angle0=None):
+    """Element counts of the chunked scan's inputs: x (Bt,T,H,P); dt, lam
+    (Bt,T,H); A, D (H); theta (Bt,T,H,K); B, C (Bt,T,G,[R,]N); W_x, W_y
+    (H,R,P); h0, prevBx0 (Bt,H,N,P); angle0 (Bt,H,K)."""
+    Bt, T, H, P = x.shape
+    N, G, K = B.shape[-1], B.shape[2], theta.shape[-1]
+    f, dev, io = torch.float32, x.device, _io_dtype(w, x)
+    for name, t in (("dt", dt), ("lam", lam)):
+        _expect(w, dev, name, t, Bt * T * H, f)
+    for name, t in (("A", A), ("D", D)):
+        _expect(w, dev, name, t, H, f)
+    _expect(w, dev, "theta", theta, Bt * T * H * K, f)
+    _expect(w, dev, "B", B, Bt * T * G * R * N, io)
+    _expect(w, dev, "C", C, Bt * T * G * R * N, io)
+    for name, t in (("W_x", W_x), ("W_y", W_y)):
+        _expect(w, dev, name, t, H * R * P, f, required=False)
+    for name, t in (("h0", h0), ("prevBx0", prevBx0)):
+        _expect(w, dev, name, t, Bt * H * N * P, f, required=False)
+    _expect(w, dev, "angle0", angle0, Bt * H * K, f, required=False)
+    _expect_norm(w, dev, norm, H, R, N)
+    return io
+
+
+def _expect_state_outs(w, x, N, K, outs):
+    Bt, T, H, P = x.shape
+    y, hf, uf, af = outs
+    f, dev = torch.float32, x.device
+    _expect(w, dev, "y", y, x.numel(), x.dtype)
+    _expect(w, dev, "h_final", hf, Bt * H * N * P, f, required=False)
+    _expect(w, dev, "prevBx_final", uf, Bt * H * N * P, f, required=False)
+    _expect(w, dev, "angle_final", af, Bt * H * K, f, required=False)
+
+
 def _workspace(which, d, dtype, workspace, dev):
     need = workspace_bytes(which, d, dtype)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if workspace is not None and workspace.device != dev:
+        raise ValueError("workspace is on %s, expected %s" % (workspace.device, dev))
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     return workspace, nbytes
 
@@ -237,7 +319,10 @@ def siso_chunked_fwd(x, dt, A, lam, theta, B, C, D, chunk, norm=None, h0=None, p
     (Bt,H,K).  B, C (Bt,T,G,N) with G dividing H; theta (Bt,T,H,K)."""
     Bt, T, H, P = x.shape
     N, G, K = B.shape[-1], B.shape[2], theta.shape[-1]
+    w = "m3_siso_chunked_fwd"
+    _expect_scan(w, x, dt, A, lam, theta, B, C, D, 1, norm=norm, h0=h0, prevBx0=prevBx0, angle0=angle0)
     y, hf, uf, af = _state_outs(x, N, P, K, out)
+    _expect_state_outs(w, x, N, K, (y, hf, uf, af))
     d = Dims(Bt, T, H, P, N, 1, int(chunk), G, K)
     dtype = _DTYPE[x.dtype]
     ws, nbytes = _workspace(M3_WS_SISO, d, dtype, workspace, x.device)
@@ -254,7 +339,10 @@ def mimo_chunked_fwd(x, dt, A, lam, theta, B, C, D, chunk, W_x=None, W_y=None, n
     """S4: B, C (Bt,T,G,R,N); W_x, W_y (H,R,P) or None for ones."""
     Bt, T, H, P = x.shape
     R, N, G, K = B.shape[-2], B.shape[-1], B.shape[2], theta.shape[-1]
+    w = "m3_mimo_chunked_fwd"
+    _expect_scan(w, x, dt, A, lam, theta, B, C, D, R, W_x, W_y, norm, h0, prevBx0, angle0)
     y, hf, uf, af = _state_outs(x, N, P, K, out)
+    _expect_state_outs(w, x, N, K, (y, hf, uf, af))
     d = Dims(Bt, T, H, P, N, R, int(chunk), G, K)
     dtype = _DTYPE[x.dtype]
     ws, nbytes = _workspace(M3_WS_MIMO, d, dtype, workspace, x.device)
@@ -267,6 +355,29 @@ def mimo_chunked_fwd(x, dt, A, lam, theta, B, C, D, chunk, W_x=None, W_y=None, n
     return y, hf, uf, af
 
 
+def _expect_decode(w, x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, R, y, h, angle, W_x=None, W_y=None,
+                   norm=None):
+    """Element counts of a decode step's arguments: x_t, y (Bt,H,P); dt_t,
+    lam_t (Bt,H); A, D (H); theta_t, angle (Bt,H,K); B_t, C_t (Bt,G,[R,]N);
+    W_x, W_y (H,R,P); h (Bt,H,N,P)."""
+    Bt, H, P = x_t.shape
+    N, G, K = B_t.shape[-1], B_t.shape[1], theta_t.shape[-1]
+    f, dev, io = torch.float32, x_t.device, _io_dtype(w, x_t)
+    for name, t in (("dt_t", dt_t), ("lam_t", lam_t)):
+        _expect(w, dev, name, t, Bt * H, f)
+    for name, t in (("A", A), ("D", D)):
+        _expect(w, dev, name, t, H, f)
+    _expect(w, dev, "theta_t", theta_t, Bt * H * K, f)
+    _expect(w, dev, "B_t", B_t, Bt * G * R * N, io)
+    _expect(w, dev, "C_t", C_t, Bt * G * R * N, io)
+    for name, t in (("W_x", W_x), ("W_y", W_y)):
+        _expect(w, dev, name, t, H * R * P, f, required=False)
+    _expect(w, dev, "y_t", y, Bt * H * P, io)
+    _expect(w, dev, "h", h, Bt * H * N * P, f)
+    _expect(w, dev, "angle", angle, Bt * H * K, f)
+    _expect_norm(w, dev, norm, H, R, N)
+
+
 def step_decode(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, prevBx, angle, norm=None, y_out=None,
                 stream=None):
     """S5: one decode step; B_t, C_t (Bt,G,N); theta_t (Bt,H,K); h, prevBx, angle
@@ -274,6 +385,9 @@ def step_decode(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, prevBx, angle, nor
     Bt, H, P = x_t.shape
     N, G, K = B_t.shape[-1], B_t.shape[1], theta_t.shape[-1]
     y = torch.empty_like(x_t) if y_out is None else y_out
+    w = "m3_step_decode"
+    _expect_decode(w, x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, 1, y, h, angle, norm=norm)
+    _expect(w, x_t.device, "prevBx", prevBx, h.numel(), torch.float32)
     d = Dims(Bt, 1, H, P, N, 1, 1, G, K)
     nptr, keep = _norm(norm)
     _check(lib().m3_step_decode(_ptr(x_t), _ptr(dt_t), _ptr(A), _ptr(lam_t), _ptr(theta_t),
@@ -290,6 +404,9 @@ def mimo_step_decode(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, prevBx, angle
     Bt, H, P = x_t.shape
     R, N, G, K = B_t.shape[-2], B_t.shape[-1], B_t.shape[1], theta_t.shape[-1]
     y = torch.empty_like(x_t) if y_out is None else y_out
+    w = "m3_mimo_step_decode"
+    _expect_decode(w, x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, R, y, h, angle, W_x, W_y, norm)
+    _expect(w, x_t.device, "prevBx", prevBx, h.numel(), torch.float32)
     d = Dims(Bt, 1, H, P, N, R, 1, G, K)
     nptr, keep = _norm(norm)
     _check(lib().m3_mimo_step_decode(_ptr(x_t), _ptr(dt_t), _ptr(A), _ptr(lam_t), _ptr(theta_t), _ptr(B_t),
@@ -307,6 +424,10 @@ def step_decode_factored(x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, h, b_prev, x
     Bt, H, P = x_t.shape
     R, N, G, K = B_t.shape[-2], B_t.shape[-1], B_t.shape[1], theta_t.shape[-1]
     y = torch.empty_like(x_t) if y_out is None else y_out
+    w = "m3_step_decode_factored"
+    _expect_decode(w, x_t, dt_t, A, lam_t, theta_t, B_t, C_t, D, R, y, h, angle, W_x, W_y, norm)
+    _expect(w, x_t.device, "b_prev", b_prev, Bt * H * R * N, torch.float32)
+    _expect(w, x_t.device, "x_prev", x_prev, Bt * H * P, torch.float32)
     d = Dims(Bt, 1, H, P, N, R, 1, G, K)
     nptr, keep = _norm(norm)
     _check(lib().m3_step_decode_factored(_ptr(x_t), _ptr(dt_t), _ptr(A), _ptr(lam_t), _ptr(theta_t),
@@ -330,6 +451,12 @@ def chunked_bwd(x, dt, A, lam, theta, B, C, D, dy, chunk, W_x=None, W_y=None, no
     R = B.shape[3] if B.dim() == 5 else 1
     N, G, K = B.shape[-1], B.shape[2], theta.shape[-1]
     mimo = B.dim() == 5
+    w, f = "m3_chunked_bwd", torch.float32
+    io = _expect_scan(w, x, dt, A, lam, theta, B, C, D, R, W_x, W_y, norm, h0, prevBx0, angle0)
+    _expect(w, x.device, "dy", dy, x.numel(), io)
+    for name, t, n in (("dh_final", dh_final, Bt * H * N * P), ("dprevBx_final", dprevBx_final, Bt * H * N * P),
+                       ("dangle_final", dangle_final, Bt * H * K)):
+        _expect(w, x.device, name, t, n, f, required=False)
     if want is None:
         want = tuple(k for k in GRAD_FIELDS if mimo or k not in ("dW_x", "dW_y"))
     dev = x.device
@@ -342,6 +469,11 @@ def chunked_bwd(x, dt, A, lam, theta, B, C, D, dy, chunk, W_x=None, W_y=None, no
     pre = out or {}
     out = {k: (pre[k] if k in pre else torch.empty(shapes[k], device=dev, dtype=torch.float32)) for k in want
            if k not in off or nm.get(off[k]) is not None}
+    for k, t in out.items():
+        n = 1
+        for e in shapes[k]:
+            n *= e
+        _expect(w, dev, k, t, n, f)
     g = Grads(*[_ptr(out.get(k)) for k in GRAD_FIELDS])
     d = Dims(Bt, T, H, P, N, R if mimo else 1, int(chunk), G, K)
     dtype = _DTYPE[x.dtype]
