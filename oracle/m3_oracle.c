@@ -40,9 +40,23 @@
  */
 #include <math.h>
 #include <pthread.h>
+#include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
 #include <unistd.h>
+
+/* Host allocation that never returns NULL: the oracle is a checker, so
+ * running out of memory ends the process loudly instead of yielding a
+ * partial result. */
+static void *xmalloc(size_t n)
+{
+    void *p = malloc(n ? n : 1);
+    if (!p) {
+        fputs("m3_oracle: out of host memory\n", stderr);
+        abort();
+    }
+    return p;
+}
 
 typedef struct {
     long batch, seqlen, nheads, headdim, dstate, rank;
@@ -136,8 +150,8 @@ int m3o_rope_bc(const double *B, const double *C, const double *theta,
     if (N <= 0 || (N & 1)) return -1;
     long G = n_groups(d), K = n_pairs(d);
     if (H % G || K < 1 || K > N / 2) return -1;
-    double *phi = (double *)malloc(sizeof(double) * K);
-    double *tmp = (double *)malloc(sizeof(double) * N);
+    double *phi = (double *)xmalloc(sizeof(double) * K);
+    double *tmp = (double *)xmalloc(sizeof(double) * N);
     for (long b = 0; b < Bt; b++)
         for (long h = 0; h < H; h++) {
             for (long i = 0; i < K; i++)
@@ -190,13 +204,13 @@ static void siso_lane(const lane_job *J, long b, long h)
 {
     long T = J->d.seqlen, H = J->d.nheads, P = J->d.headdim, N = J->d.dstate;
     long NP = N * P;
-    double *hs = (double *)malloc(sizeof(double) * NP);
-    double *Up = (double *)malloc(sizeof(double) * NP);
+    double *hs = (double *)xmalloc(sizeof(double) * NP);
+    double *Up = (double *)xmalloc(sizeof(double) * NP);
     long K = n_pairs(J->d);
-    double *phi = (double *)malloc(sizeof(double) * K);
-    double *tmp = (double *)malloc(sizeof(double) * N);
-    double *Bb = (double *)malloc(sizeof(double) * N);
-    double *Cb = (double *)malloc(sizeof(double) * N);
+    double *phi = (double *)xmalloc(sizeof(double) * K);
+    double *tmp = (double *)xmalloc(sizeof(double) * N);
+    double *Bb = (double *)xmalloc(sizeof(double) * N);
+    double *Cb = (double *)xmalloc(sizeof(double) * N);
     long lane = b * H + h;
     for (long k = 0; k < NP; k++) {
         hs[k] = J->h0 ? J->h0[lane * NP + k] : 0.0;
@@ -252,15 +266,15 @@ static void mimo_lane(const lane_job *J, long b, long h)
     long T = J->d.seqlen, H = J->d.nheads, P = J->d.headdim, N = J->d.dstate;
     long R = J->d.rank;
     long NP = N * P;
-    double *hs = (double *)malloc(sizeof(double) * NP);
-    double *Up = (double *)malloc(sizeof(double) * NP);
-    double *Ut = (double *)malloc(sizeof(double) * NP);
+    double *hs = (double *)xmalloc(sizeof(double) * NP);
+    double *Up = (double *)xmalloc(sizeof(double) * NP);
+    double *Ut = (double *)xmalloc(sizeof(double) * NP);
     long K = n_pairs(J->d);
-    double *phi = (double *)malloc(sizeof(double) * K);
-    double *tmp = (double *)malloc(sizeof(double) * N);
-    double *Bb = (double *)malloc(sizeof(double) * R * N);
-    double *Cb = (double *)malloc(sizeof(double) * R * N);
-    double *Xr = (double *)malloc(sizeof(double) * R * P);
+    double *phi = (double *)xmalloc(sizeof(double) * K);
+    double *tmp = (double *)xmalloc(sizeof(double) * N);
+    double *Bb = (double *)xmalloc(sizeof(double) * R * N);
+    double *Cb = (double *)xmalloc(sizeof(double) * R * N);
+    double *Xr = (double *)xmalloc(sizeof(double) * R * P);
     long lane = b * H + h;
     for (long k = 0; k < NP; k++) {
         hs[k] = J->h0 ? J->h0[lane * NP + k] : 0.0;
@@ -335,17 +349,17 @@ static void siso_chunked_lane(const lane_job *J, long b, long h)
     long NP = N * P;
     long lane = b * H + h;
     const m3o_bcnorm *nr = J->nrm;
-    double *Bb = (double *)malloc(sizeof(double) * T * N);
-    double *Cb = (double *)malloc(sizeof(double) * T * N);
+    double *Bb = (double *)xmalloc(sizeof(double) * T * N);
+    double *Cb = (double *)xmalloc(sizeof(double) * T * N);
     long K = n_pairs(J->d);
-    double *phi = (double *)malloc(sizeof(double) * K);
-    double *tmp = (double *)malloc(sizeof(double) * N);
-    double *la = (double *)malloc(sizeof(double) * T);   /* log alpha */
-    double *ga = (double *)malloc(sizeof(double) * T);
-    double *w = (double *)malloc(sizeof(double) * T);
-    double *g = (double *)malloc(sizeof(double) * NP);
-    double *gn = (double *)malloc(sizeof(double) * NP);
-    double *cum = (double *)malloc(sizeof(double) * Q);
+    double *phi = (double *)xmalloc(sizeof(double) * K);
+    double *tmp = (double *)xmalloc(sizeof(double) * N);
+    double *la = (double *)xmalloc(sizeof(double) * T);   /* log alpha */
+    double *ga = (double *)xmalloc(sizeof(double) * T);
+    double *w = (double *)xmalloc(sizeof(double) * T);
+    double *g = (double *)xmalloc(sizeof(double) * NP);
+    double *gn = (double *)xmalloc(sizeof(double) * NP);
+    double *cum = (double *)xmalloc(sizeof(double) * Q);
     for (long i = 0; i < K; i++)
         phi[i] = J->angle0 ? J->angle0[lane * K + i] : 0.0;
     for (long t = 0; t < T; t++) {
@@ -443,16 +457,22 @@ static int run_lanes(lane_job *proto, int nthreads)
         nthreads = nc > 0 ? (int)nc : 1;
     }
     if (nthreads > lanes) nthreads = (int)lanes;
-    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * nthreads);
-    lane_job *jobs = (lane_job *)malloc(sizeof(lane_job) * nthreads);
+    pthread_t *th = (pthread_t *)xmalloc(sizeof(pthread_t) * nthreads);
+    lane_job *jobs = (lane_job *)xmalloc(sizeof(lane_job) * nthreads);
     for (int i = 0; i < nthreads; i++) {
         jobs[i] = *proto;
         jobs[i].lane_begin = lanes * i / nthreads;
         jobs[i].lane_end = lanes * (i + 1) / nthreads;
     }
-    for (int i = 1; i < nthreads; i++) pthread_create(&th[i], NULL, lane_worker, &jobs[i]);
+    char *started = (char *)xmalloc((size_t)nthreads);
+    for (int i = 1; i < nthreads; i++) started[i] = pthread_create(&th[i], NULL, lane_worker, &jobs[i]) == 0;
     lane_worker(&jobs[0]);
-    for (int i = 1; i < nthreads; i++) pthread_join(th[i], NULL);
+    /* a job whose thread could not start runs here, so every lane is done */
+    for (int i = 1; i < nthreads; i++) {
+        if (started[i]) pthread_join(th[i], NULL);
+        else lane_worker(&jobs[i]);
+    }
+    free(started);
     free(th);
     free(jobs);
     return nthreads;
@@ -542,9 +562,9 @@ int m3o_step_decode(const double *x, const double *dt, const double *A,
     if (!h || !prevBx || !angle) return -1;
     d.seqlen = 1;
     long lanes = d.batch * d.nheads, NP = d.dstate * d.headdim;
-    double *h1 = (double *)malloc(sizeof(double) * (lanes * NP + 1));
-    double *u1 = (double *)malloc(sizeof(double) * (lanes * NP + 1));
-    double *a1 = (double *)malloc(sizeof(double) * (lanes * n_pairs(d) + 1));
+    double *h1 = (double *)xmalloc(sizeof(double) * (lanes * NP + 1));
+    double *u1 = (double *)xmalloc(sizeof(double) * (lanes * NP + 1));
+    double *a1 = (double *)xmalloc(sizeof(double) * (lanes * n_pairs(d) + 1));
     int rc = m3o_siso_loop(x, dt, A, lam, theta, B, C, D, nrm, h, prevBx, angle,
                            d, y, h1, u1, a1, nthreads);
     if (rc >= 0) {
@@ -569,9 +589,9 @@ int m3o_mimo_step_decode(const double *x, const double *dt, const double *A,
     if (!h || !prevBx || !angle) return -1;
     d.seqlen = 1;
     long lanes = d.batch * d.nheads, NP = d.dstate * d.headdim;
-    double *h1 = (double *)malloc(sizeof(double) * (lanes * NP + 1));
-    double *u1 = (double *)malloc(sizeof(double) * (lanes * NP + 1));
-    double *a1 = (double *)malloc(sizeof(double) * (lanes * n_pairs(d) + 1));
+    double *h1 = (double *)xmalloc(sizeof(double) * (lanes * NP + 1));
+    double *u1 = (double *)xmalloc(sizeof(double) * (lanes * NP + 1));
+    double *a1 = (double *)xmalloc(sizeof(double) * (lanes * n_pairs(d) + 1));
     int rc = m3o_mimo_loop(x, dt, A, lam, theta, B, C, D, Wx, Wy, nrm, h, prevBx, angle,
                            d, y, h1, u1, a1, nthreads);
     if (rc >= 0) {
@@ -608,11 +628,11 @@ int m3o_step_decode_factored(const double *x, const double *dt, const double *A,
         return -1;
     d.seqlen = 1;
     long H = d.nheads, P = d.headdim, N = d.dstate, R = d.rank, NP = N * P, K = n_pairs(d);
-    double *tmp = (double *)malloc(sizeof(double) * N);
-    double *Bb = (double *)malloc(sizeof(double) * R * N);
-    double *Cb = (double *)malloc(sizeof(double) * R * N);
-    double *Xr = (double *)malloc(sizeof(double) * R * P);
-    double *Xp = (double *)malloc(sizeof(double) * R * P);
+    double *tmp = (double *)xmalloc(sizeof(double) * N);
+    double *Bb = (double *)xmalloc(sizeof(double) * R * N);
+    double *Cb = (double *)xmalloc(sizeof(double) * R * N);
+    double *Xr = (double *)xmalloc(sizeof(double) * R * P);
+    double *Xp = (double *)xmalloc(sizeof(double) * R * P);
     for (long lane = 0; lane < d.batch * H; lane++) {
         long hh = lane % H;
         double dl = dt[lane], lm = lam[lane];
@@ -755,28 +775,28 @@ int m3o_mimo_loop_bwd(const double *x, const double *dt, const double *A,
     double eps = nrm ? nrm->eps : 0.0;
     const double *wB = nrm ? nrm->normw_B : NULL, *wC = nrm ? nrm->normw_C : NULL;
 
-    double *phis = (double *)malloc(sizeof(double) * (T + 1) * K);   /* Phi_{t-1}, t = 0..T */
-    double *Bp = (double *)malloc(sizeof(double) * (T * RN + 1));    /* QkNorm'd + bias'd */
-    double *Cp = (double *)malloc(sizeof(double) * (T * RN + 1));
-    double *Bb = (double *)malloc(sizeof(double) * (T * RN + 1));    /* rotated */
-    double *Cb = (double *)malloc(sizeof(double) * (T * RN + 1));
-    double *X = (double *)malloc(sizeof(double) * (T * RP + 1));     /* W_x[r] x_t */
-    double *al = (double *)malloc(sizeof(double) * (T + 1));
-    double *be = (double *)malloc(sizeof(double) * (T + 1));
-    double *ga = (double *)malloc(sizeof(double) * (T + 1));
-    double *hs = (double *)malloc(sizeof(double) * (T + 1) * NP);    /* h_{t-1}, t = 0..T */
-    double *Ut = (double *)malloc(sizeof(double) * NP);
-    double *Um = (double *)malloc(sizeof(double) * NP);
-    double *Gh = (double *)malloc(sizeof(double) * NP);
-    double *GU = (double *)malloc(sizeof(double) * NP);
-    double *GUf = (double *)malloc(sizeof(double) * NP);
-    double *Gphi = (double *)malloc(sizeof(double) * K);
-    double *dBb = (double *)malloc(sizeof(double) * RN);
-    double *dCb = (double *)malloc(sizeof(double) * RN);
-    double *dBp = (double *)malloc(sizeof(double) * N);
-    double *dCp = (double *)malloc(sizeof(double) * N);
-    double *dX = (double *)malloc(sizeof(double) * RP);
-    double *tmp = (double *)malloc(sizeof(double) * N);
+    double *phis = (double *)xmalloc(sizeof(double) * (T + 1) * K);   /* Phi_{t-1}, t = 0..T */
+    double *Bp = (double *)xmalloc(sizeof(double) * (T * RN + 1));    /* QkNorm'd + bias'd */
+    double *Cp = (double *)xmalloc(sizeof(double) * (T * RN + 1));
+    double *Bb = (double *)xmalloc(sizeof(double) * (T * RN + 1));    /* rotated */
+    double *Cb = (double *)xmalloc(sizeof(double) * (T * RN + 1));
+    double *X = (double *)xmalloc(sizeof(double) * (T * RP + 1));     /* W_x[r] x_t */
+    double *al = (double *)xmalloc(sizeof(double) * (T + 1));
+    double *be = (double *)xmalloc(sizeof(double) * (T + 1));
+    double *ga = (double *)xmalloc(sizeof(double) * (T + 1));
+    double *hs = (double *)xmalloc(sizeof(double) * (T + 1) * NP);    /* h_{t-1}, t = 0..T */
+    double *Ut = (double *)xmalloc(sizeof(double) * NP);
+    double *Um = (double *)xmalloc(sizeof(double) * NP);
+    double *Gh = (double *)xmalloc(sizeof(double) * NP);
+    double *GU = (double *)xmalloc(sizeof(double) * NP);
+    double *GUf = (double *)xmalloc(sizeof(double) * NP);
+    double *Gphi = (double *)xmalloc(sizeof(double) * K);
+    double *dBb = (double *)xmalloc(sizeof(double) * RN);
+    double *dCb = (double *)xmalloc(sizeof(double) * RN);
+    double *dBp = (double *)xmalloc(sizeof(double) * N);
+    double *dCp = (double *)xmalloc(sizeof(double) * N);
+    double *dX = (double *)xmalloc(sizeof(double) * RP);
+    double *tmp = (double *)xmalloc(sizeof(double) * N);
 
     for (long b = 0; b < Bt; b++)
         for (long h = 0; h < H; h++) {
