@@ -5,10 +5,13 @@
 The ptxas report (registers, spills, shared memory per kernel) is written to
 ``_build/ptxas.log``.
 """
+import concurrent.futures
 import glob
 import os
+import shutil
 import subprocess
 import sys
+import tempfile
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -42,25 +45,37 @@ def build(force=False, verbose=False):
         return LIB
     os.makedirs(BUILD, exist_ok=True)
     nvcc = os.environ.get("NVCC", "nvcc")
-    objs = []
-    log = []
-    for src in sources():
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+    srcs = sources()
+    # objects in a directory of this process's own, so that builds started
+    # side by side (test workers) never link each other's half-written files
+    objdir = tempfile.mkdtemp(prefix="obj.", dir=BUILD)
+    objs = [os.path.join(objdir, os.path.basename(src)[:-3] + ".o") for src in srcs]
+
+    def compile_one(src, obj):
         cmd = [nvcc] + NVCC_FLAGS + ["-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
+        return cmd, subprocess.run(cmd, capture_output=True, text=True)
+
+    try:
+        # one nvcc per source file, side by side
+        workers = max(1, min(len(srcs), os.cpu_count() or 1))
+        with concurrent.futures.ThreadPoolExecutor(max_workers=workers) as pool:
+            results = list(pool.map(compile_one, srcs, objs))
+        log = []
+        for src, (cmd, r) in zip(srcs, results):
+            log.append("$ " + " ".join(cmd) + "\n" + r.stdout + r.stderr)
+            if r.returncode != 0:
+                sys.stderr.write(r.stdout + r.stderr)
+                raise RuntimeError("nvcc failed on " + src)
+        tmp = LIB + ".tmp%d" % os.getpid()
+        cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp] + objs
         r = subprocess.run(cmd, capture_output=True, text=True)
         log.append("$ " + " ".join(cmd) + "\n" + r.stdout + r.stderr)
         if r.returncode != 0:
             sys.stderr.write(r.stdout + r.stderr)
-            raise RuntimeError("nvcc failed on " + src)
-        objs.append(obj)
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp] + objs
-    r = subprocess.run(cmd, capture_output=True, text=True)
-    log.append("$ " + " ".join(cmd) + "\n" + r.stdout + r.stderr)
-    if r.returncode != 0:
-        sys.stderr.write(r.stdout + r.stderr)
-        raise RuntimeError("nvcc link failed")
-    os.replace(tmp, LIB)
+            raise RuntimeError("nvcc link failed")
+        os.replace(tmp, LIB)
+    finally:
+        shutil.rmtree(objdir, ignore_errors=True)
     with open(os.path.join(BUILD, "ptxas.log"), "w") as f:
         f.write("\n".join(log))
     if verbose:
