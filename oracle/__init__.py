@@ -9,4 +9,4 @@ from .oracle import (  # noqa: F401
     step_decode, mimo_step_decode, step_decode_factored, loop_bwd, GRAD_NAMES, oracle_lib_path,
     oracle_source_path, compile_source, use_library,
 )
-from .chunked_bwd import siso_chunked_bwd  # noqa: F401
+from .chunked_bwd import chunked_bwd  # noqa: F401

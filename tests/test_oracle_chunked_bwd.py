@@ -2,13 +2,13 @@
 (oracle/chunked_bwd.py) equals the loop's reverse sweep, which finite
 differences pin, for every gradient, every chunk length (including 1 and
 chunks longer than the sequence), ragged tails, grouped B/C, partial RoPE,
-initial states and final-state adjoints.  Both are fp64, so they agree to
+rank R with W_x and W_y, initial states and final-state adjoints.  Both are fp64, so they agree to
 rounding (1e-11 relative)."""
 import numpy as np
 import pytest
 
 import oracle
-from oracle.chunked_bwd import siso_chunked_bwd
+from oracle.chunked_bwd import chunked_bwd
 
 KEYS = ("dx", "ddt", "dA", "dlam", "dtheta", "dB", "dC", "dD", "dh0", "dprevBx0", "dangle0")
 
@@ -45,7 +45,7 @@ def _build():
 def test_chunked_backward_equals_the_loop(T, Q, states):
     inp, dy, st, adj = _case(11 + T + Q, 2, T, 2, 2, 5, 6, 3, states)
     ref = oracle.loop_bwd(**inp, dy=dy, **st, **adj)
-    got = siso_chunked_bwd(**inp, dy=dy, chunk=Q, **st, **adj)
+    got = chunked_bwd(**inp, dy=dy, chunk=Q, **st, **adj)
     if T == 1 and not states:
         # one token from zero states: y_0 holds Cbar_0 . Bbar_0, which no
         # rotation changes, so every angle gradient is zero on both sides
@@ -69,7 +69,7 @@ def test_chunked_backward_equals_the_loop(T, Q, states):
 def test_chunked_backward_groups_and_partial_rope(H, G, K):
     inp, dy, st, adj = _case(5 * H + G + K, 1, 45, H, G, 4, 8, K, True)
     ref = oracle.loop_bwd(**inp, dy=dy, **st, **adj)
-    got = siso_chunked_bwd(**inp, dy=dy, chunk=8, **st, **adj)
+    got = chunked_bwd(**inp, dy=dy, chunk=8, **st, **adj)
     errs = {k: _rel(got[k], ref[k]) for k in KEYS}
     assert max(errs.values()) <= 1e-11, errs
 
@@ -79,6 +79,24 @@ def test_chunked_backward_strong_decay():
     chunked walk still agrees with the loop."""
     inp, dy, st, adj = _case(3, 1, 90, 2, 2, 4, 6, 3, True, shift=5.0)
     ref = oracle.loop_bwd(**inp, dy=dy, **st, **adj)
-    got = siso_chunked_bwd(**inp, dy=dy, chunk=32, **st, **adj)
+    got = chunked_bwd(**inp, dy=dy, chunk=32, **st, **adj)
     errs = {k: _rel(got[k], ref[k]) for k in KEYS}
+    assert max(errs.values()) <= 1e-11, errs
+
+
+@pytest.mark.parametrize("R,G,K,T,Q,states", [(2, 2, 3, 37, 8, True), (3, 1, 2, 20, 4, True), (4, 2, 4, 33, 16, False),
+                                              (2, 2, 1, 9, 1, True)])
+def test_chunked_backward_rank_r(R, G, K, T, Q, states):
+    """Rank R: the walk over (token, rank) rows with W_x, W_y equals the loop,
+    including the W_x and W_y gradients."""
+    H, P, N = 2, 4, 8
+    inp, dy, st, adj = _case(100 * R + T, 1, T, H, G, P, N, K, states)
+    rng = np.random.default_rng(R + T)
+    inp["B"] = rng.standard_normal((1, T, G, R, N)) / np.sqrt(N)
+    inp["C"] = rng.standard_normal((1, T, G, R, N)) / np.sqrt(N)
+    W = dict(Wx=1 + 0.3 * rng.standard_normal((H, R, P)), Wy=1 + 0.3 * rng.standard_normal((H, R, P)))
+    ref = oracle.loop_bwd(**inp, dy=dy, **W, **st, **adj)
+    got = chunked_bwd(**inp, dy=dy, chunk=Q, **W, **st, **adj)
+    keys = KEYS + ("dWx", "dWy")
+    errs = {k: _rel(got[k], ref[k]) for k in keys if states or k != "dangle0"}
     assert max(errs.values()) <= 1e-11, errs
