@@ -311,6 +311,14 @@ m3_status m3_device_error(void *stream, int *site);
 #define M3_SELFTEST_SITE 99
 m3_status m3_selftest_bounded_wait(void *stream);
 
+/* Host-side failure injection, for testing callers' error paths.  After
+ * this call the next n entry-point calls that pass their argument checks
+ * return M3_ERR_CUDA, as a failed launch would, and enqueue nothing (their
+ * outputs are left as they were).  n <= 0 turns it off.  Calls that fail
+ * their checks still return their own status and do not count.  Nothing on
+ * the device is touched, so it is safe with or without a GPU. */
+void m3_debug_fail_next_launches(int n);
+
 /* Number of kernels the library has enqueued since it was loaded (host-side
  * counter, incremented once per launch; used to count launches in a timed
  * region). */

@@ -95,6 +95,24 @@ m3_status read_norm(const m3_bcnorm *n, NormArgs &o) {
 
 inline m3_status launched(cudaError_t e) { return e == cudaSuccess ? M3_OK : M3_ERR_CUDA; }
 
+// Failure-injection hook (m3_debug_fail_next_launches): the next n calls that
+// pass validation report a launch failure without launching anything.
+std::atomic<int> g_fail_launches{0};
+inline bool injected_failure() {
+    int n = g_fail_launches.load(std::memory_order_relaxed);
+    while (n > 0)
+        if (g_fail_launches.compare_exchange_weak(n, n - 1, std::memory_order_relaxed)) return true;
+    return false;
+}
+
+// Every entry point ends here, after its validation: the launch, or the
+// injected failure in its place.
+template <typename F>
+inline m3_status launch_unless_injected(F &&launch) {
+    if (injected_failure()) return M3_ERR_CUDA;
+    return launched(launch());
+}
+
 m3_status chunked_common(const void *x, const float *dt, const float *A, const float *lam,
                          const float *theta, const void *B, const void *C, const float *D,
                          const float *Wx, const float *Wy, m3_dtype dtype, const m3_bcnorm *norm,
@@ -140,9 +158,10 @@ m3_status chunked_common(const void *x, const float *dt, const float *A, const f
     a.mimo_layout = mimo ? 1 : 0;
     a.ws = workspace;
     a.Q = chunk_request(d.chunk);
-    if (scan_tc_supported(a, dtype)) return launched(launch_scan_tc(a, (cudaStream_t)stream));
+    if (scan_tc_supported(a, dtype))
+        return launch_unless_injected([&] { return launch_scan_tc(a, (cudaStream_t)stream); });
     a.Q = q;
-    return launched(launch_scan_simt(a, dtype, (cudaStream_t)stream));
+    return launch_unless_injected([&] { return launch_scan_simt(a, dtype, (cudaStream_t)stream); });
 }
 
 }  // namespace
@@ -173,8 +192,11 @@ m3_status m3_device_error(void *stream, int *site) {
     return e ? M3_ERR_TIMEOUT : M3_OK;
 }
 
+void m3_debug_fail_next_launches(int n) { g_fail_launches.store(n > 0 ? n : 0, std::memory_order_relaxed); }
+
 m3_status m3_selftest_bounded_wait(void *stream) {
-    return launched(launch_wait_selftest(M3_SELFTEST_SITE, (cudaStream_t)stream));
+    return launch_unless_injected(
+        [&] { return launch_wait_selftest(M3_SELFTEST_SITE, (cudaStream_t)stream); });
 }
 
 size_t m3_workspace_bytes(int which, m3_dims d, m3_dtype dtype) {
@@ -204,8 +226,9 @@ m3_status m3_discretize(const float *dt, const float *A, const float *lam, m3_di
     M3_REQ(A);
     if (d.batch * d.seqlen == 0) return M3_OK;
     M3_REQ(dt); M3_REQ(lam); M3_REQ(alpha); M3_REQ(beta); M3_REQ(gamma);
-    return launched(launch_discretize(dt, A, lam, d.batch, d.seqlen, d.nheads, alpha, beta, gamma,
-                                      (cudaStream_t)stream));
+    return launch_unless_injected([&] {
+        return launch_discretize(dt, A, lam, d.batch, d.seqlen, d.nheads, alpha, beta, gamma, (cudaStream_t)stream);
+    });
 }
 
 m3_status m3_rope_bc(const void *B, const void *C, m3_dtype dtype, const float *theta, const float *dt,
@@ -230,7 +253,7 @@ m3_status m3_rope_bc(const void *B, const void *C, m3_dtype dtype, const float *
     a.B = B; a.C = C; a.theta = theta; a.dt = dt; a.angle0 = angle0; a.nrm = nrm;
     a.Bo = B_rot; a.Co = C_rot; a.angle_out = angle_final;
     a.Bt = d.batch; a.T = d.seqlen; a.H = d.nheads; a.R = R; a.N = d.dstate; a.G = G; a.K = K;
-    return launched(launch_rope(a, dtype, (cudaStream_t)stream));
+    return launch_unless_injected([&] { return launch_rope(a, dtype, (cudaStream_t)stream); });
 }
 
 m3_status m3_siso_chunked_fwd(const void *x, const float *dt, const float *A, const float *lam,
@@ -275,7 +298,7 @@ m3_status m3_step_decode(const void *x_t, const float *dt_t, const float *A, con
     a.x = x_t; a.B = B_t; a.C = C_t; a.dt = dt_t; a.A = A; a.lam = lam_t; a.theta = theta_t; a.D = D;
     a.nrm = nrm; a.h = h; a.prevBx = prevBx; a.angle = angle; a.y = y_t;
     a.Bt = d.batch; a.H = d.nheads; a.P = d.headdim; a.N = d.dstate; a.G = G; a.K = K;
-    return launched(launch_decode(a, dtype, (cudaStream_t)stream));
+    return launch_unless_injected([&] { return launch_decode(a, dtype, (cudaStream_t)stream); });
 }
 
 namespace {
@@ -307,7 +330,7 @@ m3_status decode_gen(const void *x_t, const float *dt_t, const float *A, const f
     a.nrm = nrm; a.h = h; a.prevBx = prevBx; a.angle = angle; a.y = y_t;
     a.Bt = d.batch; a.H = d.nheads; a.P = d.headdim; a.N = d.dstate; a.G = G; a.K = K;
     a.Wx = W_x; a.Wy = W_y; a.bprev = b_prev; a.xprev = x_prev; a.R = d.rank;
-    return launched(launch_decode_gen(a, dtype, factored, (cudaStream_t)stream));
+    return launch_unless_injected([&] { return launch_decode_gen(a, dtype, factored, (cudaStream_t)stream); });
 }
 }  // namespace
 
@@ -375,7 +398,7 @@ m3_status m3_chunked_bwd(const void *x, const float *dt, const float *A, const f
     a.Q = q;
     a.ws = static_cast<float *>(workspace);
     if (d.batch == 0) return M3_OK;
-    return launched(launch_scan_bwd(a, dtype, (cudaStream_t)stream));
+    return launch_unless_injected([&] { return launch_scan_bwd(a, dtype, (cudaStream_t)stream); });
 }
 
 }  // extern "C"

@@ -23,7 +23,7 @@ ABI_FUNCTIONS = (
     "m3_get_limits", "m3_discretize", "m3_rope_bc", "m3_siso_chunked_fwd",
     "m3_mimo_chunked_fwd", "m3_step_decode", "m3_workspace_bytes", "m3_status_string",
     "m3_launch_count", "m3_device_error", "m3_siso_chunked_fwd_noalloc", "m3_mimo_step_decode",
-    "m3_step_decode_factored", "m3_chunked_bwd", "m3_selftest_bounded_wait",
+    "m3_step_decode_factored", "m3_chunked_bwd", "m3_selftest_bounded_wait", "m3_debug_fail_next_launches",
 )
 M3_SELFTEST_SITE = 99
 
@@ -111,6 +111,8 @@ def lib():
                                           ctypes.POINTER(BcNorm), Dims, _VP, _VP, _VP, _VP, _VP, _VP]
     L.m3_selftest_bounded_wait.restype = ctypes.c_int
     L.m3_selftest_bounded_wait.argtypes = [_VP]
+    L.m3_debug_fail_next_launches.restype = None
+    L.m3_debug_fail_next_launches.argtypes = [ctypes.c_int]
     L.m3_chunked_bwd.restype = ctypes.c_int
     L.m3_chunked_bwd.argtypes = [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int,
                                  ctypes.POINTER(BcNorm), _VP, _VP, _VP, Dims, _VP, _VP, _VP, _VP,
@@ -140,6 +142,13 @@ def selftest_bounded_wait(stream=None):
     """Enqueue the timeout-path self-test (one bounded wait that runs out after
     about a second); read the outcome with device_error()."""
     _check(lib().m3_selftest_bounded_wait(_stream(stream)), "m3_selftest_bounded_wait")
+
+
+def debug_fail_next_launches(n):
+    """Failure injection for tests: the next n library calls that pass their
+    argument checks fail with M3_ERR_CUDA (raised as M3Error here) and
+    launch nothing.  n <= 0 turns it off."""
+    lib().m3_debug_fail_next_launches(int(n))
 
 
 def limits():

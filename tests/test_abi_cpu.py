@@ -257,3 +257,37 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     with pytest.raises(RuntimeError):
         mod.limits()
     importlib.reload(m3)
+
+
+def test_injected_launch_failure(L):
+    """m3_debug_fail_next_launches: calls that pass their checks report
+    M3_ERR_CUDA and launch nothing; calls that fail their checks keep their
+    own status and do not use up the count."""
+    L = m3.lib()        # this module's current binding (another test reloads it)
+    n0 = m3.launch_count()
+    g = m3.Grads(*([None] * len(m3.GRAD_FIELDS)))
+    d = dims()
+    need = m3.workspace_bytes(m3.M3_WS_BWD_SISO, d, m3.M3_BF16)
+    valid = [
+        lambda: siso(L, d),
+        lambda: L.m3_mimo_chunked_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, m3.M3_BF16, None,
+                                      None, None, None, dims(rank=2), FAKE, None, None, None, None, 0, None),
+        lambda: L.m3_rope_bc(FAKE, FAKE, m3.M3_BF16, FAKE, FAKE, None, None, d, FAKE, FAKE, None, None),
+        lambda: L.m3_discretize(FAKE, FAKE, FAKE, d, FAKE, FAKE, FAKE, None),
+        lambda: L.m3_step_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, m3.M3_BF16, None, d, FAKE, FAKE,
+                                 FAKE, FAKE, None),
+        lambda: L.m3_step_decode_factored(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, m3.M3_BF16,
+                                          None, dims(rank=2), FAKE, FAKE, FAKE, FAKE, FAKE, None),
+        lambda: L.m3_chunked_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, m3.M3_BF16, None, None,
+                                 None, None, d, FAKE, None, None, None, ctypes.byref(g), FAKE, need, None),
+    ]
+    try:
+        m3.debug_fail_next_launches(len(valid))
+        assert siso(L, dims(dstate=5)) == m3.M3_ERR_INVALID_ARG      # a failed check does not count
+        for call in valid:
+            assert call() == m3.M3_ERR_CUDA
+        # the count is used up; another failed check still reports itself
+        assert siso(L, dims(headdim=512)) == m3.M3_ERR_UNSUPPORTED
+        assert m3.launch_count() == n0                                # nothing was enqueued
+    finally:
+        m3.debug_fail_next_launches(0)
