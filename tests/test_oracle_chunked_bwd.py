@@ -3,7 +3,8 @@
 differences pin, for every gradient, every chunk length (including 1 and
 chunks longer than the sequence), ragged tails, grouped B/C, partial RoPE,
 rank R with W_x and W_y, initial states and final-state adjoints.  Both are fp64, so they agree to
-rounding (1e-11 relative)."""
+rounding (1e-11 relative).  Nine plausible mistakes planted in a copy of the
+chunked walk each break that agreement, so the pin constrains every term."""
 import numpy as np
 import pytest
 
@@ -100,3 +101,43 @@ def test_chunked_backward_rank_r(R, G, K, T, Q, states):
     keys = KEYS + ("dWx", "dWy")
     errs = {k: _rel(got[k], ref[k]) for k in keys if states or k != "dangle0"}
     assert max(errs.values()) <= 1e-11, errs
+
+
+CHUNKED_MUTATIONS = [
+    ("inter-chunk decay of the adjoint state dropped", "dgin = dgin + np.exp(ce) * Gout", "dgin = dgin + Gout"),
+    ("mask diagonal takes w instead of gamma", "M = E * wc[None, :] + np.diag(gc)",
+     "M = E * wc[None, :] + np.diag(wc)"),
+    ("chunk-state weight without the decay", "sc = rows(es * wc)", "sc = rows(wc)"),
+    ("decay adjoint of the chunk-state weights dropped", "        dcum -= des\n", "\n"),
+    ("rotation adjoint sign", "dphi += cross.reshape(T, R, K).sum(axis=1)", "dphi -= cross.reshape(T, R, K).sum(axis=1)"),
+    ("angle adjoint summed forwards", "rc = np.cumsum(dphi[::-1], axis=0)[::-1]", "rc = np.cumsum(dphi, axis=0)"),
+    ("boundary fold adjoint dropped", "    ddt[0] += (1.0 - lam[0]) * dsg_m1\n", "\n"),
+    ("prevBx_final adjoint from the wrong token", "last = slice((T - 1) * R, T * R)", "last = slice(0, R)"),
+    ("W_y gradient without the inter-chunk term", "Y = rows(ec)[:, None] * (Cc @ gi) + (Mr * S) @ Xc",
+     "Y = (Mr * S) @ Xc"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", CHUNKED_MUTATIONS, ids=[m[0] for m in CHUNKED_MUTATIONS])
+def test_planted_mistakes_in_the_chunked_backward_fail_the_pin(name, old, new):
+    """Each plausible mistake planted in a copy of the chunked walk makes it
+    disagree with the loop on one of the pin's cases."""
+    import os
+    import types
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "chunked_bwd.py")).read()
+    assert src.count(old) == 1, name
+    mod = types.ModuleType("mutated_chunked_bwd")
+    exec(compile(src.replace(old, new), "mutated_chunked_bwd", "exec"), mod.__dict__)
+    worst = 0.0
+    for R in (1, 2):
+        inp, dy, st, adj = _case(7 + R, 1, 23, 2, 2, 4, 6, 2, True)
+        kw = {}
+        if R > 1:
+            rng = np.random.default_rng(R)
+            inp["B"] = rng.standard_normal((1, 23, 2, R, 6)) / np.sqrt(6)
+            inp["C"] = rng.standard_normal((1, 23, 2, R, 6)) / np.sqrt(6)
+            kw = dict(Wx=1 + 0.3 * rng.standard_normal((2, R, 4)), Wy=1 + 0.3 * rng.standard_normal((2, R, 4)))
+        ref = oracle.loop_bwd(**inp, dy=dy, **kw, **st, **adj)
+        got = mod.chunked_bwd(**inp, dy=dy, chunk=5, **kw, **st, **adj)
+        worst = max([worst] + [_rel(got[k], ref[k]) for k in got])
+    assert worst > 1e-6, name
