@@ -50,6 +50,39 @@ def dist_env():
     return world, rank, local
 
 
+def launch_plan(gpus, env):
+    """How a run asked for ``--gpus N`` proceeds, given the environment.
+
+    Returns ("run", world) to run here as one rank of ``world``,
+    ("relaunch", N) when N > 1 was asked without torchrun (the script starts
+    itself again under torchrun with N ranks), or ("error", message) when
+    torchrun's WORLD_SIZE disagrees with --gpus."""
+    if gpus < 1:
+        return "error", "--gpus must be >= 1 (got %d)" % gpus
+    if "WORLD_SIZE" not in env:
+        return ("relaunch", gpus) if gpus > 1 else ("run", 1)
+    world = int(env["WORLD_SIZE"])
+    if world != gpus:
+        return "error", "--gpus %d but WORLD_SIZE=%d: launch %d ranks, or pass --gpus %d" % (
+            gpus, world, gpus, world)
+    return "run", world
+
+
+def torchrun_command(gpus, argv, port):
+    """The torchrun command line that runs this script as ``gpus`` ranks."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", str(gpus),
+            "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + list(argv)
+
+
+def _free_port():
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
 def init_dist(world, backend):
     if world <= 1:
         return None
@@ -378,6 +411,79 @@ class BwdWorkload(ScanWorkload):
         return n, time.perf_counter() - t0, 1
 
 
+def prep_bytes(c):
+    """Algorithmic bytes of one standalone prep pass over a whole workload.
+    Discretize: dt, lam in (8 B) and alpha, beta, gamma out (12 B) per
+    token-head, A once.  Rope: B, C in and the rotated B, C out (one row per
+    head), theta and dt in, per token-head; the final angle out per lane."""
+    Bt, T, H, N, R = c["batch"], c["seqlen"], c["nheads"], c["dstate"], c["rank"]
+    G, K = c.get("ngroups", 0) or H, c.get("rope_pairs", 0) or N // 2
+    es = 2 if c["dtype"] == "bf16" else 4
+    if c["prep"] == "discretize":
+        return Bt * T * H * 20 + H * 4
+    per_token_head = 2 * es * R * N + 4 * K + 4
+    per_token_group = 2 * es * R * N
+    return Bt * T * (H * per_token_head + G * per_token_group) + Bt * H * K * 4
+
+
+class PrepWorkload(ScanWorkload):
+    """One standalone S1 (m3_discretize) or S2 (m3_rope_bc) call over the
+    default workload's inputs, outputs preallocated."""
+
+    def __init__(self, idx, device):
+        super().__init__(idx, device)
+        c = self.c
+        Bt, T, H, N = c["batch"], c["seqlen"], c["nheads"], c["dstate"]
+        self.kind = c["prep"]
+        d = self.dev
+        if self.kind == "discretize":
+            self.out = tuple(torch.empty_like(d["dt"]) for _ in range(3))
+            self.kernel = "k_discretize"
+        else:
+            self.out = (torch.empty(Bt, T, H, N, device=device, dtype=d["B"].dtype),
+                        torch.empty(Bt, T, H, N, device=device, dtype=d["B"].dtype),
+                        torch.empty(Bt, H, self.K, device=device))
+            self.kernel = "k_rope"
+        self.kernel_label = self.kernel
+        self.srcs = [os.path.join(ROOT, "state_space_lm_b200", "csrc", "k_elementwise.cu")]
+        self.bytes = prep_bytes(c)
+        self.flops = 0
+        keys = ("dt", "A", "lam") if self.kind == "discretize" else ("B", "C", "theta", "dt")
+        self.host = {k: self.host[k] for k in keys}
+        self.input_bytes = sum(self.host[k].numel() * self.host[k].element_size() for k in keys)
+
+    def step(self, dev=None, out=None, stream=None):
+        d = self.dev if dev is None else dev
+        o = self.out if out is None else out
+        if self.kind == "discretize":
+            self.m3.discretize(d["dt"], d["A"], d["lam"], out=o, stream=stream)
+        else:
+            self.m3.rope_bc(d["B"], d["C"], d["theta"], d["dt"], out=o, stream=stream)
+
+    def config(self):
+        cfg = super().config()
+        cfg.pop("chunk", None)
+        cfg["pass"] = ("S1 alone: alpha, beta, gamma of every token-head" if self.kind == "discretize" else
+                       "S2 alone: rotated B, C (one row per head) and the final angle")
+        cfg["inputs"] = ("dt/lam/A fp32, seeded synthetic" if self.kind == "discretize" else
+                         "B/C %s, theta/dt fp32, seeded synthetic" % self.c["dtype"])
+        return cfg
+
+    def oracle_sample(self, n_lanes, threads):
+        """The oracle's S1 or S2 on the first batch rows holding n lanes."""
+        import oracle
+        c = self.c
+        H = c["nheads"]
+        nb = max(1, min(c["batch"], n_lanes // H))
+        a = {k: gen.to_f64(v[:nb] if k != "A" else v) for k, v in self.host.items()}
+        t0 = time.perf_counter()
+        if self.kind == "discretize":
+            oracle.discretize(a["dt"], a["A"], a["lam"])
+        else:
+            oracle.rope_bc(a["B"], a["C"], a["theta"], a["dt"])
+        return nb * H, time.perf_counter() - t0, 1
+
+
 class DecodeWorkload:
     """Decode steps: every step advances all (batch, head) lanes by one token.
     The carried state comes from a seeded prefill (a chunked forward over the
@@ -482,12 +588,13 @@ def run_cpu_baseline(w, target_s=10.0, wall_s=1.5):
             dt += d1
         used = used2
     tokens = reps * nl * w.c["seqlen"] / H
-    # one thread on one lane, scaled to whole tokens of all heads
-    _, d1, _ = w.oracle_sample(1, 1)
+    # one thread on one lane (a prep pass: one batch row), scaled to whole
+    # tokens of all heads
+    nl1, d1, _ = w.oracle_sample(1, 1)
     return {"value": tokens / dt, "unit": UNIT, "cores": int(used), "kind": "oracle",
             "sample": "%d x %d of %d (b,h) lanes x %d tokens, fp64 C loop, %.1f s wall on %d threads"
                       % (reps, nl, total_lanes, w.c["seqlen"], dt, used),
-            "one_thread_value": w.c["seqlen"] / H / d1, "cpu_model": cpu_model()}
+            "one_thread_value": nl1 * w.c["seqlen"] / H / d1, "cpu_model": cpu_model()}
 
 
 def decode_oracle_sample(c, nb, steps, threads):
@@ -563,6 +670,8 @@ def run_ours(args, world, rank, local):
         w = DecodeWorkload(args.config, device, args.steps + args.warmup)
     elif gen.CONFIGS[args.config].get("grad"):
         w = BwdWorkload(args.config, device)
+    elif gen.CONFIGS[args.config].get("prep"):
+        w = PrepWorkload(args.config, device)
     else:
         w = ScanWorkload(args.config, device)
     stream = torch.cuda.current_stream(device)
@@ -692,11 +801,15 @@ def run_reference(args, world, rank):
         run_reference_decode(args, world)
         return
     bwd = bool(gen.CONFIGS[args.config].get("grad"))
-    w = (BwdWorkload if bwd else ScanWorkload).__new__(BwdWorkload if bwd else ScanWorkload)
+    prep = gen.CONFIGS[args.config].get("prep")
+    cls = BwdWorkload if bwd else (PrepWorkload if prep else ScanWorkload)
+    w = cls.__new__(cls)
     w.c = dict(gen.CONFIGS[args.config])
     w.idx = args.config
     w.host = gen.config_inputs(args.config)
     w.host.pop("generator")
+    if prep:
+        w.kind = prep
     if bwd:
         w.host["dy"] = gen.grad_seed(w.host["x"], gen.SEED_BASE + 1000 + args.config)
     w.mimo = w.c["rank"] > 1
@@ -766,6 +879,12 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    plan, what = launch_plan(args.gpus, os.environ)
+    if plan == "error":
+        raise SystemExit("bench.py: " + what)
+    if plan == "relaunch":
+        import subprocess
+        raise SystemExit(subprocess.call(torchrun_command(what, sys.argv[1:], _free_port())))
     world, rank, local = dist_env()
     if args.impl == "reference":
         run_reference(args, world, rank)

@@ -51,6 +51,12 @@ CONFIGS = {
     # the backward (all input gradients) of the default workload
     8: dict(name="bwd_siso_8x2048_h16_p64_n128", batch=8, seqlen=2048, nheads=16, headdim=64,
             dstate=128, rank=1, chunk=64, dtype="bf16", dt_shift=-2.0, grad=True),
+    # the standalone prep passes on the default workload's inputs: S1 alone
+    # (alpha, beta, gamma out) and S2 alone (rotated B, C and the angle out)
+    9: dict(name="discretize_8x2048_h16", batch=8, seqlen=2048, nheads=16, headdim=64,
+            dstate=128, rank=1, chunk=64, dtype="bf16", dt_shift=-2.0, prep="discretize"),
+    10: dict(name="rope_bc_8x2048_h16_n128", batch=8, seqlen=2048, nheads=16, headdim=64,
+             dstate=128, rank=1, chunk=64, dtype="bf16", dt_shift=-2.0, prep="rope"),
 }
 
 _DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}

@@ -52,3 +52,11 @@ def test_backward_bytes_and_flops():
     assert bench.bwd_flops(c) == 128 * 32 * per_chunk
     assert bench.bwd_flops(c) / (8 * 2048 * 16) == pytest.approx(131.6e3, rel=1e-3)
     assert bench.FFMA_PEAK_TFLOPS == pytest.approx(74.4, rel=1e-3)
+
+
+def test_prep_bytes():
+    # S1: dt, lam in, alpha, beta, gamma out (20 B per token-head) + A
+    assert bench.prep_bytes(gen.CONFIGS[9]) == 8 * 2048 * 16 * 20 + 16 * 4
+    # S2: B, C in (512), theta (256), dt (4), rotated B, C out (512) = 1284 B
+    # per token-head, + the final angle per lane
+    assert bench.prep_bytes(gen.CONFIGS[10]) == 8 * 2048 * 16 * 1284 + 128 * 64 * 4
