@@ -264,11 +264,16 @@ m3_status m3_chunked_bwd(const void *x, const float *dt, const float *A, const f
  * workspace from.  This entry point takes the arguments of
  * m3_siso_chunked_fwd without the workspace, and uses instead a scratch
  * buffer of M3_NOALLOC_SCRATCH_BYTES that is part of the library: a static
- * device array, held on every GPU that loads the library until the process
- * exits.  It allocates nothing and calls no allocating routine.
- *  - Set-up: the first call on each device looks up the buffer's device
- *    address (cudaGetSymbolAddress, with that device current).  Make that
- *    first call before any stream capture.
+ * device array.  It allocates nothing and calls no allocating routine.
+ *  - Set-up: each call looks up the buffer's device address on the current
+ *    device (cudaGetSymbolAddress).  CUDA loads modules lazily, so the first
+ *    call on a device loads the library's module there and commits the
+ *    buffer's M3_NOALLOC_SCRATCH_BYTES of device memory, which stay held
+ *    until the process exits.  That first call can therefore fail with
+ *    M3_ERR_CUDA when the device has no memory left (for example under a
+ *    framework that has already reserved it all): make it during warm-up,
+ *    and before any stream capture.  Later calls only repeat the lookup,
+ *    which allocates nothing and stays valid after a device reset.
  *  - Limit: sizes whose scratch need, m3_workspace_bytes(M3_WS_SISO, d,
  *    dtype), exceeds M3_NOALLOC_SCRATCH_BYTES are rejected with
  *    M3_ERR_WORKSPACE before anything is enqueued.

@@ -352,8 +352,14 @@ static cudaError_t launch_decode_gen_rt(const DecodeArgs &a, bool factored, cuda
     const int threads = 256;
     const int ngroups = threads / (int)(a.P / 4);
     const size_t smem = sizeof(float) * (3 * RT * a.N + 32 + a.N / 2 + (size_t)ngroups * RT * a.P);
-    if (factored) k_decode_gen<T, RT, true><<<(unsigned)(a.Bt * a.H), threads, smem, s>>>(a);
-    else k_decode_gen<T, RT, false><<<(unsigned)(a.Bt * a.H), threads, smem, s>>>(a);
+    // rank 8 at dstate 256 needs about 57 KB, past the 48 KB a launch gets by default
+    if (factored) {
+        cudaFuncSetAttribute(k_decode_gen<T, RT, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        k_decode_gen<T, RT, true><<<(unsigned)(a.Bt * a.H), threads, smem, s>>>(a);
+    } else {
+        cudaFuncSetAttribute(k_decode_gen<T, RT, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        k_decode_gen<T, RT, false><<<(unsigned)(a.Bt * a.H), threads, smem, s>>>(a);
+    }
     count_launch();
     return cudaGetLastError();
 }

@@ -7,38 +7,25 @@
 // hosts that must not allocate between a warm-up and a latency-critical
 // phase.  This entry point gives them the same computation with its scratch
 // in a fixed buffer that is part of the library image: a file-scope
-// __device__ array of M3_NOALLOC_SCRATCH_BYTES, which every GPU that loads
-// the library holds until the process exits.
-#include <mutex>
-
+// __device__ array of M3_NOALLOC_SCRATCH_BYTES.  CUDA loads modules lazily,
+// so a device commits the buffer at the first call there (the first symbol
+// lookup loads this file's module) and keeps it until the process exits.
 #include "m3_internal.cuh"
 
 namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[M3_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void *g_scratch_ptr[kMaxDevices];   // device address of the buffer, per device ordinal
-bool g_scratch_ready[kMaxDevices];
-
 // Device address of the buffer on the current device.  In host code the
 // array's name is only a host-side stand-in, so the address comes from
-// cudaGetSymbolAddress, once per device, with that device current.
+// cudaGetSymbolAddress with that device current.  The lookup runs on every
+// call (it allocates nothing once the module is loaded), so the address stays
+// right after the caller resets the device and its context is recreated.
 cudaError_t scratch_on_current_device(void **out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ready[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = p;
-        g_scratch_ready[dev] = true;
-    }
-    *out = g_scratch_ptr[dev];
+    *out = p;
     return cudaSuccess;
 }
 
