@@ -666,6 +666,15 @@ __global__ void __launch_bounds__(THREADS, 1)
                                                              : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         };
+        // QkNorm gain and BC-bias of pair q of one raw row (QkNorm / bias variant)
+        auto norm_bias = [&](int row, int r, int q, float2 &bv, float2 &cv) {
+            const int e0 = 8 * j4 + 2 * q;
+            const int64_t bo = (h * R + r) * N + e0;
+            if (nr.wB) { const float ib = inv[row]; bv.x *= ib * nr.wB[e0]; bv.y *= ib * nr.wB[e0 + 1]; }
+            if (nr.wC) { const float ic = inv[Q + row]; cv.x *= ic * nr.wC[e0]; cv.y *= ic * nr.wC[e0 + 1]; }
+            if (nr.biasB) { bv.x += nr.biasB[bo]; bv.y += nr.biasB[bo + 1]; }
+            if (nr.biasC) { cv.x += nr.biasC[bo]; cv.y += nr.biasC[bo + 1]; }
+        };
         load_theta(0);
         for (int c = 0; c < nchunks; c++) {
             const int sb = c % NB, kb = c / NB, scf = c % NC, kc = c / NC;
@@ -750,66 +759,44 @@ __global__ void __launch_bounds__(THREADS, 1)
             float phr[4];
 #pragma unroll
             for (int q = 0; q < 4; q++) phr[q] = reduce_2pi(phi[q]);
-            // pass 2: rotate my tokens (the same angles for every rank).  The
-            // token loop stays rolled (a small hot loop); the QkNorm / bias
-            // variant is a separate copy of it, so the plain one carries none
-            // of that code.
-            const bool last_chunk = last_seg && (c == nchunks - 1);
+            // pass 2: rotate my tokens (the same angles for every rank).  In the
+            // plain variant the body has no branches: rows past the sequence end
+            // were zero-filled by the TMA load (a chunk ends inside its segment
+            // only at the sequence end), so they rotate to zeros.  The QkNorm /
+            // bias variant is a separate copy that skips those rows (a bias or a
+            // zero-row norm would make them non-zero there).
+            const float phi_in[4] = {phi[0], phi[1], phi[2], phi[3]};   // angle entering my tokens
             auto rotate_tokens = [&](auto generic, auto fast_sc) {
                 constexpr bool G = decltype(generic)::value, F = decltype(fast_sc)::value;
 #pragma unroll
                 for (int u = 0; u < TPT; u++) {
                     const int i = i0 + u;
-                    float d[4] = {dph[0][0], dph[0][1], dph[0][2], dph[0][3]};
-#pragma unroll
-                    for (int k = 1; k < TPT; k++)
-                        if (u == k) {
-                            d[0] = dph[k][0]; d[1] = dph[k][1]; d[2] = dph[k][2]; d[3] = dph[k][3];
-                        }
                     float sn[4], cs[4];
 #pragma unroll
                     for (int q = 0; q < 4; q++) {
                         if (F) {
-                            phr[q] += d[q];
+                            phr[q] += dph[u][q];
                             __sincosf(phr[q], &sn[q], &cs[q]);
                         } else {
-                            phi[q] += d[q];
+                            phi[q] += dph[u][q];
                             sincos_rr(phi[q], &sn[q], &cs[q]);
                         }
                     }
-#pragma unroll 1
+#pragma unroll
                     for (int r = 0; r < R; r++) {
                         const int row = i * R + r;
                         uint4 ob = make_uint4(0u, 0u, 0u, 0u), oc = make_uint4(0u, 0u, 0u, 0u);
-                        if (i < Lc) {
+                        if (!G || i < Lc) {
                             const uint4 rb = braw[row * 16 + j4];
                             const uint4 rc = SO ? make_uint4(0u, 0u, 0u, 0u) : craw[row * 16 + j4];
                             const uint32_t rbw[4] = {rb.x, rb.y, rb.z, rb.w}, rcw[4] = {rc.x, rc.y, rc.z, rc.w};
                             uint32_t pbw[4], pcw[4];
-                            float ib = 1.f, ic = 1.f;
-                            if (G) {
-                                ib = nr.wB ? inv[row] : 1.f;
-                                ic = nr.wC ? inv[Q + row] : 1.f;
-                            }
 #pragma unroll
                             for (int q = 0; q < 4; q++) {
                                 float2 bv = unpack_bf16(rbw[q]), cv = unpack_bf16(rcw[q]);
-                                if (G) {
-                                    const int e0 = 8 * j4 + 2 * q;
-                                    const int64_t bo = (h * R + r) * N + e0;
-                                    if (nr.wB) { bv.x *= ib * nr.wB[e0]; bv.y *= ib * nr.wB[e0 + 1]; }
-                                    if (nr.wC) { cv.x *= ic * nr.wC[e0]; cv.y *= ic * nr.wC[e0 + 1]; }
-                                    if (nr.biasB) { bv.x += nr.biasB[bo]; bv.y += nr.biasB[bo + 1]; }
-                                    if (nr.biasC) { cv.x += nr.biasC[bo]; cv.y += nr.biasC[bo + 1]; }
-                                }
-                                const float rb0 = cs[q] * bv.x - sn[q] * bv.y, rb1 = sn[q] * bv.x + cs[q] * bv.y;
-                                pbw[q] = pack_bf16(rb0, rb1);
-                                if (!SO) pcw[q] = pack_bf16(cs[q] * cv.x - sn[q] * cv.y, sn[q] * cv.x + cs[q] * cv.y);
-                                else pcw[q] = 0u;
-                                if (last_chunk && i == Lc - 1) {
-                                    blast[r * N + 8 * j4 + 2 * q] = rb0;
-                                    blast[r * N + 8 * j4 + 2 * q + 1] = rb1;
-                                }
+                                if (G) norm_bias(row, r, q, bv, cv);
+                                pbw[q] = pack_bf16(cs[q] * bv.x - sn[q] * bv.y, sn[q] * bv.x + cs[q] * bv.y);
+                                pcw[q] = SO ? 0u : pack_bf16(cs[q] * cv.x - sn[q] * cv.y, sn[q] * cv.x + cs[q] * cv.y);
                             }
                             ob = make_uint4(pbw[0], pbw[1], pbw[2], pbw[3]);
                             oc = make_uint4(pcw[0], pcw[1], pcw[2], pcw[3]);
@@ -828,6 +815,34 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int q = 0; q < 4; q++) phi[q] += acc[q];   // the exact angle after my tokens
             } else {
                 rotate_tokens(BoolC<false>{}, BoolC<false>{});
+            }
+            if (last_seg && c == nchunks - 1) {
+                // the sequence's last token: its rotated B rows in fp32, for
+                // prev_Bx (once per lane, off the hot loop)
+                const int ul = Lc - 1 - i0;
+                if (ul >= 0 && ul < TPT) {
+                    float sn[4], cs[4];
+#pragma unroll
+                    for (int q = 0; q < 4; q++) {
+                        float ang = phi_in[q];
+#pragma unroll
+                        for (int u = 0; u < TPT; u++)
+                            if (u <= ul) ang += dph[u][q];
+                        sincos_rr(ang, &sn[q], &cs[q]);
+                    }
+                    for (int r = 0; r < R; r++) {
+                        const int row = (i0 + ul) * R + r;
+                        const uint4 rb = braw[row * 16 + j4];
+                        const uint32_t rbw[4] = {rb.x, rb.y, rb.z, rb.w};
+#pragma unroll
+                        for (int q = 0; q < 4; q++) {
+                            float2 bv = unpack_bf16(rbw[q]), cv = make_float2(0.f, 0.f);
+                            if (has_norm || has_bias) norm_bias(row, r, q, bv, cv);
+                            blast[r * N + 8 * j4 + 2 * q] = cs[q] * bv.x - sn[q] * bv.y;
+                            blast[r * N + 8 * j4 + 2 * q + 1] = sn[q] * bv.x + cs[q] * bv.y;
+                        }
+                    }
+                }
             }
             load_theta(c + 1);                     // in flight while the X operands are built
             fence_async_smem();
@@ -1026,6 +1041,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int ta = ra / R, tb = rb / R;          // their tokens
         const int cq = 2 * (l32 & 3);                // column offset inside a group of 8
         const int et = tid - W_EPI0 * 32;            // 0..255
+        // my rows 16q..16q+15 against my columns 32ch..32ch+31 (tokens row / R,
+        // col / R): wholly above the diagonal for ch = 1, q < 2; wholly below
+        // it for ch = 0, q >= 2; across it otherwise (R = 1, 2, 4 alike)
+        const bool blk_zero = ch == 1 && q < 2, blk_below = ch == 0 && q >= 2;
         const float Dh = a.D[h];
         uint8_t *sp = sm + L::OFF_SP;
         __nv_bfloat16 *yg = static_cast<__nv_bfloat16 *>(a.y);
@@ -1127,9 +1146,23 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (!(ok = group_wait(B_CFULL + scf, kc & 1, 20))) break;
                 const bool unsafe = cf[CF_SCAL + 1] != 0.f;
                 // ---- masked scores S' (rows ra, rb of D1; my 32 columns) ----
-                if (!(ok = group_wait(B_SFULL, c & 1, 21))) break;
-                tc_fence_after();
-                {
+                // My 16 x 32 block of the 64 x 64 tile lies wholly above the
+                // diagonal (zero: written at the first chunk, never again),
+                // wholly below it (every score takes r_t e_s w_s), or across it.
+                if (blk_zero) {
+                    if (c == 0) {
+#pragma unroll
+                        for (int hf = 0; hf < 2; hf++)
+#pragma unroll
+                            for (int i = 0; i < 2; i++) {
+                                const int col = cb0 + 16 * hf + 8 * i + cq, cc = col >> 3;
+                                *reinterpret_cast<uint32_t *>(sp + ra * 128 + ((cc ^ (ra & 7)) << 4) + 2 * cq) = 0u;
+                                *reinterpret_cast<uint32_t *>(sp + rb * 128 + ((cc ^ (rb & 7)) << 4) + 2 * cq) = 0u;
+                            }
+                    }
+                } else {
+                    if (!(ok = group_wait(B_SFULL, c & 1, 21))) break;
+                    tc_fence_after();
                     const float rta = cf[CF_R + ta], gta = cf[CF_GAM + ta];
                     const float rtb = cf[CF_R + tb], gtb = cf[CF_GAM + tb];
 #pragma unroll 1
@@ -1143,17 +1176,24 @@ __global__ void __launch_bounds__(THREADS, 1)
                             const int col = c0 + 8 * i + cq;
                             const int s0 = col / R, s1 = (col + 1) / R;   // tokens of the two columns
                             const float w0 = cf[CF_WM + s0], w1 = cf[CF_WM + s1];
-                            v[4 * i + 0] *= s0 < ta ? rta * w0 : (s0 == ta ? gta : 0.f);
-                            v[4 * i + 1] *= s1 < ta ? rta * w1 : (s1 == ta ? gta : 0.f);
-                            v[4 * i + 2] *= s0 < tb ? rtb * w0 : (s0 == tb ? gtb : 0.f);
-                            v[4 * i + 3] *= s1 < tb ? rtb * w1 : (s1 == tb ? gtb : 0.f);
-                            if (R == 1) {
-                                // SISO: the skip D x_t rides on the intra UMMA as D on the
-                                // diagonal of the scores (its B operand is x itself)
-                                v[4 * i + 0] += s0 == ta ? Dh : 0.f;
-                                v[4 * i + 1] += s1 == ta ? Dh : 0.f;
-                                v[4 * i + 2] += s0 == tb ? Dh : 0.f;
-                                v[4 * i + 3] += s1 == tb ? Dh : 0.f;
+                            if (blk_below) {
+                                v[4 * i + 0] *= rta * w0;
+                                v[4 * i + 1] *= rta * w1;
+                                v[4 * i + 2] *= rtb * w0;
+                                v[4 * i + 3] *= rtb * w1;
+                            } else {
+                                v[4 * i + 0] *= s0 < ta ? rta * w0 : (s0 == ta ? gta : 0.f);
+                                v[4 * i + 1] *= s1 < ta ? rta * w1 : (s1 == ta ? gta : 0.f);
+                                v[4 * i + 2] *= s0 < tb ? rtb * w0 : (s0 == tb ? gtb : 0.f);
+                                v[4 * i + 3] *= s1 < tb ? rtb * w1 : (s1 == tb ? gtb : 0.f);
+                                if (R == 1) {
+                                    // SISO: the skip D x_t rides on the intra UMMA as D on the
+                                    // diagonal of the scores (its B operand is x itself)
+                                    v[4 * i + 0] += s0 == ta ? Dh : 0.f;
+                                    v[4 * i + 1] += s1 == ta ? Dh : 0.f;
+                                    v[4 * i + 2] += s0 == tb ? Dh : 0.f;
+                                    v[4 * i + 3] += s1 == tb ? Dh : 0.f;
+                                }
                             }
                             const int cc = col >> 3;
                             *reinterpret_cast<uint32_t *>(sp + ra * 128 + ((cc ^ (ra & 7)) << 4) + 2 * cq) =
