@@ -431,9 +431,17 @@ class PrepWorkload(ScanWorkload):
     default workload's inputs, outputs preallocated."""
 
     def __init__(self, idx, device):
-        super().__init__(idx, device)
-        c = self.c
+        from state_space_lm_b200 import m3
+        self.m3 = m3
+        self.c = c = dict(gen.CONFIGS[idx])
+        self.idx = idx
+        self.host = gen.config_inputs(idx)
+        self.host.pop("generator")
+        self.dev = {k: v.to(device) for k, v in self.host.items() if isinstance(v, torch.Tensor)}
         Bt, T, H, N = c["batch"], c["seqlen"], c["nheads"], c["dstate"]
+        self.G, self.K = c.get("ngroups", 0) or H, c.get("rope_pairs", 0) or N // 2
+        self.mimo = False
+        self.units = Bt * T
         self.kind = c["prep"]
         d = self.dev
         if self.kind == "discretize":

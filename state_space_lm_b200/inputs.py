@@ -51,9 +51,11 @@ CONFIGS = {
     # the backward (all input gradients) of the default workload
     8: dict(name="bwd_siso_8x2048_h16_p64_n128", batch=8, seqlen=2048, nheads=16, headdim=64,
             dstate=128, rank=1, chunk=64, dtype="bf16", dt_shift=-2.0, grad=True),
-    # the standalone prep passes on the default workload's inputs: S1 alone
-    # (alpha, beta, gamma out) and S2 alone (rotated B, C and the angle out)
-    9: dict(name="discretize_8x2048_h16", batch=8, seqlen=2048, nheads=16, headdim=64,
+    # the standalone prep passes: S1 alone (alpha, beta, gamma out) over the
+    # decode workload's 512 sequences at the default 2048 tokens (the default
+    # batch's dt and lam, 2 MB, would sit in L2), and S2 alone (rotated B, C and
+    # the angle out) on the default workload's inputs
+    9: dict(name="discretize_512x2048_h16", batch=512, seqlen=2048, nheads=16, headdim=64,
             dstate=128, rank=1, chunk=64, dtype="bf16", dt_shift=-2.0, prep="discretize"),
     10: dict(name="rope_bc_8x2048_h16_n128", batch=8, seqlen=2048, nheads=16, headdim=64,
              dstate=128, rank=1, chunk=64, dtype="bf16", dt_shift=-2.0, prep="rope"),
@@ -143,14 +145,31 @@ def decode_step_inputs(generator, batch, nheads, headdim, dstate, dtype="bf16",
     return out
 
 
+def discretize_inputs(batch, seqlen, nheads, dt_shift=-2.0, seed=SEED_BASE):
+    """Inputs of a standalone discretization: dt, lam (Bt,T,H) and A (H), drawn
+    from one generator in the order dt, A, lam with the laws above."""
+    g = make_generator(seed)
+    Bt, T, H = batch, seqlen, nheads
+    out = {}
+    out["dt"] = torch.nn.functional.softplus(_normal(g, (Bt, T, H)) + dt_shift).float()
+    out["A"] = (-torch.exp(_uniform(g, (H,), 0.0, 1.0))).float()
+    out["lam"] = torch.sigmoid(_normal(g, (Bt, T, H))).float()
+    out["generator"] = g
+    return out
+
+
 def config_inputs(idx, seed=None, **overrides):
     """Inputs of workload ``idx`` (0-3, 7 and 8: one chunked-scan call, forward
     or backward; 4-6: the prefill of a decode workload -- its steps come from
-    ``decode_step_inputs`` with the returned generator).  The backward's dy is
-    drawn by ``grad_seed``."""
+    ``decode_step_inputs`` with the returned generator; 9: dt, A, lam of a
+    standalone discretization; 10: a chunked-scan call's inputs, of which the
+    standalone rotation uses B, C, theta and dt).  The backward's dy is drawn
+    by ``grad_seed``."""
     c = dict(CONFIGS[idx])
     c.update(overrides)
     s = SEED_BASE + idx if seed is None else seed
+    if c.get("prep") == "discretize":
+        return discretize_inputs(c["batch"], c["seqlen"], c["nheads"], dt_shift=c["dt_shift"], seed=s)
     return scan_inputs(c["batch"], c["seqlen"], c["nheads"], c["headdim"], c["dstate"],
                        rank=c["rank"], dtype=c["dtype"], dt_shift=c["dt_shift"], seed=s,
                        mimo_weights=c["rank"] > 1, ngroups=c.get("ngroups", 0),

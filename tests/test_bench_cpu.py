@@ -56,7 +56,7 @@ def test_backward_bytes_and_flops():
 
 def test_prep_bytes():
     # S1: dt, lam in, alpha, beta, gamma out (20 B per token-head) + A
-    assert bench.prep_bytes(gen.CONFIGS[9]) == 8 * 2048 * 16 * 20 + 16 * 4
+    assert bench.prep_bytes(gen.CONFIGS[9]) == 512 * 2048 * 16 * 20 + 16 * 4
     # S2: B, C in (512), theta (256), dt (4), rotated B, C out (512) = 1284 B
     # per token-head, + the final angle per lane
     assert bench.prep_bytes(gen.CONFIGS[10]) == 8 * 2048 * 16 * 1284 + 128 * 64 * 4

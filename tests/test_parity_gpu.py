@@ -77,6 +77,50 @@ def test_rope_bc(dtype, R, T, N, bcnorm):
     assert relerr(ang, rA) <= 1e-5
 
 
+@pytest.mark.parametrize("dtype", [FP32, BF16])
+@pytest.mark.parametrize("N,R,bcnorm,T", [(128, 1, False, 700), (256, 1, True, 100), (256, 2, False, 65),
+                                          (64, 1, True, 1), (128, 4, True, 33)])
+def test_rope_bc_tiles(dtype, N, R, bcnorm, T):
+    """The tiled rotation (whole quads of pairs): several tiles with a ragged
+    last one, the angle carried from tile to tile, a slice of a row per CTA
+    without QkNorm and the whole row with it (dstate 256: one token per warp)."""
+    inp = gen.scan_inputs(2, T, 3, 4, N, rank=R, dtype=dtype, seed=13 + N + T, mimo_weights=R > 1,
+                          bcnorm=bcnorm)
+    _, _, a0 = _states(2, 3, N, 4, 6)
+    d = cuda(inp)
+    Br, Cr, ang = m3.rope_bc(d["B"], d["C"], d["theta"], d["dt"], angle0=a0.cuda(), norm=norm_dev(inp))
+    rB, rC, rA = oracle.rope_bc(to_f64(inp["B"]), to_f64(inp["C"]), to_f64(inp["theta"]),
+                                to_f64(inp["dt"]), angle0=to_f64(a0), norm=norm_f64(inp))
+    tol = _tol(dtype)
+    assert relerr(Br, rB) <= tol
+    assert relerr(Cr, rC) <= tol
+    assert relerr(ang, rA) <= 1e-5
+
+
+def test_rope_bc_empty_sequence_passes_the_angle_through():
+    inp = gen.scan_inputs(2, 0, 3, 4, 128, seed=14)
+    _, _, a0 = _states(2, 3, 128, 4, 8)
+    d = cuda(inp)
+    _, _, ang = m3.rope_bc(d["B"], d["C"], d["theta"], d["dt"], angle0=a0.cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(ang.cpu(), a0)
+
+
+def test_rope_bc_full_size_sampled_lanes():
+    """The standalone rotation at the default workload's shape (the S2 bench
+    line), compared on sampled (b, h) lanes."""
+    inp = gen.config_inputs(1)
+    d = cuda({k: inp[k] for k in ("B", "C", "theta", "dt")})
+    Br, Cr, ang = m3.rope_bc(d["B"], d["C"], d["theta"], d["dt"])
+    torch.cuda.synchronize()
+    for b, h in sample_lanes(8, 16):
+        sl = lambda t: to_f64(t[b:b + 1, :, h:h + 1])
+        rB, rC, rA = oracle.rope_bc(sl(inp["B"]), sl(inp["C"]), sl(inp["theta"]), sl(inp["dt"]))
+        assert relerr(Br[b:b + 1, :, h:h + 1], rB) <= 2e-2
+        assert relerr(Cr[b:b + 1, :, h:h + 1], rC) <= 2e-2
+        assert relerr(ang[b:b + 1, h:h + 1], rA) <= 1e-5
+
+
 # ----------------------------------------------------------------------------
 # S3 SISO chunked scan: small cases, every element
 # ----------------------------------------------------------------------------
