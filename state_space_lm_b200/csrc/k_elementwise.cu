@@ -270,14 +270,16 @@ __device__ __forceinline__ void sincos_for(const float *, float x, float *s, flo
 // angle carried from the previous tile, so every token's angle is the
 // sequential sum without a sequential walk.  The next tile's inputs are
 // loaded while the current one is rotated (rank 1).  QkNorm needs the whole
-// row, so with a norm QS covers all N / 8 quads.  Needs N % 8 == 0 and K % 4 ==
+// row, so with a norm QS covers all N / 8 quads.  PLAIN (rank 1, no QkNorm,
+// no bias) carries none of that code and fits four CTAs per SM, so the
+// default workload's 512 CTAs run in one wave.  Needs N % 8 == 0 and K % 4 ==
 // 0 (a quad turns wholly or not at all).
-template <typename T, int QS>
-__global__ void __launch_bounds__(256, 3) k_rope_tiled(RopeArgs a) {
+template <typename T, int QS, bool PLAIN>
+__global__ void __launch_bounds__(256, PLAIN ? 4 : 3) k_rope_tiled(RopeArgs a) {
     constexpr int TT = 256 / QS;
     const int64_t lane = blockIdx.x, b = lane / a.H, h = lane % a.H;
     const int64_t Tn = a.T, H = a.H, G = a.G, hg = h / (H / G);
-    const int N = (int)a.N, R = (int)a.R, K = (int)a.K;
+    const int N = (int)a.N, R = PLAIN ? 1 : (int)a.R, K = (int)a.K;
     const int tid = threadIdx.x, warp = tid >> 5, l32 = tid & 31;
     const int tr = tid / QS, qq = tid % QS;
     const int jq = (int)blockIdx.y * QS + qq;
@@ -287,7 +289,7 @@ __global__ void __launch_bounds__(256, 3) k_rope_tiled(RopeArgs a) {
     T *Bo = static_cast<T *>(a.Bo);
     T *Co = static_cast<T *>(a.Co);
     const NormArgs nr = a.nrm;
-    const bool has_norm = nr.wB || nr.wC;
+    const bool has_norm = !PLAIN && (nr.wB || nr.wC), has_bias = !PLAIN && (nr.biasB || nr.biasC);
     __shared__ float4 wt[2][8][QS];      // per-warp angle totals, double-buffered
     __shared__ float4 carry[2][QS];      // angle entering the tile, double-buffered
 
@@ -389,7 +391,7 @@ __global__ void __launch_bounds__(256, 3) k_rope_tiled(RopeArgs a) {
                     if (nr.wC) fc[e] *= ic * nr.wC[8 * jq + e];
                 }
             }
-            if (nr.biasB || nr.biasC) {
+            if (has_bias) {
                 const int64_t bo = (h * R + r) * N + 8 * jq;
 #pragma unroll
                 for (int e = 0; e < 8; e++) {
@@ -419,21 +421,27 @@ __global__ void __launch_bounds__(256, 3) k_rope_tiled(RopeArgs a) {
     }
 }
 
-template <typename T>
-static cudaError_t launch_rope_tiled(const RopeArgs &a, int qs, cudaStream_t s) {
+template <typename T, bool PLAIN>
+static cudaError_t launch_rope_tiled_p(const RopeArgs &a, int qs, cudaStream_t s) {
     const int nq = (int)(a.N / 8);
     const dim3 grid((unsigned)(a.Bt * a.H), (unsigned)(nq / qs));
     switch (qs) {
-        case 1: k_rope_tiled<T, 1><<<grid, 256, 0, s>>>(a); break;
-        case 2: k_rope_tiled<T, 2><<<grid, 256, 0, s>>>(a); break;
-        case 4: k_rope_tiled<T, 4><<<grid, 256, 0, s>>>(a); break;
-        case 8: k_rope_tiled<T, 8><<<grid, 256, 0, s>>>(a); break;
-        case 16: k_rope_tiled<T, 16><<<grid, 256, 0, s>>>(a); break;
-        case 32: k_rope_tiled<T, 32><<<grid, 256, 0, s>>>(a); break;
+        case 1: k_rope_tiled<T, 1, PLAIN><<<grid, 256, 0, s>>>(a); break;
+        case 2: k_rope_tiled<T, 2, PLAIN><<<grid, 256, 0, s>>>(a); break;
+        case 4: k_rope_tiled<T, 4, PLAIN><<<grid, 256, 0, s>>>(a); break;
+        case 8: k_rope_tiled<T, 8, PLAIN><<<grid, 256, 0, s>>>(a); break;
+        case 16: k_rope_tiled<T, 16, PLAIN><<<grid, 256, 0, s>>>(a); break;
+        case 32: k_rope_tiled<T, 32, PLAIN><<<grid, 256, 0, s>>>(a); break;
         default: return cudaErrorInvalidValue;
     }
     count_launch();
     return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_rope_tiled(const RopeArgs &a, int qs, cudaStream_t s) {
+    const bool plain = a.R == 1 && !a.nrm.wB && !a.nrm.wC && !a.nrm.biasB && !a.nrm.biasC;
+    return plain ? launch_rope_tiled_p<T, true>(a, qs, s) : launch_rope_tiled_p<T, false>(a, qs, s);
 }
 
 // Quads per CTA of the tiled kernel, or 0 when it does not apply: whole quads
