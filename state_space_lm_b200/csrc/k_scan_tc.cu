@@ -507,15 +507,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tma_prefetch4(&map_th, 0, (int)h, t0, (int)b);
                 tma_prefetch4(&map_x, 0, (int)h, t0, (int)b);
             };
-            if (elect_one())
-                for (int c = 1; c < PFD; c++) prefetch(c);
-            __syncwarp();
             int issued = 0;
             for (int c = 0; c < nchunks; c++) {
                 const int sb = c % NB, kb = c / NB, sx = c % L::NXR, kx = c / L::NXR;
                 const int t0 = (int)(t_beg + (int64_t)c * QT);
-                if (elect_one()) prefetch(c + PFD);
-                __syncwarp();
                 if (kb > 0 && !warp_wait(bar(B_BEMPTY + sb), (kb - 1) & 1, abort_flag, a.err, 1)) break;
                 const uint32_t st = sbase + L::OFF_BCT + sb * L::SZ_BCT;
                 const uint32_t fb = bar(B_BFULL + sb);
@@ -530,6 +525,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (elect_one()) {
                     mbar_expect_tx(xb, L::SZ_X);
                     tma_load4(sbase + L::OFF_X + sx * L::SZ_X, &map_x, 0, (int)h, t0, (int)b, xb);
+                    // the L2 prefetches go out after this chunk's loads: at the
+                    // start every CTA's first chunk then comes before the
+                    // look-ahead traffic of all of them
+                    if (c == 0)
+                        for (int k = 1; k <= PFD; k++) prefetch(k);
+                    else
+                        prefetch(c + PFD);
                 }
                 __syncwarp();
                 issued = c + 1;
@@ -976,7 +978,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (c > 0 && !warp_wait_spin(bar(B_STAKEN), (c - 1) & 1, abort_flag, a.err, 11)) break;
                 tc_fence_after();
                 if (elect_one()) {
-#pragma unroll 1
+#pragma unroll
                     for (int kk = 0; kk < N / 16; kk++)
                         umma(tmem + COL_D1, d_cb_k + kstep_k(kk), d_bb_k + kstep_k(kk), id_kk, kk > 0);
                     umma_commit(bar(B_SFULL));
@@ -985,7 +987,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (!warp_wait_spin(bar(B_STTAKEN), c & 1, abort_flag, a.err, 12)) break;
                 tc_fence_after();
                 if (elect_one()) {
-#pragma unroll 1
+#pragma unroll
                     for (int kk = 0; kk < Q / 16; kk++)
                         umma(tmem + COL_D4, d_bb_mn + kstep_mn(kk), d_xw + kstep_mn(kk), id_st, kk > 0);
                     umma_commit(bar(B_STFULL));
@@ -997,7 +999,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tc_fence_after();
                 if (elect_one()) {
                     const uint32_t d3 = tmem + COL_D3 + (uint32_t)(c & 1) * D3_STRIDE;
-#pragma unroll 1
+#pragma unroll
                     for (int kk = 0; kk < N / 16; kk++)
                         umma(d3, d_cb_k + kstep_k(kk), dg + kstep_mn(kk), id_kmn, kk > 0);
                     // SISO: B, C and Xw of chunk c are read by now (the intra UMMA
@@ -1008,7 +1010,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (!warp_wait_spin(bar(B_SPFULL), c & 1, abort_flag, a.err, 14)) break;
                 tc_fence_after();
                 if (elect_one()) {
-#pragma unroll 1
+#pragma unroll
                     for (int kk = 0; kk < Q / 16; kk++)
                         umma(tmem + COL_D2, d_sp + (uint64_t)((kk * 32) >> 4), dx + kstep_mn(kk), id_kmn, kk > 0);
                     umma_commit(bar(B_YFULL));
