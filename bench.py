@@ -688,9 +688,12 @@ def run_ours(args, world, rank, local):
         w.step()
     torch.cuda.synchronize(device)
 
-    # ---- device-timed region: K steps, inputs resident in HBM ----
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
+    # ---- device-timed region: K steps back to back, inputs resident in HBM ----
+    # One event before the first step and one after the last, on the launching
+    # stream: a pair of events around every step would put two event writes
+    # between consecutive launches (about 5 % of a 0.1 ms step, measured).  The
+    # average launch time of a one-launch step is then the region time / K; a
+    # step of several launches reports the whole call.
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize(device)
@@ -700,16 +703,14 @@ def run_ours(args, world, rank, local):
     with ClockSampler(local) as clk:
         start.record(stream)
         for i in range(args.steps):
-            evs[i][0].record(stream)
             w.step()
-            evs[i][1].record(stream)
         stop.record(stream)
         torch.cuda.synchronize(device)
     launches = m3.launch_count() - n0
     if dist is not None:
         dist.barrier()
     elapsed = start.elapsed_time(stop) / 1e3
-    kernel_s = statistics.mean(a.elapsed_time(b) for a, b in evs) / 1e3
+    kernel_s = elapsed / args.steps
     value, tmax, units = aggregate(elapsed, w.units * args.steps, dist, device)
 
     # ---- end to end through the C ABI with host buffers ----
