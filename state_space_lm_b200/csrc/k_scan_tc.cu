@@ -887,7 +887,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint8_t *xt = sm + L::OFF_X + sx * L::SZ_X;
                 uint4 *dw = reinterpret_cast<uint4 *>(sm + L::OFF_XW + ob * (Q * P * 2));
                 uint4 *dr = reinterpret_cast<uint4 *>(sm + L::OFF_XR + ob * (Q * P * 2));
-#pragma unroll 4
+                // unrolled twice, not four times: measured 4 % faster calls
+                // (the hot code of all roles shares the instruction cache)
+#pragma unroll 2
                 for (int v = l32; v < Q * P / 8; v += 32) {
                     const int row = v >> 3, pc = v & 7;
                     const int sq = row / R;                       // token of the row
