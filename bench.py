@@ -492,6 +492,17 @@ class PrepWorkload(ScanWorkload):
         return nb * H, time.perf_counter() - t0, 1
 
 
+def decode_config(c):
+    """The config dict of a decode workload's bench line (both arms)."""
+    factored = c.get("state") == "factored"
+    state_bytes = (1 if factored else 2) * c["batch"] * c["nheads"] * c["dstate"] * c["headdim"] * 4
+    return {"workload": c["name"], "batch": c["batch"], "nheads": c["nheads"], "headdim": c["headdim"],
+            "dstate": c["dstate"], "prefill": c["seqlen"], "decode_steps_per_call": 1,
+            "rank": c["rank"], "state": "factored (h, b_prev, x_prev)" if factored else "full (h, prev_Bx)",
+            "inputs": "x/B/C bf16, dt/lam/theta fp32 per step; fp32 state and angle",
+            "l2": "state larger than L2 (%.0f MB vs 126 MB), no flush" % (state_bytes / 1e6)}
+
+
 class DecodeWorkload:
     """Decode steps: every step advances all (batch, head) lanes by one token.
     The carried state comes from a seeded prefill (a chunked forward over the
@@ -554,12 +565,7 @@ class DecodeWorkload:
                                 self.h, self.u, self.a, y_out=y, stream=stream)
 
     def config(self):
-        c = self.c
-        return {"workload": c["name"], "batch": c["batch"], "nheads": c["nheads"], "headdim": c["headdim"],
-                "dstate": c["dstate"], "prefill": c["seqlen"], "decode_steps_per_call": 1,
-                "rank": c["rank"], "state": "factored (h, b_prev, x_prev)" if self.factored else "full (h, prev_Bx)",
-                "inputs": "x/B/C bf16, dt/lam/theta fp32 per step; fp32 state and angle",
-                "l2": "state larger than L2 (%.0f MB vs 126 MB), no flush" % (self.input_bytes / 1e6)}
+        return decode_config(self.c)
 
 
 def cpu_model():
@@ -824,6 +830,10 @@ def run_reference(args, world, rank):
     w.mimo = w.c["rank"] > 1
     w.G = w.c.get("ngroups", 0) or w.c["nheads"]
     w.K = w.c.get("rope_pairs", 0) or w.c["dstate"] // 2
+    # the same config dict as the GPU arm's line (input bytes from the host copies)
+    keys = (("dt", "A", "lam") if prep == "discretize" else ("B", "C", "theta", "dt")) if prep else \
+        [k for k, v in w.host.items() if isinstance(v, torch.Tensor)]
+    w.input_bytes = sum(w.host[k].numel() * w.host[k].element_size() for k in keys)
     cores = os.cpu_count() or 1
     H = w.c["nheads"]
     total_lanes = w.c["batch"] * H
@@ -846,9 +856,7 @@ def run_reference(args, world, rank):
     line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": c["name"], "batch": c["batch"], "seqlen": c["seqlen"],
-                       "nheads": c["nheads"], "headdim": c["headdim"], "dstate": c["dstate"],
-                       "rank": c["rank"], "chunk": c["chunk"]},
+            "config": dict(w.config(), parallelism="replicas x%d (independent lanes, no collective)" % world),
             "impl": "reference",
             "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": int(used), "kind": "oracle",
                              "sample": sample},
@@ -867,8 +875,7 @@ def run_reference_decode(args, world):
     line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": c["name"], "batch": c["batch"], "nheads": c["nheads"], "headdim": c["headdim"],
-                       "dstate": c["dstate"], "rank": c["rank"], "state": c.get("state", "full")},
+            "config": dict(decode_config(c), parallelism="replicas x%d (independent lanes, no collective)" % world),
             "impl": "reference",
             "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": int(used), "kind": "oracle",
                              "sample": "%d of %d sequences (all heads) per decode step, fp64 C step"
