@@ -166,83 +166,178 @@ cudaError_t launch_decode(const DecodeArgs &a, m3_dtype dt, cudaStream_t s) {
 //   h <- alpha h + beta U_prev + gamma U_t
 //   y = sum_r W_y[r] (Cbar_r^T h) + D x_t
 //   prev_Bx <- U_t   or   b_prev <- Bbar, x_prev <- x_t      (factored)
-// One CTA per (b, h) lane; rank bound RT (R <= RT, the rest predicated off);
-// threads stream 4-wide rows of h (and prev_Bx).  The factored form reads and
-// writes only h, so a step moves about half the bytes of the full form.
+// One CTA per (b, h) lane; rank bound RT (R <= RT, the ranks past R are zero
+// rows); threads stream 4-wide rows of h (and prev_Bx).  The factored form
+// reads and writes only h, so a step moves about half the bytes of the full
+// form.  Its update of an (n, p) element is one sum of 2R products,
+//   h' = alpha h + sum_r (beta b_prev_r[n]) (W_x[r][p] x_prev[p])
+//                      + (gamma Bbar_r[n]) (W_x[r][p] x[p]),
+// the row factors in shared memory ([n][term], read as 16-byte vectors) and
+// the column factors in registers.  Each thread's first NB rows of h (and
+// prev_Bx) are loaded before anything else, so their HBM latency overlaps the
+// rotation of B and C; the y partial sums meet in warp shuffles and one
+// shared-memory pass over the warps.
 // ---------------------------------------------------------------------------
-template <typename T, int RT, bool FACT>
-__global__ void __launch_bounds__(256) k_decode_gen(DecodeArgs a) {
-    constexpr int VEC = 4;
+template <int M>
+__device__ __forceinline__ void lds_row(const float *p, float (&o)[M]) {
+    if constexpr (M % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < M / 4; i++) {
+            const float4 v = reinterpret_cast<const float4 *>(p)[i];
+            o[4 * i] = v.x; o[4 * i + 1] = v.y; o[4 * i + 2] = v.z; o[4 * i + 3] = v.w;
+        }
+    } else if constexpr (M == 2) {
+        const float2 v = *reinterpret_cast<const float2 *>(p);
+        o[0] = v.x; o[1] = v.y;
+    } else {
+#pragma unroll
+        for (int i = 0; i < M; i++) o[i] = p[i];
+    }
+}
+
+__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(
+                     dst_smem))),
+                 "l"(src)
+                 : "memory");
+}
+
+template <int RT, bool FACT>
+struct DecodeGenPlan {
+    static constexpr int NV = FACT ? 2 * RT : RT;   // update terms per element
+    static constexpr int NS = FACT ? 1 : 2;         // N x P states copied in (h, prev_Bx)
+    // y partial sums: one per warp when the lanes of a column share a warp
+    static __host__ __device__ int parts(int P, int nt) {
+        const int PV = P / 4;
+        return (PV < 32 && (PV & (PV - 1)) == 0) ? nt / 32 : nt / PV;
+    }
+    static __host__ __device__ size_t smem_floats(int N, int P, int nt) {
+        return (size_t)NS * N * P + (size_t)NV * N + 2 * (size_t)RT * N + N / 2 + 16 * RT +
+               (size_t)(parts(P, nt) + 1) * RT * P;
+    }
+};
+
+// NC, PC: dstate and headdim fixed at compile time (0: taken from the
+// arguments), so that the row loops unroll fully and the indexing folds.
+constexpr int DEC_THREADS = 256;
+template <typename T, int RT, bool FACT, int NC, int PC>
+__global__ void __launch_bounds__(DEC_THREADS, RT == 1 ? 4 : (RT >= 8 ? 1 : (NC ? 3 : 2))) k_decode_gen(DecodeArgs a) {
+    using PL = DecodeGenPlan<RT, FACT>;
+    constexpr int VEC = 4, NV = PL::NV, nt = DEC_THREADS;
     const int64_t lane = blockIdx.x, h = lane % a.H;
-    const int P = (int)a.P, N = (int)a.N, NP2 = N / 2, R = (int)a.R, K = (int)a.K;
-    const int tid = threadIdx.x, nt = blockDim.x;
+    const int P = PC ? PC : (int)a.P, N = NC ? NC : (int)a.N, NP2 = N / 2, R = (int)a.R, K = (int)a.K;
+    const int tid = threadIdx.x, wid = tid >> 5, ln = tid & 31;
     const int64_t grow = (lane / a.H) * a.G + h / (a.H / a.G);  // the group's B/C rows
     const T *x = static_cast<const T *>(a.x);
     const T *Bg = static_cast<const T *>(a.B) + grow * R * N;
     const T *Cg = static_cast<const T *>(a.C) + grow * R * N;
     T *y = static_cast<T *>(a.y);
 
-    extern __shared__ float sm[];
-    float *Bb = sm;                 // RT x N  rotated B of this token
-    float *Cb = Bb + RT * N;        // RT x N  rotated C
-    float *Pb = Cb + RT * N;        // RT x N  b_prev (factored form)
-    float *red = Pb + RT * N;       // 32
-    float *phs = red + 32;          // N/2 angles of this token
-    float *ypart = phs + N / 2;     // ngroups x RT x P
+    extern __shared__ float4 sm4[];
+    float *hs = reinterpret_cast<float *>(sm4);   // N x P   h of this lane (then prev_Bx)
+    float *Vs = hs + PL::NS * N * P;              // N x NV  row factors of the update
+    float *Cs = Vs + NV * N;                      // N x RT  rotated C, [n][rank]
+    float *Bn = Cs + RT * N;                      // RT x N  rotated B (the next b_prev)
+    float *phs = Bn + RT * N;                     // N/2     angles of this token
+    float *red = phs + N / 2;                     // 16 RT   norm partial sums
+    const int npart = PL::parts(P, nt);
+    float *ypart = red + 16 * RT;                 // npart x RT x P
+    float *yr = ypart + npart * RT * P;           // RT x P
 
     const int PV = P / VEC;              // vectors per state row
     const int ngroups = nt / PV;         // rows streamed concurrently
     const int pv = tid % PV, ng = tid / PV;
-    float4 *hp = reinterpret_cast<float4 *>(a.h + lane * (int64_t)N * P);
-    // start pulling my rows of h into L2 now: the state stream below then
-    // finds them there instead of waiting on HBM after the prologue
-    if (ng < ngroups)
-        for (int n = ng; n < N; n += ngroups)
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(hp + n * PV + pv));
+    const bool streams = ng < ngroups;
+    float4 *hp = reinterpret_cast<float4 *>(a.h + lane * (int64_t)N * P) + pv;
+    float4 *up = FACT ? hp : reinterpret_cast<float4 *>(a.prevBx + lane * (int64_t)N * P) + pv;
+    float *us = hs + (FACT ? 0 : N * P);
+    if (streams) {
+#pragma unroll(NC ? 8 : 4)
+        for (int n = ng; n < N; n += ngroups) {
+            cp_async16(hs + n * P + pv * VEC, hp + n * PV);
+            if (!FACT) cp_async16(us + n * P + pv * VEC, up + n * PV);
+        }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
 
     const float dl = a.dt[lane], lm = a.lam[lane];
     const float al = expf(dl * a.A[h]);
     const float be = (1.f - lm) * dl * al;
     const float ga = lm * dl;
 
-    // QkNorm inverse RMS per rank
+    // column factors: W_x[r][p] x_prev[p] (factored form) and W_x[r][p] x[p]
+    float Z[NV][VEC];
+    {
+        float xv[VEC], xq[VEC];
+#pragma unroll
+        for (int k = 0; k < VEC; k++) {
+            xv[k] = ldf(x, lane * P + pv * VEC + k);
+            xq[k] = FACT ? a.xprev[lane * P + pv * VEC + k] : 0.f;
+        }
+#pragma unroll
+        for (int r = 0; r < RT; r++)
+#pragma unroll
+            for (int k = 0; k < VEC; k++) {
+                const int p = pv * VEC + k;
+                const float w = r < R ? (a.Wx ? a.Wx[(h * R + r) * P + p] : 1.f) : 0.f;
+                if (FACT) {
+                    Z[r][k] = w * xq[k];
+                    Z[RT + r][k] = w * xv[k];
+                } else {
+                    Z[r][k] = w * xv[k];
+                }
+            }
+    }
+
+    // QkNorm inverse RMS per rank, every rank in one pass
     float invB[RT], invC[RT];
 #pragma unroll
     for (int r = 0; r < RT; r++) { invB[r] = 1.f; invC[r] = 1.f; }
     if (a.nrm.wB || a.nrm.wC) {
+        float sb[RT], sc[RT];
+#pragma unroll
+        for (int r = 0; r < RT; r++) { sb[r] = 0.f; sc[r] = 0.f; }
+        for (int it = tid; it < R * N; it += nt) {
+            const int r = it / N;
+            const float vb = ldf(Bg, it), vc = ldf(Cg, it);
+#pragma unroll
+            for (int rr = 0; rr < RT; rr++)
+                if (rr == r) { sb[rr] += vb * vb; sc[rr] += vc * vc; }
+        }
+#pragma unroll
+        for (int r = 0; r < RT; r++)
+            for (int o = 16; o > 0; o >>= 1) {
+                sb[r] += __shfl_xor_sync(0xffffffffu, sb[r], o);
+                sc[r] += __shfl_xor_sync(0xffffffffu, sc[r], o);
+            }
+        if (ln == 0)
+#pragma unroll
+            for (int r = 0; r < RT; r++) { red[(wid * RT + r) * 2] = sb[r]; red[(wid * RT + r) * 2 + 1] = sc[r]; }
+        __syncthreads();
 #pragma unroll
         for (int r = 0; r < RT; r++) {
-            if (r >= R) break;
-            float sb = 0.f, sc = 0.f;
-            for (int n = tid; n < N; n += nt) {
-                const float vb = ldf(Bg, r * N + n), vc = ldf(Cg, r * N + n);
-                sb += vb * vb;
-                sc += vc * vc;
-            }
-            sb = block_sum(sb, red);
-            __syncthreads();
-            sc = block_sum(sc, red);
-            __syncthreads();
-            invB[r] = rsqrtf(sb / N + a.nrm.eps);
-            invC[r] = rsqrtf(sc / N + a.nrm.eps);
+            float s = 0.f, c = 0.f;
+            for (int w = 0; w < (nt >> 5); w++) { s += red[(w * RT + r) * 2]; c += red[(w * RT + r) * 2 + 1]; }
+            invB[r] = rsqrtf(s / N + a.nrm.eps);
+            invC[r] = rsqrtf(c / N + a.nrm.eps);
         }
     }
-    if (FACT)
-        for (int k = tid; k < R * N; k += nt) Pb[k] = a.bprev[lane * R * N + k];
-    for (int j = tid; j < K; j += nt) {
-        const float phi = a.angle[lane * K + j] + dl * a.theta[lane * K + j];
-        a.angle[lane * K + j] = phi;
-        phs[j] = phi;
-    }
-    __syncthreads();
-    // one (pair, rank) per thread: every rank's loads in flight at once
-    for (int it = tid; it < R * NP2; it += nt) {
-        const int j = it % NP2, r = it / NP2;
-        float sn = 0.f, cn = 1.f;
-        if (j < K) sincosf(phs[j], &sn, &cn);
-        {
+
+    // one (pair, rank) per thread, rank fastest: every rank's loads in flight
+    // at once, and the [n][rank] stores below spread over the banks
+    for (int it = tid; it < RT * NP2; it += nt) {
+        const int j = it / RT, r = it % RT;
+        float b0 = 0.f, b1 = 0.f, c0 = 0.f, c1 = 0.f, q0 = 0.f, q1 = 0.f;
+        if (r < R) {
             const int64_t o = r * N + 2 * j;
-            float b0 = ldf(Bg, o), b1 = ldf(Bg, o + 1), c0 = ldf(Cg, o), c1 = ldf(Cg, o + 1);
+            b0 = ldf(Bg, o); b1 = ldf(Bg, o + 1); c0 = ldf(Cg, o); c1 = ldf(Cg, o + 1);
+            if (FACT) { q0 = a.bprev[lane * R * N + o]; q1 = a.bprev[lane * R * N + o + 1]; }
+            float sn = 0.f, cn = 1.f;
+            if (j < K) {
+                const float phi = a.angle[lane * K + j] + dl * a.theta[lane * K + j];
+                if (r == 0) phs[j] = phi;   // written back after every read of the old angle
+                sincosf(phi, &sn, &cn);
+            }
             float ib = 1.f, ic = 1.f;   // this rank's inverse RMS (selected, not indexed)
 #pragma unroll
             for (int rr = 0; rr < RT; rr++)
@@ -252,116 +347,139 @@ __global__ void __launch_bounds__(256) k_decode_gen(DecodeArgs a) {
             const int64_t bo = (h * R + r) * N + 2 * j;
             if (a.nrm.biasB) { b0 += a.nrm.biasB[bo]; b1 += a.nrm.biasB[bo + 1]; }
             if (a.nrm.biasC) { c0 += a.nrm.biasC[bo]; c1 += a.nrm.biasC[bo + 1]; }
-            Bb[r * N + 2 * j] = cn * b0 - sn * b1;
-            Bb[r * N + 2 * j + 1] = sn * b0 + cn * b1;
-            Cb[r * N + 2 * j] = cn * c0 - sn * c1;
-            Cb[r * N + 2 * j + 1] = sn * c0 + cn * c1;
+            const float rb0 = cn * b0 - sn * b1, rb1 = sn * b0 + cn * b1;
+            const float rc0 = cn * c0 - sn * c1, rc1 = sn * c0 + cn * c1;
+            b0 = rb0; b1 = rb1; c0 = rc0; c1 = rc1;
+        }
+        Cs[(2 * j) * RT + r] = c0;
+        Cs[(2 * j + 1) * RT + r] = c1;
+        if (FACT) {
+            Vs[(2 * j) * NV + r] = be * q0;
+            Vs[(2 * j + 1) * NV + r] = be * q1;
+            Vs[(2 * j) * NV + RT + r] = ga * b0;
+            Vs[(2 * j + 1) * NV + RT + r] = ga * b1;
+            Bn[r * N + 2 * j] = b0;
+            Bn[r * N + 2 * j + 1] = b1;
+        } else {
+            Vs[(2 * j) * NV + r] = b0;
+            Vs[(2 * j + 1) * NV + r] = b1;
         }
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");   // this thread's rows (it reads only those)
     __syncthreads();
 
-    // Small ranks keep X_r = W_x[r] x (and W_x[r] x_prev) per rank; ranks 4
-    // and 8 keep W_x[r] alone and scale the rank sums by x (x_prev) after, which
-    // holds half the registers:  U_t[n][p] = x[p] sum_r Bbar_r[n] W_x[r][p].
-    constexpr bool WF = RT >= 4;
-    constexpr int RX = WF ? 1 : RT;                 // per-rank products kept
-    float xv[VEC], xq[VEC], W[RT][VEC], X[RX][VEC], Xp[RX][VEC], Y[RT][VEC];
+    float Y[RT][VEC];
 #pragma unroll
-    for (int k = 0; k < VEC; k++) {
-        xv[k] = ldf(x, lane * P + pv * VEC + k);
-        xq[k] = FACT ? a.xprev[lane * P + pv * VEC + k] : 0.f;
-    }
+    for (int r = 0; r < RT; r++)
 #pragma unroll
-    for (int r = 0; r < RT; r++) {
-#pragma unroll
-        for (int k = 0; k < VEC; k++) {
-            const int p = pv * VEC + k;
-            W[r][k] = r < R ? (a.Wx ? a.Wx[(h * R + r) * P + p] : 1.f) : 0.f;
-            Y[r][k] = 0.f;
-            if (!WF) {
-                X[r < RX ? r : 0][k] = W[r][k] * xv[k];
-                Xp[r < RX ? r : 0][k] = W[r][k] * xq[k];
-            }
-        }
-    }
-    if (ng < ngroups) {
-        float4 *up = FACT ? nullptr : reinterpret_cast<float4 *>(a.prevBx + lane * (int64_t)N * P);
-#pragma unroll 2
+        for (int k = 0; k < VEC; k++) Y[r][k] = 0.f;
+    if (streams) {
+#pragma unroll(NC ? 8 : 4)
         for (int n = ng; n < N; n += ngroups) {
-            const float4 hq = hp[n * PV + pv];
+            float v[NV], c[RT];
+            lds_row<NV>(Vs + n * NV, v);
+            lds_row<RT>(Cs + n * RT, c);
+            const float4 hq = *reinterpret_cast<const float4 *>(hs + n * P + pv * VEC);
             float hv[VEC] = {hq.x, hq.y, hq.z, hq.w}, uv[VEC], ut[VEC];
             if (!FACT) {
-                const float4 uq = up[n * PV + pv];
+                const float4 uq = *reinterpret_cast<const float4 *>(us + n * P + pv * VEC);
                 uv[0] = uq.x; uv[1] = uq.y; uv[2] = uq.z; uv[3] = uq.w;
             }
 #pragma unroll
             for (int k = 0; k < VEC; k++) {
-                ut[k] = 0.f;
-                if (FACT) uv[k] = 0.f;
-            }
+                if (FACT) {
+                    float acc = al * hv[k];
 #pragma unroll
-            for (int r = 0; r < RT; r++) {
-                const float bn = Bb[r * N + n], pn = FACT ? Pb[r * N + n] : 0.f;
+                    for (int s = 0; s < NV; s++) acc = fmaf(v[s], Z[s][k], acc);
+                    hv[k] = acc;
+                } else {
+                    float u = 0.f;
 #pragma unroll
-                for (int k = 0; k < VEC; k++) {
-                    ut[k] = fmaf(bn, WF ? W[r][k] : X[r < RX ? r : 0][k], ut[k]);
-                    if (FACT) uv[k] = fmaf(pn, WF ? W[r][k] : Xp[r < RX ? r : 0][k], uv[k]);
-                }
-            }
-            if (WF) {
-#pragma unroll
-                for (int k = 0; k < VEC; k++) {
-                    ut[k] *= xv[k];
-                    if (FACT) uv[k] *= xq[k];
+                    for (int r = 0; r < RT; r++) u = fmaf(v[r], Z[r][k], u);
+                    ut[k] = u;
+                    hv[k] = fmaf(ga, u, fmaf(be, uv[k], al * hv[k]));
                 }
             }
 #pragma unroll
-            for (int k = 0; k < VEC; k++) hv[k] = al * hv[k] + be * uv[k] + ga * ut[k];
+            for (int r = 0; r < RT; r++)
 #pragma unroll
-            for (int r = 0; r < RT; r++) {
-                const float cn = Cb[r * N + n];
-#pragma unroll
-                for (int k = 0; k < VEC; k++) Y[r][k] = fmaf(cn, hv[k], Y[r][k]);
-            }
-            hp[n * PV + pv] = make_float4(hv[0], hv[1], hv[2], hv[3]);
-            if (!FACT) up[n * PV + pv] = make_float4(ut[0], ut[1], ut[2], ut[3]);
+                for (int k = 0; k < VEC; k++) Y[r][k] = fmaf(c[r], hv[k], Y[r][k]);
+            hp[n * PV] = make_float4(hv[0], hv[1], hv[2], hv[3]);
+            if (!FACT) up[n * PV] = make_float4(ut[0], ut[1], ut[2], ut[3]);
         }
+    }
+
+    // y: sum the partials over the rows (warp shuffles first where a warp
+    // holds whole rows), weight each rank by W_y, add D x
+    if (PV < 32 && (PV & (PV - 1)) == 0) {
+        for (int o = PV; o < 32; o <<= 1)
+#pragma unroll
+            for (int r = 0; r < RT; r++)
+#pragma unroll
+                for (int k = 0; k < VEC; k++) Y[r][k] += __shfl_xor_sync(0xffffffffu, Y[r][k], o);
+        if (ln < PV)
+#pragma unroll
+            for (int r = 0; r < RT; r++)
+#pragma unroll
+                for (int k = 0; k < VEC; k++) ypart[(wid * RT + r) * P + pv * VEC + k] = Y[r][k];
+    } else if (streams) {
 #pragma unroll
         for (int r = 0; r < RT; r++)
 #pragma unroll
             for (int k = 0; k < VEC; k++) ypart[(ng * RT + r) * P + pv * VEC + k] = Y[r][k];
     }
     __syncthreads();
-    for (int p = tid; p < P; p += nt) {
-        float s = 0.f;
-        for (int r = 0; r < R; r++) {
-            float yr = 0.f;
-            for (int g = 0; g < ngroups; g++) yr += ypart[(g * RT + r) * P + p];
-            s += (a.Wy ? a.Wy[(h * R + r) * P + p] : 1.f) * yr;
+    const float Dh = a.D[h];
+    if (RT == 1 || R == 1) {
+        for (int p = tid; p < P; p += nt) {
+            float s = 0.f;
+            for (int g = 0; g < npart; g++) s += ypart[g * RT * P + p];
+            const float xn = ldf(x, lane * P + p);
+            stf(y, lane * P + p, (a.Wy ? a.Wy[h * P + p] : 1.f) * s + Dh * xn);
+            if (FACT) a.xprev[lane * P + p] = xn;
         }
-        const float xp_new = ldf(x, lane * P + p);
-        stf(y, lane * P + p, s + a.D[h] * xp_new);
-        if (FACT) a.xprev[lane * P + p] = xp_new;
+    } else {
+        for (int it = tid; it < R * P; it += nt) {
+            const int r = it / P, p = it % P;
+            float s = 0.f;
+            for (int g = 0; g < npart; g++) s += ypart[(g * RT + r) * P + p];
+            yr[it] = (a.Wy ? a.Wy[(h * R + r) * P + p] : 1.f) * s;
+        }
+        __syncthreads();
+        for (int p = tid; p < P; p += nt) {
+            float s = 0.f;
+            for (int r = 0; r < R; r++) s += yr[r * P + p];
+            const float xn = ldf(x, lane * P + p);
+            stf(y, lane * P + p, s + Dh * xn);
+            if (FACT) a.xprev[lane * P + p] = xn;
+        }
     }
+    for (int j = tid; j < K; j += nt) a.angle[lane * K + j] = phs[j];
     if (FACT)
-        for (int k = tid; k < R * N; k += nt) a.bprev[lane * R * N + k] = Bb[k];
+        for (int k = tid; k < R * N; k += nt) a.bprev[lane * R * N + k] = Bn[k];
+}
+
+template <typename T, int RT, bool FACT, int NC, int PC>
+static cudaError_t launch_decode_gen_k(const DecodeArgs &a, cudaStream_t s) {
+    // the lane's state is staged in shared memory: up to 64 KB (h) or 128 KB (h and
+    // prev_Bx) at dstate x headdim = 16384, past the 48 KB a launch gets by default
+    const size_t smem = sizeof(float) * DecodeGenPlan<RT, FACT>::smem_floats((int)a.N, (int)a.P, DEC_THREADS);
+    auto kern = k_decode_gen<T, RT, FACT, NC, PC>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)(a.Bt * a.H), DEC_THREADS, smem, s>>>(a);
+    count_launch();
+    return cudaGetLastError();
 }
 
 template <typename T, int RT>
 static cudaError_t launch_decode_gen_rt(const DecodeArgs &a, bool factored, cudaStream_t s) {
-    const int threads = 256;
-    const int ngroups = threads / (int)(a.P / 4);
-    const size_t smem = sizeof(float) * (3 * RT * a.N + 32 + a.N / 2 + (size_t)ngroups * RT * a.P);
-    // rank 8 at dstate 256 needs about 57 KB, past the 48 KB a launch gets by default
-    if (factored) {
-        cudaFuncSetAttribute(k_decode_gen<T, RT, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_decode_gen<T, RT, true><<<(unsigned)(a.Bt * a.H), threads, smem, s>>>(a);
-    } else {
-        cudaFuncSetAttribute(k_decode_gen<T, RT, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_decode_gen<T, RT, false><<<(unsigned)(a.Bt * a.H), threads, smem, s>>>(a);
-    }
-    count_launch();
-    return cudaGetLastError();
+    // dstate 128 x headdim 64 (the pages' layer shapes) compiled as constants
+    if constexpr (RT <= 4)
+        if (a.N == 128 && a.P == 64)
+            return factored ? launch_decode_gen_k<T, RT, true, 128, 64>(a, s)
+                            : launch_decode_gen_k<T, RT, false, 128, 64>(a, s);
+    return factored ? launch_decode_gen_k<T, RT, true, 0, 0>(a, s) : launch_decode_gen_k<T, RT, false, 0, 0>(a, s);
 }
 
 template <typename T>
