@@ -20,6 +20,11 @@ template <> struct vecf<4> {
     }
     static __device__ __forceinline__ float4 pack(const float *o) { return make_float4(o[0], o[1], o[2], o[3]); }
 };
+template <> struct vecf<2> {
+    using type = float2;
+    static __device__ __forceinline__ void unpack(const float2 &v, float *o) { o[0] = v.x; o[1] = v.y; }
+    static __device__ __forceinline__ float2 pack(const float *o) { return make_float2(o[0], o[1]); }
+};
 template <> struct vecf<1> {
     using type = float;
     static __device__ __forceinline__ void unpack(const float &v, float *o) { o[0] = v; }
@@ -206,9 +211,13 @@ template <int RT, bool FACT>
 struct DecodeGenPlan {
     static constexpr int NV = FACT ? 2 * RT : RT;   // update terms per element
     static constexpr int NS = FACT ? 1 : 2;         // N x P states copied in (h, prev_Bx)
+    // columns per thread: 2 for the factored form at rank >= 4, whose column
+    // factors (2R x VEC) and y sums (R x VEC) would otherwise hold too many
+    // registers for four CTAs per SM
+    static constexpr int VEC = (FACT && RT >= 4) ? 2 : 4;
     // y partial sums: one per warp when the lanes of a column share a warp
     static __host__ __device__ int parts(int P, int nt) {
-        const int PV = P / 4;
+        const int PV = P / VEC;
         return (PV < 32 && (PV & (PV - 1)) == 0) ? nt / 32 : nt / PV;
     }
     static __host__ __device__ size_t smem_floats(int N, int P, int nt) {
@@ -221,9 +230,11 @@ struct DecodeGenPlan {
 // arguments), so that the row loops unroll fully and the indexing folds.
 constexpr int DEC_THREADS = 256;
 template <typename T, int RT, bool FACT, int NC, int PC>
-__global__ void __launch_bounds__(DEC_THREADS, RT == 1 ? 4 : (RT >= 8 ? 1 : (NC ? 3 : 2))) k_decode_gen(DecodeArgs a) {
+__global__ void __launch_bounds__(DEC_THREADS, RT == 1 ? 5 : (RT >= 8 ? 1 : (NC ? (FACT && RT >= 4 ? 4 : 3) : 2)))
+    k_decode_gen(DecodeArgs a) {
     using PL = DecodeGenPlan<RT, FACT>;
-    constexpr int VEC = 4, NV = PL::NV, nt = DEC_THREADS;
+    constexpr int VEC = PL::VEC, NV = PL::NV, nt = DEC_THREADS;
+    using V = typename vecf<VEC>::type;
     const int64_t lane = blockIdx.x, h = lane % a.H;
     const int P = PC ? PC : (int)a.P, N = NC ? NC : (int)a.N, NP2 = N / 2, R = (int)a.R, K = (int)a.K;
     const int tid = threadIdx.x, wid = tid >> 5, ln = tid & 31;
@@ -248,14 +259,17 @@ __global__ void __launch_bounds__(DEC_THREADS, RT == 1 ? 4 : (RT >= 8 ? 1 : (NC 
     const int ngroups = nt / PV;         // rows streamed concurrently
     const int pv = tid % PV, ng = tid / PV;
     const bool streams = ng < ngroups;
-    float4 *hp = reinterpret_cast<float4 *>(a.h + lane * (int64_t)N * P) + pv;
-    float4 *up = FACT ? hp : reinterpret_cast<float4 *>(a.prevBx + lane * (int64_t)N * P) + pv;
+    V *hp = reinterpret_cast<V *>(a.h + lane * (int64_t)N * P) + pv;
+    V *up = FACT ? hp : reinterpret_cast<V *>(a.prevBx + lane * (int64_t)N * P) + pv;
     float *us = hs + (FACT ? 0 : N * P);
-    if (streams) {
+    {   // the lane's state, 16 bytes per copy, consecutive threads on consecutive bytes
+        const float4 *hsrc = reinterpret_cast<const float4 *>(a.h + lane * (int64_t)N * P);
+        const float4 *usrc = reinterpret_cast<const float4 *>(a.prevBx + lane * (int64_t)N * P);
+        const int nv4 = N * P / 4;
 #pragma unroll(NC ? 8 : 4)
-        for (int n = ng; n < N; n += ngroups) {
-            cp_async16(hs + n * P + pv * VEC, hp + n * PV);
-            if (!FACT) cp_async16(us + n * P + pv * VEC, up + n * PV);
+        for (int o = tid; o < nv4; o += nt) {
+            cp_async16(hs + 4 * o, hsrc + o);
+            if (!FACT) cp_async16(us + 4 * o, usrc + o);
         }
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
@@ -365,8 +379,8 @@ __global__ void __launch_bounds__(DEC_THREADS, RT == 1 ? 4 : (RT >= 8 ? 1 : (NC 
             Vs[(2 * j + 1) * NV + r] = b1;
         }
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");   // this thread's rows (it reads only those)
-    __syncthreads();
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();   // every thread's copies have landed
 
     float Y[RT][VEC];
 #pragma unroll
@@ -379,12 +393,9 @@ __global__ void __launch_bounds__(DEC_THREADS, RT == 1 ? 4 : (RT >= 8 ? 1 : (NC 
             float v[NV], c[RT];
             lds_row<NV>(Vs + n * NV, v);
             lds_row<RT>(Cs + n * RT, c);
-            const float4 hq = *reinterpret_cast<const float4 *>(hs + n * P + pv * VEC);
-            float hv[VEC] = {hq.x, hq.y, hq.z, hq.w}, uv[VEC], ut[VEC];
-            if (!FACT) {
-                const float4 uq = *reinterpret_cast<const float4 *>(us + n * P + pv * VEC);
-                uv[0] = uq.x; uv[1] = uq.y; uv[2] = uq.z; uv[3] = uq.w;
-            }
+            float hv[VEC], uv[VEC], ut[VEC];
+            vecf<VEC>::unpack(*reinterpret_cast<const V *>(hs + n * P + pv * VEC), hv);
+            if (!FACT) vecf<VEC>::unpack(*reinterpret_cast<const V *>(us + n * P + pv * VEC), uv);
 #pragma unroll
             for (int k = 0; k < VEC; k++) {
                 if (FACT) {
@@ -404,8 +415,8 @@ __global__ void __launch_bounds__(DEC_THREADS, RT == 1 ? 4 : (RT >= 8 ? 1 : (NC 
             for (int r = 0; r < RT; r++)
 #pragma unroll
                 for (int k = 0; k < VEC; k++) Y[r][k] = fmaf(c[r], hv[k], Y[r][k]);
-            hp[n * PV] = make_float4(hv[0], hv[1], hv[2], hv[3]);
-            if (!FACT) up[n * PV] = make_float4(ut[0], ut[1], ut[2], ut[3]);
+            hp[n * PV] = vecf<VEC>::pack(hv);
+            if (!FACT) up[n * PV] = vecf<VEC>::pack(ut);
         }
     }
 
