@@ -220,9 +220,14 @@ struct DecodeGenPlan {
         const int PV = P / VEC;
         return (PV < 32 && (PV & (PV - 1)) == 0) ? nt / 32 : nt / PV;
     }
+    // the y partial sums (and the rank sums) reuse the staged state once the
+    // update has read it, when they fit there
+    static __host__ __device__ bool y_in_state(int N, int P, int nt) {
+        return (size_t)(parts(P, nt) + 1) * RT * P <= (size_t)N * P;
+    }
     static __host__ __device__ size_t smem_floats(int N, int P, int nt) {
         return (size_t)NS * N * P + (size_t)NV * N + 2 * (size_t)RT * N + N / 2 + 16 * RT +
-               (size_t)(parts(P, nt) + 1) * RT * P;
+               (y_in_state(N, P, nt) ? 0 : (size_t)(parts(P, nt) + 1) * RT * P);
     }
 };
 
@@ -230,7 +235,7 @@ struct DecodeGenPlan {
 // arguments), so that the row loops unroll fully and the indexing folds.
 constexpr int DEC_THREADS = 256;
 template <typename T, int RT, bool FACT, int NC, int PC>
-__global__ void __launch_bounds__(DEC_THREADS, RT == 1 ? 5 : (RT >= 8 ? 1 : (NC ? (FACT && RT >= 4 ? 4 : 3) : 2)))
+__global__ void __launch_bounds__(DEC_THREADS, RT == 1 ? (NC ? 6 : 4) : (RT >= 8 ? 1 : (NC ? (RT >= 4 ? (FACT ? 5 : 2) : 3) : 2)))
     k_decode_gen(DecodeArgs a) {
     using PL = DecodeGenPlan<RT, FACT>;
     constexpr int VEC = PL::VEC, NV = PL::NV, nt = DEC_THREADS;
@@ -252,7 +257,8 @@ __global__ void __launch_bounds__(DEC_THREADS, RT == 1 ? 5 : (RT >= 8 ? 1 : (NC 
     float *phs = Bn + RT * N;                     // N/2     angles of this token
     float *red = phs + N / 2;                     // 16 RT   norm partial sums
     const int npart = PL::parts(P, nt);
-    float *ypart = red + 16 * RT;                 // npart x RT x P
+    const bool y_in_hs = PL::y_in_state(N, P, nt);
+    float *ypart = y_in_hs ? hs : red + 16 * RT;  // npart x RT x P
     float *yr = ypart + npart * RT * P;           // RT x P
 
     const int PV = P / VEC;              // vectors per state row
@@ -422,6 +428,7 @@ __global__ void __launch_bounds__(DEC_THREADS, RT == 1 ? 5 : (RT >= 8 ? 1 : (NC 
 
     // y: sum the partials over the rows (warp shuffles first where a warp
     // holds whole rows), weight each rank by W_y, add D x
+    if (y_in_hs) __syncthreads();   // every thread has read its rows of the staged state
     if (PV < 32 && (PV & (PV - 1)) == 0) {
         for (int o = PV; o < 32; o <<= 1)
 #pragma unroll
