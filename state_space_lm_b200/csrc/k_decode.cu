@@ -172,16 +172,20 @@ cudaError_t launch_decode(const DecodeArgs &a, m3_dtype dt, cudaStream_t s) {
 //   y = sum_r W_y[r] (Cbar_r^T h) + D x_t
 //   prev_Bx <- U_t   or   b_prev <- Bbar, x_prev <- x_t      (factored)
 // One CTA per (b, h) lane; rank bound RT (R <= RT, the ranks past R are zero
-// rows); threads stream 4-wide rows of h (and prev_Bx).  The factored form
-// reads and writes only h, so a step moves about half the bytes of the full
-// form.  Its update of an (n, p) element is one sum of 2R products,
+// rows).  The factored form reads and writes only h, so a step moves about
+// half the bytes of the full form.  Its update of an (n, p) element is one
+// sum of 2R products,
 //   h' = alpha h + sum_r (beta b_prev_r[n]) (W_x[r][p] x_prev[p])
 //                      + (gamma Bbar_r[n]) (W_x[r][p] x[p]),
 // the row factors in shared memory ([n][term], read as 16-byte vectors) and
-// the column factors in registers.  Each thread's first NB rows of h (and
-// prev_Bx) are loaded before anything else, so their HBM latency overlaps the
-// rotation of B and C; the y partial sums meet in warp shuffles and one
-// shared-memory pass over the warps.
+// the column factors in registers; each thread owns VEC columns of every
+// ngroups-th row.  At entry the CTA starts 16-byte cp.async copies of the
+// lane's whole h (and prev_Bx) into shared memory, so the state is in flight
+// while B and C are rotated and the copies hold no registers.  The kernel is
+// bound by latency, so occupancy decides its speed: the y partial sums meet
+// in warp shuffles and then in the staged state's space once the update has
+// read it, and the factored form at rank >= 4 takes two columns per thread
+// (the register arrays halve).
 // ---------------------------------------------------------------------------
 template <int M>
 __device__ __forceinline__ void lds_row(const float *p, float (&o)[M]) {
