@@ -147,7 +147,9 @@ def test_mimo_fp32_grouped_partial():
 # ----------------------------------------------------------------------------
 @pytest.mark.parametrize("form,R,G,K,dtype", [("siso", 1, 2, 32, "bf16"), ("siso", 1, 1, 3, "f32"),
                                               ("mimo", 2, 1, 16, "bf16"), ("mimo", 4, 3, 5, "f32"),
+                                              ("mimo", 4, 2, 64, "bf16"),
                                               ("factored", 1, 2, 32, "bf16"), ("factored", 4, 1, 32, "bf16"),
+                                              ("factored", 2, 3, 64, "bf16"), ("factored", 3, 1, 16, "bf16"),
                                               ("factored", 3, 3, 2, "f32")])
 def test_decode_grouped_partial(form, R, G, K, dtype):
     Bt, T0, H, P, N, steps = 3, 20, 6, 8, 16, 6
